@@ -1,0 +1,31 @@
+"""CPU oracle of the streaming KV-cache Compressor.
+
+TEST INFRASTRUCTURE ONLY. Only the tests, the smoke check and the benchmark's
+CPU-baseline leg may import this package. The CUDA library neither imports nor
+links it, and the two share no code; both take their inputs from the seeded
+generators in ``workloads``.
+
+* ``oracle.compressor`` — the definition in float64 (numpy), step by step.
+* ``oracle.brute`` — a pure-Python restatement from the closed-form formula,
+  for tiny inputs, used to pin the former.
+
+Parity status: pinned. No page prints a numeric example of this operator, so
+the pins are brute force on tiny inputs, closed forms (equal scores give the
+window mean, one dominant score selects its row, masked first window, RMSNorm
+unit rms, RoPE identity and pair norms, Hadamard orthogonality) and the
+streaming invariants (token by token, chunked and reordered calls equal one
+call). See tests/test_oracle_pins.py.
+"""
+
+from . import brute, compressor  # noqa: F401
+from .compressor import (  # noqa: F401
+    Layout,
+    Result,
+    bf16_to_f64,
+    coff_of,
+    f64_to_bf16_bits,
+    layout,
+    out_rows,
+    run_inputs,
+    window_row_positions,
+)
