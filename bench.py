@@ -1,0 +1,470 @@
+#!/usr/bin/env python
+"""Benchmark of the streaming KV-cache Compressor on B200.
+
+One step = one Compressor call over one batch: the C128A 128K prefill (one
+sequence of 131072 tokens, H=4096, D=512, ratio 128, block_size 128), which is
+the workload of the headline metric (128K-prefill tokens/s). Inputs are seeded
+synthetic tensors of that shape, resident in HBM; x alone (1 GiB) is larger
+than the 126 MB L2, so no flush is needed between prefill steps.
+
+Also reported on the same line:
+  * e2e: the same metric through the public call with host buffers: every step
+    copies x, cu_seqlens, start_pos, the block tables and sin/cos from pinned
+    host memory and reads the output back;
+  * decode: the C4A 32-request decode step (one token each), microseconds per
+    call, with L2 flushed before every timed call;
+  * roofline: the projection kernel's tensor throughput against the measured
+    bf16 peak, and the decode call's HBM throughput against measured bandwidth;
+  * cpu_baseline: the CPU oracle on a bounded sample of the same workload.
+
+Multi-GPU (torchrun): every rank runs its own replica on its own GPU (requests
+are independent; no data-path collective), the time is the max over ranks and
+value counts the tokens of all ranks ("scaling": "weak").
+
+--impl reference times the CPU oracle (the only reference implementation this
+method has) on the same workload; rank 0 alone prints its line.
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "128K-prefill tokens/s"
+PREFILL = dict(name="c128a_128k", B=1, T=131072, H=4096, D=512, ratio=128, block_size=128)
+DECODE_ALG_BYTES = None  # computed from the decode workload
+
+
+# ----------------------------------------------------------------------------
+# distributed plumbing
+# ----------------------------------------------------------------------------
+
+def dist_setup():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if ws > 1:
+        import datetime
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    return ws, rank, local
+
+
+def barrier(ws):
+    if ws > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(v: float, ws: int) -> float:
+    if ws == 1:
+        return v
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ----------------------------------------------------------------------------
+# clocks during the timed region
+# ----------------------------------------------------------------------------
+
+class ClockSampler:
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.samples = []
+        self.proc = None
+        self.dev = device_index
+
+    def __enter__(self):
+        try:
+            import torch
+            uuid = str(torch.cuda.get_device_properties(self.dev).uuid)
+            sel = ["-i", uuid if uuid.startswith("GPU-") else "GPU-" + uuid]
+        except Exception:  # noqa: BLE001
+            sel = []
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", *sel, f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "50"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except OSError:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) == 7:
+                self.samples.append(parts)
+
+    def __exit__(self, *a):
+        if self.proc:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        num = lambda v: float(v) if v.replace(".", "", 1).isdigit() else None
+        sm = [num(s[0]) for s in self.samples if num(s[0]) is not None]
+        mx = [num(s[1]) for s in self.samples if num(s[1]) is not None]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for s in self.samples for i in range(4)
+                          if s[3 + i].lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
+                "samples": len(self.samples)}
+
+
+# ----------------------------------------------------------------------------
+# workloads on the device
+# ----------------------------------------------------------------------------
+
+def prefill_inputs(device, seed: int):
+    """The C128A 128K prefill, drawn on the device with a seeded generator:
+    x ~ N(0,1); wkv, wgate ~ N(0, 1/H); ape ~ N(0, 0.1); norm_weight ~ 1 + N(0, 0.05);
+    states ~ N(0,1); block table = a random permutation of the 1024 pool rows."""
+    import numpy as np
+    import torch
+
+    import streaming_kv_cache_varlen_b200 as cmp
+    from workloads import rope_tables
+
+    c = PREFILL
+    T, H, D, r, bs = c["T"], c["H"], c["D"], c["ratio"], c["block_size"]
+    C = D
+    g = torch.Generator(device=device)
+    g.manual_seed(seed)
+    bf = torch.bfloat16
+    x = torch.randn(T, H, generator=g, device=device).to(bf)
+    wkv = (torch.randn(C, H, generator=g, device=device) / H ** 0.5).to(bf)
+    wgate = (torch.randn(C, H, generator=g, device=device) / H ** 0.5).to(bf)
+    ape = torch.randn(r, C, generator=g, device=device) * 0.1 ** 0.5
+    norm_w = (1 + torch.randn(D, generator=g, device=device) * 0.05 ** 0.5).to(bf)
+    nblk = T // bs
+    kv_state = torch.randn(nblk, bs, C, generator=g, device=device)
+    score_state = torch.randn(nblk, bs, C, generator=g, device=device)
+    perm = torch.randperm(nblk, generator=g, device=device).to(torch.int32).view(1, nblk)
+    cu = torch.tensor([0, T], dtype=torch.int32, device=device)
+    sp = torch.zeros(1, dtype=torch.int32, device=device)
+    # sin / cos per output row from the library's own row layout (window w at w*ratio)
+    rs, rw = cmp.out_row_layout(np.array([0, T], np.int32), np.array([0], np.int32), r)
+    cos, sin = rope_tables(np.where(rw >= 0, rw * r, 0), 64)
+    cos_t = torch.from_numpy(cos.view(np.int16)).to(device).view(bf)
+    sin_t = torch.from_numpy(sin.view(np.int16)).to(device).view(bf)
+    return dict(x=x, kv_state=kv_state, score_state=score_state, kv_block_table=perm,
+                state_block_table=perm.clone(), sin=sin_t, cos=cos_t, wkv=wkv, wgate=wgate,
+                ape=ape, norm_weight=norm_w, hadamard=None, start_pos=sp, cu_seqlens=cu,
+                ratio=r, rope_head_dim=64, rotate=False)
+
+
+def decode_inputs(device):
+    import numpy as np
+    import torch
+
+    import streaming_kv_cache_varlen_b200 as cmp
+    from workloads import make_config, rope_tables
+
+    inp = make_config("c4a_decode")
+    rs, rw = cmp.out_row_layout(inp.cu_seqlens, inp.start_pos, inp.ratio)
+    cos, sin = rope_tables(np.where(rw >= 0, rw * inp.ratio, 0), 64)
+    inp = inp.__class__(**{**inp.__dict__, "cos": cos, "sin": sin})
+
+    def bfd(a):
+        return None if a is None else torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).to(device).view(torch.bfloat16)
+
+    def d(a):
+        return torch.from_numpy(np.ascontiguousarray(a)).to(device)
+
+    args = dict(x=bfd(inp.x), kv_state=d(inp.kv_state), score_state=d(inp.score_state),
+                kv_block_table=d(inp.kv_block_table), state_block_table=d(inp.state_block_table),
+                sin=bfd(inp.sin), cos=bfd(inp.cos), wkv=bfd(inp.wkv), wgate=bfd(inp.wgate),
+                ape=d(inp.ape), norm_weight=bfd(inp.norm_weight), hadamard=None,
+                start_pos=d(inp.start_pos), cu_seqlens=d(inp.cu_seqlens), ratio=inp.ratio,
+                rope_head_dim=64, rotate=False)
+    # algorithmic bytes of one decode call: both weight matrices, x, the earlier
+    # state rows the completed windows pool (coff*ratio - 1 half rows of D floats,
+    # kv and score), the state rows written (every token, kv and score), the ape
+    # rows, the output rows and the sin/cos rows of the windows, norm_weight
+    C, H, D = inp.C, inp.H, inp.D
+    n_win = int((((inp.start_pos + 1) % inp.ratio) == 0).sum())
+    hist_half_rows = n_win * (inp.coff * inp.ratio - 1)
+    alg = (2 * C * H * 2 + inp.T * H * 2 + hist_half_rows * D * 4 * 2 + inp.T * C * 4 * 2
+           + inp.ratio * C * 4 + inp.B * D * 2 + n_win * 64 * 2 * 2 + D * 2)
+    return args, alg, inp
+
+
+# ----------------------------------------------------------------------------
+# measurement
+# ----------------------------------------------------------------------------
+
+def read_peaks():
+    try:
+        p = json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json")))
+        return p, "measured"
+    except OSError:
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
+
+
+def traffic_for(kernel_file: str, kernel: str, units_scale: float = 1.0):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken on the
+    kernel source as it is now (else None)."""
+    try:
+        t = json.load(open(os.path.join(ROOT, "profiles", "traffic.json")))
+    except OSError:
+        return None
+    e = t.get(kernel)
+    if not e:
+        return None
+    src = os.path.join(ROOT, "streaming_kv_cache_varlen_b200", "csrc", kernel_file)
+    sha = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+    if e.get("source_sha") != sha:
+        return None
+    return e["bytes_per_launch"] * units_scale
+
+
+def run_ours(args):
+    import torch
+
+    import streaming_kv_cache_varlen_b200 as cmp
+
+    ws, rank, local = dist_setup()
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    stream = torch.cuda.current_stream(device)
+    peaks, peak_src = read_peaks()
+
+    # ---------------- prefill: device-resident inputs ----------------
+    pf = prefill_inputs(device, seed=1234 + rank)
+    out = torch.empty((cmp.out_rows(1, PREFILL["T"], PREFILL["ratio"]), PREFILL["D"]),
+                      dtype=torch.bfloat16, device=device)
+    for _ in range(args.warmup):
+        cmp.compressor(**pf, out=out)
+    torch.cuda.synchronize()
+    assert cmp.get_error() == 0
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    launches0 = cmp.launch_count()
+    with ClockSampler(local) as clk:
+        barrier(ws)
+        torch.cuda.synchronize()
+        cmp.profile_start()
+        e0.record(stream)
+        for _ in range(args.steps):
+            cmp.compressor(**pf, out=out)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        prof = cmp.profile_stop()
+        barrier(ws)
+    launches = cmp.launch_count() - launches0
+    assert cmp.get_error() == 0
+    ms = max_over_ranks(e0.elapsed_time(e1), ws)
+    ms_step = ms / args.steps
+    tokens = PREFILL["T"] * ws * args.steps
+    value = tokens / (ms / 1e3)
+
+    # dominant kernel: the projection (a dense bf16 contraction)
+    proj_name = max(("proj_tcgen05", "proj_mma_sync", "proj_decode"), key=lambda k: prof[k][0])
+    p_ms, p_n = prof[proj_name]
+    T, H, C = PREFILL["T"], PREFILL["H"], PREFILL["D"]
+    flops = 2.0 * T * H * 2 * C
+    achieved = flops / (p_ms / p_n / 1e3) / 1e12 if p_n else None
+    peak = peaks["bf16_tflops"]
+    kfile = {"proj_tcgen05": "cmp_proj_tc.cu", "proj_mma_sync": "cmp_proj_mma.cu",
+             "proj_decode": "cmp_proj_decode.cu"}[proj_name]
+    roofline = {"kernel": proj_name, "bound": "tensor", "achieved": achieved, "peak": peak,
+                "unit": "TFLOP/s", "frac": achieved / peak if achieved else None,
+                "traffic": traffic_for(kfile, proj_name), "peak_source": peak_src + " (burst)",
+                "algorithmic_flops_per_launch": flops,
+                "kernel_ms": {k: (v[0] / v[1] if v[1] else None) for k, v in prof.items()}}
+
+    # ---------------- e2e: host buffers, copies inside the timed region ----------------
+    host_names = ("x", "cu_seqlens", "start_pos", "kv_block_table", "state_block_table", "sin", "cos")
+    host = {k: pf[k].cpu().pin_memory() for k in host_names}
+    out_host = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    dev_in = {k: torch.empty_like(pf[k]) for k in host_names}
+    h2d = sum(v.numel() * v.element_size() for v in host.values())
+    d2h = out.numel() * out.element_size()
+    e2e_steps = max(1, min(args.steps, 20))
+    call = dict(pf)
+
+    def e2e_step():
+        for k in host_names:
+            dev_in[k].copy_(host[k], non_blocking=True)
+            call[k] = dev_in[k]
+        cmp.compressor(**call, out=out)
+        out_host.copy_(out, non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
+    torch.cuda.synchronize()
+    barrier(ws)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), ws)
+    e2e_value = PREFILL["T"] * ws * e2e_steps / (e2e_ms / 1e3)
+    del host, dev_in, call
+    del pf
+    torch.cuda.empty_cache()
+
+    # ---------------- decode: microseconds per call, L2 flushed ----------------
+    dec, dec_bytes, dec_inp = decode_inputs(device)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=device)
+    dout = torch.empty((cmp.out_rows(dec_inp.B, dec_inp.T, dec_inp.ratio), dec_inp.D),
+                       dtype=torch.bfloat16, device=device)
+    for _ in range(max(3, args.warmup)):
+        cmp.compressor(**dec, out=dout)
+    torch.cuda.synchronize()
+    n_dec = max(20, min(200, args.steps))
+    times = []
+    cmp.profile_start()
+    for _ in range(n_dec):
+        flush.fill_(1)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        cmp.compressor(**dec, out=dout)
+        b.record(stream)
+        times.append((a, b))
+    torch.cuda.synchronize()
+    dprof = cmp.profile_stop()
+    assert cmp.get_error() == 0
+    us = sorted(a.elapsed_time(b) * 1e3 for a, b in times)
+    dec_us = statistics.median(us)
+    dec_us = max_over_ranks(dec_us, ws)
+    decode = {"workload": "c4a_decode: 32 requests x 1 token, H=4096, D=512, ratio 4",
+              "us_per_call": dec_us, "us_per_call_min": us[0], "calls": n_dec,
+              "l2": "flushed (256 MB write) before every call",
+              "roofline": {"bound": "hbm", "achieved": dec_bytes / (dec_us / 1e6) / 1e9,
+                           "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                           "frac": dec_bytes / (dec_us / 1e6) / 1e9 / peaks["hbm_gbs"],
+                           "algorithmic_bytes_per_call": dec_bytes, "peak_source": peak_src},
+              "kernel_us": {k: (v[0] / v[1] * 1e3 if v[1] else None) for k, v in dprof.items()}}
+
+    # ---------------- CPU baseline: the oracle on a bounded sample ----------------
+    cpu = None
+    if rank == 0 and ws == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(args.cpu_tokens)
+
+    if rank == 0:
+        line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": ws,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+                "dtype": "bf16 in, fp32 accumulate / state, bf16 out", "data": "synthetic",
+                "config": {"workload": "c128a_128k: C128A prefill, 1 sequence x 131072 tokens, "
+                                       "H=4096, D=512, ratio=128, coff=1, block_size=128",
+                           "global_batch": ws, "seq_len": PREFILL["T"],
+                           "parallelism": f"dp{ws} (independent replicas)",
+                           "l2": "inputs larger than L2 (x is 1 GiB per step)"},
+                "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+                        "d2h_bytes_per_step": d2h, "steps": e2e_steps},
+                "gpu_launches": launches, "roofline": roofline, "decode": decode,
+                "clocks": clk.summary(), "cpu_baseline": cpu}
+        print(json.dumps(line), flush=True)
+    if ws > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+def cpu_baseline(tokens: int):
+    """The oracle, as it is, on the first ``tokens`` tokens of the prefill workload
+    (drawn on the host with the workload generator), on this host's cores."""
+    import numpy as np
+
+    from oracle import run_inputs, window_row_positions
+    from workloads import make_inputs
+
+    c = PREFILL
+    inp = make_inputs(name="cpu_sample", seed=2, lengths=[tokens], start_pos=[0], H=c["H"],
+                      D=c["D"], coff=1, ratio=c["ratio"], block_size=c["block_size"], rotate=False)
+    inp = inp.with_rope(window_row_positions(inp.cu_seqlens, inp.start_pos, c["ratio"]))
+    t0 = time.perf_counter()
+    run_inputs(inp)
+    dt = time.perf_counter() - t0
+    try:
+        from threadpoolctl import threadpool_info
+        cores = max(i.get("num_threads", 1) for i in threadpool_info())
+    except Exception:  # noqa: BLE001
+        cores = os.cpu_count()
+    return {"value": tokens / dt, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+            "sample": f"first {tokens} tokens ({tokens // c['ratio']} windows) of the 128K "
+                      f"prefill workload, float64 numpy oracle, {dt:.2f} s"}
+
+
+def run_reference(args):
+    """The CPU oracle as the reference arm: each step is the oracle on a bounded
+    sample of the prefill workload, sized so warm-up plus all steps take about
+    two minutes on this host."""
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    probe = cpu_baseline(512)
+    rate = probe["value"]  # tokens/s of the oracle on this host
+    per_step = int(rate * 120.0 / (args.steps + args.warmup))
+    per_step = max(PREFILL["ratio"], min(16384, per_step // PREFILL["ratio"] * PREFILL["ratio"]))
+    for _ in range(args.warmup):
+        cpu_baseline(per_step)
+    dts = []
+    for _ in range(args.steps):
+        r = cpu_baseline(per_step)
+        dts.append(per_step / r["value"])
+    total = sum(dts)
+    value = per_step * len(dts) / total
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+            "n_gpus": ws, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": total / len(dts) * 1e3, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": "c128a_128k: C128A prefill, 1 sequence x 131072 tokens, "
+                                   "H=4096, D=512, ratio=128, coff=1, block_size=128",
+                       "global_batch": 1, "seq_len": PREFILL["T"], "parallelism": "cpu",
+                       "sample_tokens_per_step": per_step},
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": r["cores"],
+                             "kind": "oracle", "sample": r["sample"]},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--cpu-tokens", type=int, default=8192)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,217 @@
+/*
+ * cmp.h — C ABI of the B200 streaming KV-cache Compressor.
+ *
+ * One call compresses every ratio-token window that the call completes into
+ * one bf16 row of D channels (DeepSeek-V4 C4A / C4Li / C128A attention):
+ *
+ *   1. dual projection   kv = x·Wkvᵀ,  score = x·Wgateᵀ + ape[p mod ratio]
+ *      ("compressor torch_extension API", 计算公式 1-2; "CANN PyPTO 算子实战:
+ *      Compressor", 主要计算过程);
+ *   2. per-window pooling: a per-channel softmax over the window's rows weights
+ *      a sum of its kv rows; for ratio 4 (coff 2) a window pairs columns [0, D)
+ *      of the previous window's 4 rows with columns [D, 2D) of its own 4 rows,
+ *      and the first window of a sequence has no previous rows
+ *      ("compressor torch_extension API", 计算公式 2-5; "NPU DeepSeek-V4 Ascend C
+ *      融合算子优化", Compressor 计算公式; "CANN PyPTO 算子实战", 压缩窗口与状态更新);
+ *   3. RMSNorm (eps 1e-6) with norm_weight, interleaved RoPE on the last
+ *      rope_head_dim channels, and, if rotate, a product with the D×D hadamard
+ *      matrix ("CANN PyPTO 算子实战", 压缩窗口与状态更新, kernel 派发逻辑).
+ *
+ * Streaming: kv_state / score_state keep, in fp32, the projected rows of
+ * windows a later call still has to pool. They are paged: position p of
+ * sequence b lives in slot (table[b][p / block_size], p % block_size) of its
+ * pool, with kv_block_table for kv_state and state_block_table for
+ * score_state ("CANN PyPTO 算子实战", 参数说明; "Triton-Ascend Compressor",
+ * state_block_table example). A call reads slots of positions before
+ * start_pos[b] and writes slots of positions from start_pos[b] on, so the
+ * slots it reads and the slots it writes are disjoint and an identical call
+ * repeated gives identical results.
+ *
+ * Conventions for every entry point below:
+ *  - bf16 tensors are passed as cmp_bf16 (their 16-bit patterns);
+ *  - all tensors are dense, row-major and contiguous;
+ *  - "device" pointers are CUDA device memory of the current device, owned by
+ *    the caller (the library never frees or keeps them past the call);
+ *  - "host" pointers are ordinary host memory;
+ *  - entry points returning int return a cmp_status.
+ */
+#ifndef CMP_H_
+#define CMP_H_
+
+#include <stdbool.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define CMP_API __attribute__((visibility("default")))
+#else
+#define CMP_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef uint16_t cmp_bf16;
+
+typedef enum cmp_status {
+  CMP_OK = 0,
+  CMP_ERR_NULLPTR = 1,      /* a required pointer is NULL */
+  CMP_ERR_INVALID = 2,      /* a size or argument outside the supported range */
+  CMP_ERR_UNSUPPORTED = 3,  /* a ratio the library does not implement */
+  CMP_ERR_CUDA = 4,         /* a CUDA runtime call or kernel launch failed */
+  CMP_ERR_DEVICE_INDEX = 5, /* a kernel met a bad index (see cmp_get_error) */
+  CMP_ERR_TIMEOUT = 6       /* a kernel gave up waiting on its own pipeline */
+} cmp_status;
+
+/* Shape scalars of one call; the pages' operator reads them from tensor shapes.
+ *   B            sequences (requests) in the call, >= 0
+ *   T            total tokens = rows of x = cu_seqlens[B], >= 0
+ *   H            hidden size: a multiple of 512 in [512, 16384]
+ *   D            compressed row width: 128 or 512
+ *   block_num    pool rows of kv_state and of score_state, >= 1
+ *   block_size   positions per pool row, in [1, 1024]
+ *   table_stride columns of kv_block_table and state_block_table, >= 1
+ * ("compressor torch_extension API", 约束说明: D in {128, 512}; H a multiple of
+ * 512; block_size 1..1024. H down to 512 is accepted for small tests.) */
+typedef struct cmp_dims {
+  int32_t B;
+  int32_t T;
+  int32_t H;
+  int32_t D;
+  int32_t block_num;
+  int32_t block_size;
+  int32_t table_stride;
+} cmp_dims;
+
+/* Rows of out, sin and cos: min(T, T / ratio + B)
+ * ("CANN PyPTO 算子实战", 返回值说明: out is [min(T, T//ratio + B), D]).
+ * Returns -1 if ratio < 1, B < 0 or T < 0. Host only. */
+CMP_API int64_t cmp_out_rows(int64_t B, int64_t T, int32_t ratio);
+
+/* Host-side output-row layout, for callers that build sin/cos per row.
+ * Window w of sequence b completes when the token at position (w+1)*ratio - 1
+ * arrives ("CANN PyPTO 算子实战", 数值精度与验证要点: (start_pos + i + 1) % ratio == 0).
+ * Sequence b reserves cap_b = min(L_b, L_b / ratio + 1) consecutive rows after
+ * those of sequences 0..b-1; its k-th completed window goes to the k-th of
+ * them. For every row n < n_out: row_seq[n] = b and row_window[n] = w if the
+ * row holds window w of sequence b, else row_seq[n] = row_window[n] = -1.
+ * cu_seqlens [B+1], start_pos [B] (NULL: all 0), row_seq / row_window
+ * [n_out]: host memory. n_out must equal cmp_out_rows(B, cu_seqlens[B], ratio).
+ * Errors: CMP_ERR_NULLPTR, CMP_ERR_INVALID (cu_seqlens not rising from 0,
+ * start_pos < 0, n_out mismatch, positions past INT32_MAX). */
+CMP_API int cmp_out_row_layout(const int32_t* cu_seqlens, const int32_t* start_pos, int32_t B,
+                       int32_t ratio, int64_t n_out, int32_t* row_seq, int32_t* row_window);
+
+/* The Compressor ("CANN PyPTO 算子实战", 函数原型 and 参数说明, plus cu_seqlens
+ * for packed variable-length input from "compressor torch_extension API").
+ *
+ *  x                  device bf16 [T, H]; sequence b owns rows
+ *                     cu_seqlens[b] .. cu_seqlens[b+1]-1, at absolute positions
+ *                     start_pos[b], start_pos[b]+1, ...
+ *  kv_state           device fp32 [block_num, block_size, coff*D], updated in place
+ *  score_state        device fp32 [block_num, block_size, coff*D], updated in place
+ *                     (holds x·Wgateᵀ + ape, as the pooling reads it)
+ *  kv_block_table     device int32 [B, table_stride]: pool row of kv_state per block
+ *  state_block_table  device int32 [B, table_stride]: pool row of score_state per block
+ *                     Entries a call does not need are never read (may be -1).
+ *  sin, cos           device bf16 [n_out, rope_head_dim]: RoPE tables of output
+ *                     row n; element 2j of a pair uses column j, element 2j+1
+ *                     column rope_head_dim/2 + j
+ *  wkv, wgate         device bf16 [coff*D, H]
+ *  ape                device fp32 [ratio, coff*D]: added to the score of the
+ *                     token at position p from row p mod ratio
+ *  norm_weight        device bf16 [D]
+ *  hadamard           device bf16 [D, D] (out = out @ hadamard); NULL iff !rotate
+ *  start_pos          device int32 [B]; NULL means every sequence starts at 0
+ *  cu_seqlens         device int32 [B+1], rising from 0 to T
+ *  ratio              tokens per window: 2, 4, 8, 16, 32, 64 or 128;
+ *                     coff = 2 for ratio 4, else 1
+ *  rope_head_dim      64 (the only value the pages support)
+ *  rotate             apply the hadamard product
+ *  out                device bf16 [n_out, D], n_out = cmp_out_rows(B, T, ratio);
+ *                     every row is written (rows with no window: 0)
+ *  stream             cudaStream_t to run on (NULL: the legacy default stream)
+ *  dims               host pointer to the shape scalars
+ *
+ * State update: for sequence b with e = start_pos[b] + L_b, the rows of
+ * positions p in [start_pos[b], e) with p >= (e/ratio - coff + 1)*ratio are
+ * written to both states — exactly the rows a later call can still read. No
+ * other state byte changes.
+ *
+ * Asynchronous on stream; no host synchronisation. The first call on a
+ * (device, stream) pair allocates a workspace that later calls reuse (it grows
+ * if a later call needs more); see cmp_workspace_size / cmp_release_workspaces.
+ * Results are bitwise reproducible run to run (no floating-point atomics).
+ * Requirements the library does not check: the pool rows used by different
+ * sequences are disjoint, and the tables map the blocks a call needs.
+ *
+ * Returns CMP_OK, CMP_ERR_NULLPTR, CMP_ERR_INVALID, CMP_ERR_UNSUPPORTED or
+ * CMP_ERR_CUDA, all decided on the host before anything is launched, except
+ * CMP_ERR_CUDA for a failed launch. B == 0 or T == 0 is a successful no-op.
+ * Faults found inside kernels (a needed table entry outside [0, block_num) or
+ * a block index past table_stride; cu_seqlens not rising from 0 to T;
+ * start_pos < 0; positions past INT32_MAX) never trap: the access is skipped,
+ * an error word on the device is set, and cmp_get_error reports it. */
+CMP_API int cmp_compressor(const cmp_bf16* x, float* kv_state, float* score_state,
+                   const int32_t* kv_block_table, const int32_t* state_block_table,
+                   const cmp_bf16* sin, const cmp_bf16* cos, const cmp_bf16* wkv,
+                   const cmp_bf16* wgate, const float* ape, const cmp_bf16* norm_weight,
+                   const cmp_bf16* hadamard, const int32_t* start_pos, const int32_t* cu_seqlens,
+                   int32_t ratio, int32_t rope_head_dim, bool rotate, cmp_bf16* out,
+                   void* stream, const cmp_dims* dims);
+
+/* Synchronises stream, then returns and clears the error word the kernels of
+ * the current device set: CMP_OK, CMP_ERR_DEVICE_INDEX or CMP_ERR_TIMEOUT
+ * (CMP_ERR_CUDA if the synchronisation itself fails). */
+CMP_API int cmp_get_error(void* stream);
+
+/* Bytes of device workspace a call with these shapes uses (the two-phase
+ * "query the workspace, then run" pattern of the aclnn API on "NsaCompressWithCache").
+ * Returns 0 for invalid dims. Host only. */
+CMP_API size_t cmp_workspace_size(const cmp_dims* dims, int32_t ratio);
+
+/* Frees every workspace the library holds (synchronises the devices first).
+ * Returns CMP_OK or CMP_ERR_CUDA. */
+CMP_API int cmp_release_workspaces(void);
+
+/* Static text for a status code. */
+CMP_API const char* cmp_status_string(int status);
+
+/* ---- measurement --------------------------------------------------------
+ * Kernels of the library, by id: */
+enum {
+  CMP_KERNEL_SCHED = 0,        /* varlen scheduler */
+  CMP_KERNEL_PROJ_TC = 1,      /* prefill projection, tcgen05 / TMEM / TMA */
+  CMP_KERNEL_PROJ_MMA = 2,     /* projection, warp-level mma.sync */
+  CMP_KERNEL_PROJ_DECODE = 3,  /* small-T projection streaming the weights */
+  CMP_KERNEL_POOL = 4,         /* pooling + RMSNorm + RoPE + Hadamard + store */
+  CMP_KERNEL_COUNT = 5
+};
+
+/* Name of a kernel id (NULL if out of range). */
+CMP_API const char* cmp_kernel_name(int kernel);
+
+/* Total kernels this library has launched in this process (all devices). */
+CMP_API int64_t cmp_launch_count(void);
+
+/* Start per-kernel timing: every launch from now on is bracketed by CUDA
+ * events on its stream. Clears earlier totals. Returns CMP_OK or CMP_ERR_CUDA. */
+CMP_API int cmp_profile_start(void);
+
+/* Stop timing; synchronise the recorded events and write, per kernel id, the
+ * summed milliseconds and launch count into ms[CMP_KERNEL_COUNT] and
+ * launches[CMP_KERNEL_COUNT] (host arrays; either may be NULL). */
+CMP_API int cmp_profile_stop(double* ms, int64_t* launches);
+
+/* Testing knob: which projection kernel prefill calls use. 0 = automatic
+ * (tcgen05 kernel for large T, weight-streaming kernel for small T), 1 = force
+ * the mma.sync kernel, 2 = force the tcgen05 kernel, 3 = force the
+ * weight-streaming kernel. Returns the previous value, or -1 if out of range. */
+CMP_API int cmp_set_proj_kernel(int which);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* CMP_H_ */

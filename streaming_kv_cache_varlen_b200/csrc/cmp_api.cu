@@ -1,0 +1,399 @@
+// Host side of the C ABI: argument checks, the per-(device, stream) workspace,
+// kernel launches, error reporting and per-kernel timing.
+#include <algorithm>
+#include <atomic>
+#include <climits>
+#include <map>
+#include <mutex>
+#include <utility>
+#include <vector>
+
+#include "cmp_internal.cuh"
+
+namespace cmp {
+cudaError_t launch_proj_tc(const Params& p, cudaStream_t s);
+cudaError_t launch_proj_decode(const Params& p, cudaStream_t s);
+bool proj_tc_supported(const Params& p);
+bool proj_decode_supported(const Params& p);
+size_t proj_decode_workspace(const Params& p);
+}  // namespace cmp
+
+namespace {
+
+using cmp::Params;
+
+// ---- workspace ---------------------------------------------------------------
+
+struct WsLayout {
+  size_t err, m_cu, m_s, m_off, proj, total;
+};
+
+WsLayout ws_layout(int64_t B, int64_t T, int64_t C) {
+  WsLayout L{};
+  size_t o = 0;
+  auto take = [&](size_t n) {
+    const size_t r = o;
+    o += (n + 255) & ~size_t(255);
+    return r;
+  };
+  L.err = take(16);
+  L.m_cu = take(sizeof(int32_t) * (B + 1));
+  L.m_s = take(sizeof(int32_t) * std::max<int64_t>(B, 1));
+  L.m_off = take(sizeof(int32_t) * (B + 1));
+  L.proj = take(sizeof(float) * (size_t)T * 2 * C);
+  L.total = o;
+  return L;
+}
+
+struct Workspace {
+  unsigned char* ptr = nullptr;
+  size_t bytes = 0;
+};
+
+std::mutex g_mu;
+std::map<std::pair<int, cudaStream_t>, Workspace> g_ws;
+std::map<std::pair<int, cudaStream_t>, unsigned> g_pending_err;  // kept across a regrow
+std::atomic<int64_t> g_launches{0};
+std::atomic<int> g_proj_kernel{0};
+
+// ---- profiling ---------------------------------------------------------------
+
+struct Timed {
+  cudaEvent_t a, b;
+  int kernel;
+};
+std::mutex g_prof_mu;
+bool g_prof = false;
+std::vector<Timed> g_timed;
+std::vector<cudaEvent_t> g_event_pool;
+
+cudaEvent_t take_event() {
+  if (!g_event_pool.empty()) {
+    cudaEvent_t e = g_event_pool.back();
+    g_event_pool.pop_back();
+    return e;
+  }
+  cudaEvent_t e = nullptr;
+  if (cudaEventCreate(&e) != cudaSuccess) return nullptr;
+  return e;
+}
+
+template <class F>
+cudaError_t launch(int kernel, cudaStream_t s, F&& f) {
+  Timed t{nullptr, nullptr, kernel};
+  bool prof = false;
+  {
+    std::lock_guard<std::mutex> lk(g_prof_mu);
+    if (g_prof) {
+      t.a = take_event();
+      t.b = take_event();
+      prof = t.a && t.b;
+    }
+  }
+  if (prof) cudaEventRecord(t.a, s);
+  const cudaError_t e = f();
+  if (prof) {
+    cudaEventRecord(t.b, s);
+    std::lock_guard<std::mutex> lk(g_prof_mu);
+    g_timed.push_back(t);
+  }
+  if (e == cudaSuccess) g_launches.fetch_add(1, std::memory_order_relaxed);
+  return e;
+}
+
+int get_workspace(cudaStream_t s, size_t need, unsigned char** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return CMP_ERR_CUDA;
+  std::lock_guard<std::mutex> lk(g_mu);
+  Workspace& w = g_ws[{dev, s}];
+  if (w.bytes >= need && w.ptr) {
+    *out = w.ptr;
+    return CMP_OK;
+  }
+  if (w.ptr) {
+    // keep an error word a pending call may still set: wait, read, carry over
+    if (cudaDeviceSynchronize() != cudaSuccess) return CMP_ERR_CUDA;
+    unsigned old = 0;
+    if (cudaMemcpy(&old, w.ptr, sizeof(old), cudaMemcpyDeviceToHost) != cudaSuccess) return CMP_ERR_CUDA;
+    g_pending_err[{dev, s}] |= old;
+    cudaFree(w.ptr);
+    w.ptr = nullptr;
+    w.bytes = 0;
+  }
+  const size_t bytes = std::max(need, size_t(1) << 20);
+  void* p = nullptr;
+  if (cudaMalloc(&p, bytes) != cudaSuccess) return CMP_ERR_CUDA;
+  if (cudaMemset(p, 0, 256) != cudaSuccess) {
+    cudaFree(p);
+    return CMP_ERR_CUDA;
+  }
+  w.ptr = static_cast<unsigned char*>(p);
+  w.bytes = bytes;
+  *out = w.ptr;
+  return CMP_OK;
+}
+
+bool valid_ratio(int r) {
+  return r == 2 || r == 4 || r == 8 || r == 16 || r == 32 || r == 64 || r == 128;
+}
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+int check_dims(const cmp_dims* d) {
+  if (!d) return CMP_ERR_NULLPTR;
+  if (d->B < 0 || d->T < 0) return CMP_ERR_INVALID;
+  if (d->D != 128 && d->D != 512) return CMP_ERR_INVALID;
+  if (d->H < 512 || d->H > 16384 || d->H % 512) return CMP_ERR_INVALID;
+  if (d->block_size < 1 || d->block_size > 1024) return CMP_ERR_INVALID;
+  if (d->block_num < 1 || d->table_stride < 1) return CMP_ERR_INVALID;
+  return CMP_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int64_t cmp_out_rows(int64_t B, int64_t T, int32_t ratio) {
+  if (ratio < 1 || B < 0 || T < 0) return -1;
+  return std::min<int64_t>(T, T / ratio + B);
+}
+
+int cmp_out_row_layout(const int32_t* cu_seqlens, const int32_t* start_pos, int32_t B, int32_t ratio,
+                       int64_t n_out, int32_t* row_seq, int32_t* row_window) {
+  if (!cu_seqlens || ((!row_seq || !row_window) && n_out > 0)) return CMP_ERR_NULLPTR;
+  if (B < 0 || ratio < 1) return CMP_ERR_INVALID;
+  if (cu_seqlens[0] != 0) return CMP_ERR_INVALID;
+  for (int b = 0; b < B; ++b) {
+    if (cu_seqlens[b + 1] < cu_seqlens[b]) return CMP_ERR_INVALID;
+    const int64_t s = start_pos ? start_pos[b] : 0;
+    if (s < 0 || s + (cu_seqlens[b + 1] - cu_seqlens[b]) > INT32_MAX) return CMP_ERR_INVALID;
+  }
+  if (n_out != cmp_out_rows(B, cu_seqlens[B], ratio)) return CMP_ERR_INVALID;
+  for (int64_t n = 0; n < n_out; ++n) row_seq[n] = row_window[n] = -1;
+  int64_t off = 0;
+  for (int b = 0; b < B; ++b) {
+    const int64_t L = cu_seqlens[b + 1] - cu_seqlens[b];
+    const int64_t s = start_pos ? start_pos[b] : 0;
+    const int64_t e = s + L;
+    const int64_t nw = e / ratio - s / ratio;
+    for (int64_t k = 0; k < nw; ++k) {
+      row_seq[off + k] = b;
+      row_window[off + k] = (int32_t)(s / ratio + k);
+    }
+    off += std::min<int64_t>(L, L / ratio + 1);
+  }
+  return CMP_OK;
+}
+
+size_t cmp_workspace_size(const cmp_dims* dims, int32_t ratio) {
+  if (check_dims(dims) != CMP_OK || !valid_ratio(ratio)) return 0;
+  const int coff = ratio == 4 ? 2 : 1;
+  size_t base = ws_layout(dims->B, dims->T, (int64_t)coff * dims->D).total;
+  Params p{};
+  p.B = dims->B;
+  p.T = dims->T;
+  p.H = dims->H;
+  p.D = dims->D;
+  p.C = coff * dims->D;
+  p.coff = coff;
+  p.ratio = ratio;
+  return base + cmp::proj_decode_workspace(p);
+}
+
+int cmp_release_workspaces(void) {
+  std::lock_guard<std::mutex> lk(g_mu);
+  int rc = CMP_OK;
+  int cur = 0;
+  cudaGetDevice(&cur);
+  for (auto& kv : g_ws) {
+    if (!kv.second.ptr) continue;
+    if (cudaSetDevice(kv.first.first) != cudaSuccess) { rc = CMP_ERR_CUDA; continue; }
+    cudaDeviceSynchronize();
+    if (cudaFree(kv.second.ptr) != cudaSuccess) rc = CMP_ERR_CUDA;
+  }
+  g_ws.clear();
+  cudaSetDevice(cur);
+  return rc;
+}
+
+int cmp_compressor(const cmp_bf16* x, float* kv_state, float* score_state,
+                   const int32_t* kv_block_table, const int32_t* state_block_table,
+                   const cmp_bf16* sin, const cmp_bf16* cos, const cmp_bf16* wkv,
+                   const cmp_bf16* wgate, const float* ape, const cmp_bf16* norm_weight,
+                   const cmp_bf16* hadamard, const int32_t* start_pos, const int32_t* cu_seqlens,
+                   int32_t ratio, int32_t rope_head_dim, bool rotate, cmp_bf16* out,
+                   void* stream, const cmp_dims* dims) {
+  // ---- host checks, nothing launched before they pass ----
+  if (!dims) return CMP_ERR_NULLPTR;
+  if (!valid_ratio(ratio)) return CMP_ERR_UNSUPPORTED;
+  int rc = check_dims(dims);
+  if (rc != CMP_OK) return rc;
+  if (rope_head_dim != 64 || rope_head_dim > dims->D) return CMP_ERR_INVALID;
+  if (dims->B == 0 && dims->T != 0) return CMP_ERR_INVALID;
+  if (dims->B == 0 || dims->T == 0) return CMP_OK;
+  if (!x || !kv_state || !score_state || !kv_block_table || !state_block_table || !sin || !cos ||
+      !wkv || !wgate || !ape || !norm_weight || !cu_seqlens || !out)
+    return CMP_ERR_NULLPTR;
+  if (rotate && !hadamard) return CMP_ERR_NULLPTR;
+  if (!aligned(x, 16) || !aligned(wkv, 16) || !aligned(wgate, 16) || !aligned(kv_state, 16) ||
+      !aligned(score_state, 16) || !aligned(ape, 16) || !aligned(out, 8) || !aligned(norm_weight, 8) ||
+      !aligned(sin, 4) || !aligned(cos, 4) || (rotate && !aligned(hadamard, 8)) ||
+      !aligned(kv_block_table, 4) || !aligned(state_block_table, 4) || !aligned(cu_seqlens, 4) ||
+      (start_pos && !aligned(start_pos, 4)))
+    return CMP_ERR_INVALID;
+
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int coff = ratio == 4 ? 2 : 1;
+  Params p{};
+  p.x = reinterpret_cast<const __nv_bfloat16*>(x);
+  p.kv_state = kv_state;
+  p.score_state = score_state;
+  p.kv_tbl = kv_block_table;
+  p.sc_tbl = state_block_table;
+  p.sin = reinterpret_cast<const __nv_bfloat16*>(sin);
+  p.cos = reinterpret_cast<const __nv_bfloat16*>(cos);
+  p.wkv = reinterpret_cast<const __nv_bfloat16*>(wkv);
+  p.wgate = reinterpret_cast<const __nv_bfloat16*>(wgate);
+  p.ape = ape;
+  p.norm_w = reinterpret_cast<const __nv_bfloat16*>(norm_weight);
+  p.had = rotate ? reinterpret_cast<const __nv_bfloat16*>(hadamard) : nullptr;
+  p.start_pos = start_pos;
+  p.cu_in = cu_seqlens;
+  p.out = reinterpret_cast<__nv_bfloat16*>(out);
+  p.B = dims->B;
+  p.T = dims->T;
+  p.H = dims->H;
+  p.D = dims->D;
+  p.C = coff * dims->D;
+  p.coff = coff;
+  p.ratio = ratio;
+  p.rope = rope_head_dim;
+  p.rotate = rotate ? 1 : 0;
+  p.block_num = dims->block_num;
+  p.bs = dims->block_size;
+  p.stride = dims->table_stride;
+  p.n_out = (int)cmp_out_rows(p.B, p.T, ratio);
+
+  const WsLayout L = ws_layout(p.B, p.T, p.C);
+  const size_t extra = cmp::proj_decode_workspace(p);
+  unsigned char* ws = nullptr;
+  rc = get_workspace(s, L.total + extra, &ws);
+  if (rc != CMP_OK) return rc;
+  p.err = reinterpret_cast<unsigned*>(ws + L.err);
+  p.m_cu = reinterpret_cast<int32_t*>(ws + L.m_cu);
+  p.m_s = reinterpret_cast<int32_t*>(ws + L.m_s);
+  p.m_off = reinterpret_cast<int32_t*>(ws + L.m_off);
+  p.proj = reinterpret_cast<float*>(ws + L.proj);
+
+  // ---- kernels ----
+  if (launch(CMP_KERNEL_SCHED, s, [&] { return cmp::launch_sched(p, s); }) != cudaSuccess)
+    return CMP_ERR_CUDA;
+  int which = g_proj_kernel.load();
+  if (which == 0) {
+    if (cmp::proj_decode_supported(p)) which = 3;
+    else if (cmp::proj_tc_supported(p)) which = 2;
+    else which = 1;
+  }
+  if (which == 2 && !cmp::proj_tc_supported(p)) which = 1;
+  if (which == 3 && !cmp::proj_decode_supported(p)) which = 1;
+  cudaError_t e;
+  if (which == 2)
+    e = launch(CMP_KERNEL_PROJ_TC, s, [&] { return cmp::launch_proj_tc(p, s); });
+  else if (which == 3)
+    e = launch(CMP_KERNEL_PROJ_DECODE, s, [&] { return cmp::launch_proj_decode(p, s); });
+  else
+    e = launch(CMP_KERNEL_PROJ_MMA, s, [&] { return cmp::launch_proj_mma(p, s); });
+  if (e != cudaSuccess) return CMP_ERR_CUDA;
+  if (launch(CMP_KERNEL_POOL, s, [&] { return cmp::launch_pool(p, s); }) != cudaSuccess)
+    return CMP_ERR_CUDA;
+  return CMP_OK;
+}
+
+int cmp_get_error(void* stream) {
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(s) != cudaSuccess) return CMP_ERR_CUDA;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return CMP_ERR_CUDA;
+  unsigned word = 0;
+  {
+    std::lock_guard<std::mutex> lk(g_mu);
+    auto pe = g_pending_err.find({dev, s});
+    if (pe != g_pending_err.end()) {
+      word |= pe->second;
+      pe->second = 0;
+    }
+    auto it = g_ws.find({dev, s});
+    if (it != g_ws.end() && it->second.ptr) {
+      unsigned v = 0;
+      if (cudaMemcpy(&v, it->second.ptr, sizeof(v), cudaMemcpyDeviceToHost) != cudaSuccess)
+        return CMP_ERR_CUDA;
+      if (v && cudaMemset(it->second.ptr, 0, sizeof(v)) != cudaSuccess) return CMP_ERR_CUDA;
+      word |= v;
+    }
+  }
+  if (word & cmp::kErrTimeout) return CMP_ERR_TIMEOUT;
+  if (word & cmp::kErrIndex) return CMP_ERR_DEVICE_INDEX;
+  return CMP_OK;
+}
+
+const char* cmp_status_string(int status) {
+  switch (status) {
+    case CMP_OK: return "ok";
+    case CMP_ERR_NULLPTR: return "a required pointer is NULL";
+    case CMP_ERR_INVALID: return "an argument or size is outside the supported range";
+    case CMP_ERR_UNSUPPORTED: return "unsupported ratio";
+    case CMP_ERR_CUDA: return "CUDA runtime error";
+    case CMP_ERR_DEVICE_INDEX: return "a kernel met an out-of-range index and skipped the access";
+    case CMP_ERR_TIMEOUT: return "a kernel gave up waiting on its pipeline";
+    default: return "unknown status";
+  }
+}
+
+const char* cmp_kernel_name(int kernel) {
+  static const char* names[CMP_KERNEL_COUNT] = {"sched", "proj_tcgen05", "proj_mma_sync",
+                                                "proj_decode", "pool_epilogue"};
+  return (kernel >= 0 && kernel < CMP_KERNEL_COUNT) ? names[kernel] : nullptr;
+}
+
+int64_t cmp_launch_count(void) { return g_launches.load(); }
+
+int cmp_profile_start(void) {
+  std::lock_guard<std::mutex> lk(g_prof_mu);
+  for (auto& t : g_timed) {
+    g_event_pool.push_back(t.a);
+    g_event_pool.push_back(t.b);
+  }
+  g_timed.clear();
+  g_prof = true;
+  return CMP_OK;
+}
+
+int cmp_profile_stop(double* ms, int64_t* launches) {
+  std::lock_guard<std::mutex> lk(g_prof_mu);
+  g_prof = false;
+  double acc[CMP_KERNEL_COUNT] = {0};
+  int64_t cnt[CMP_KERNEL_COUNT] = {0};
+  int rc = CMP_OK;
+  for (auto& t : g_timed) {
+    float v = 0.f;
+    if (cudaEventSynchronize(t.b) != cudaSuccess || cudaEventElapsedTime(&v, t.a, t.b) != cudaSuccess)
+      rc = CMP_ERR_CUDA;
+    acc[t.kernel] += v;
+    cnt[t.kernel] += 1;
+    g_event_pool.push_back(t.a);
+    g_event_pool.push_back(t.b);
+  }
+  g_timed.clear();
+  for (int k = 0; k < CMP_KERNEL_COUNT; ++k) {
+    if (ms) ms[k] = acc[k];
+    if (launches) launches[k] = cnt[k];
+  }
+  return rc;
+}
+
+int cmp_set_proj_kernel(int which) {
+  if (which < 0 || which > 3) return -1;
+  return g_proj_kernel.exchange(which);
+}
+
+}  // extern "C"

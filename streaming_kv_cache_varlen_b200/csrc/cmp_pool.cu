@@ -1,0 +1,158 @@
+// Pooling and epilogue: one CTA per output row, D/4 threads, each thread owns
+// four consecutive channels.
+//
+// For the window the row holds:
+//  * gather its rows: coff = 1: the ratio rows of the window; coff = 2: the
+//    ratio rows of the previous window, columns [0, D), then the ratio rows of
+//    the window, columns [D, 2D); the first window of a sequence has no
+//    previous rows ("compressor torch_extension API", 计算公式 2-4; "CANN PyPTO
+//    算子实战", 压缩窗口与状态更新: 0 and -inf fill the missing previous window).
+//    A row at a position inside this call comes from the projection buffer,
+//    an earlier one from the paged state;
+//  * per-channel softmax over those rows weighting a sum of the kv rows
+//    (计算公式 3-5), as an online (running max) softmax in fp32;
+//  * RMSNorm, eps 1e-6, times norm_weight; interleaved RoPE on the last
+//    rope_head_dim channels (pair (2j, 2j+1) uses table columns j and
+//    rope_head_dim/2 + j); optional product with the hadamard matrix
+//    ("CANN PyPTO 算子实战", 压缩窗口与状态更新, 算子级辅助函数, kernel 派发逻辑);
+//  * bf16 round-to-nearest-even store. Rows that hold no window are stored as 0
+//    ("CANN PyPTO 算子实战", 返回值说明).
+#include "cmp_internal.cuh"
+
+namespace cmp {
+namespace {
+
+constexpr float kRmsEps = 1e-6f;
+
+__device__ __forceinline__ float4 ld4(const float* p) { return *reinterpret_cast<const float4*>(p); }
+
+__device__ __forceinline__ void online(float& m, float& l, float& a, float z, float k) {
+  const float mn = fmaxf(m, z);
+  const float sc = __expf(m - mn);  // m = -inf on the first row: exp(-inf) = 0
+  const float pz = __expf(z - mn);
+  l = l * sc + pz;
+  a = a * sc + pz * k;
+  m = mn;
+}
+
+__global__ void __launch_bounds__(128) pool_kernel(Params p) {
+  __shared__ float red[32];
+  __shared__ float zs[512];
+  const int n = blockIdx.x;
+  const int D = p.D, C = p.C, r = p.ratio;
+  const int c = threadIdx.x * 4;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
+
+  const int b = upper_index(p.m_off, p.B, n);
+  int w = -1, s = 0, cu = 0;
+  if (b < p.B) {
+    s = p.m_s[b];
+    cu = p.m_cu[b];
+    const int e = s + (p.m_cu[b + 1] - cu);
+    const int k = n - p.m_off[b];
+    if (k < e / r - s / r) w = s / r + k;
+  }
+  uint2* dst = reinterpret_cast<uint2*>(p.out + (int64_t)n * D + c);
+  if (w < 0) {
+    *dst = make_uint2(0u, 0u);
+    return;
+  }
+
+  float m[4], l[4], a[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) { m[i] = -INFINITY; l[i] = 0.f; a[i] = 0.f; }
+  const int rows = p.coff * r;
+  for (int j = 0; j < rows; ++j) {
+    const bool bhalf = p.coff == 1 || j >= r;
+    const int q = p.coff == 1 ? w * r + j : (j < r ? (w - 1) * r + j : w * r + (j - r));
+    if (q < 0) continue;  // the first window has no previous window
+    const int col = (p.coff == 2 && bhalf) ? D + c : c;
+    float4 kv, sc;
+    if (q >= s) {
+      const float* row = p.proj + (int64_t)(cu + (q - s)) * (2 * C);
+      kv = ld4(row + col);
+      sc = ld4(row + C + col);
+    } else {
+      const int rk = table_row(p, p.kv_tbl, b, q);
+      const int rs = table_row(p, p.sc_tbl, b, q);
+      if (rk < 0 || rs < 0) continue;
+      kv = ld4(p.kv_state + ((int64_t)rk * p.bs + q % p.bs) * C + col);
+      sc = ld4(p.score_state + ((int64_t)rs * p.bs + q % p.bs) * C + col);
+    }
+    online(m[0], l[0], a[0], sc.x, kv.x);
+    online(m[1], l[1], a[1], sc.y, kv.y);
+    online(m[2], l[2], a[2], sc.z, kv.z);
+    online(m[3], l[3], a[3], sc.w, kv.w);
+  }
+  float y[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) y[i] = l[i] > 0.f ? a[i] / l[i] : 0.f;
+
+  // RMSNorm over the D channels of the row
+  float ss = y[0] * y[0] + y[1] * y[1] + y[2] * y[2] + y[3] * y[3];
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+  if (lane == 0) red[warp] = ss;
+  __syncthreads();
+  float tot = 0.f;
+  for (int i = 0; i < nwarps; ++i) tot += red[i];
+  const float inv = rsqrtf(tot / (float)D + kRmsEps);
+  const uint2 wraw = *reinterpret_cast<const uint2*>(p.norm_w + c);
+  const __nv_bfloat162 w01 = *reinterpret_cast<const __nv_bfloat162*>(&wraw.x);
+  const __nv_bfloat162 w23 = *reinterpret_cast<const __nv_bfloat162*>(&wraw.y);
+  float z[4] = {y[0] * inv * __low2float(w01), y[1] * inv * __high2float(w01),
+                y[2] * inv * __low2float(w23), y[3] * inv * __high2float(w23)};
+
+  // interleaved RoPE on the last rope channels
+  const int r0 = D - p.rope;
+  if (c >= r0) {
+    const int half = p.rope / 2;
+    const __nv_bfloat16* cs = p.cos + (int64_t)n * p.rope;
+    const __nv_bfloat16* sn = p.sin + (int64_t)n * p.rope;
+#pragma unroll
+    for (int i = 0; i < 4; i += 2) {
+      const int j = (c + i - r0) >> 1;
+      const float ce = __bfloat162float(cs[j]), se = __bfloat162float(sn[j]);
+      const float co = __bfloat162float(cs[half + j]), so = __bfloat162float(sn[half + j]);
+      const float ev = z[i], od = z[i + 1];
+      z[i] = ev * ce - od * se;
+      z[i + 1] = od * co + ev * so;
+    }
+  }
+
+  if (p.rotate) {  // out = z @ hadamard (dense product, any D x D matrix)
+#pragma unroll
+    for (int i = 0; i < 4; ++i) zs[c + i] = z[i];
+    __syncthreads();
+    float o[4] = {0.f, 0.f, 0.f, 0.f};
+    for (int k = 0; k < D; ++k) {
+      const float zk = zs[k];
+      const uint2 hr = *reinterpret_cast<const uint2*>(p.had + (int64_t)k * D + c);
+      const __nv_bfloat162 h01 = *reinterpret_cast<const __nv_bfloat162*>(&hr.x);
+      const __nv_bfloat162 h23 = *reinterpret_cast<const __nv_bfloat162*>(&hr.y);
+      o[0] = fmaf(zk, __low2float(h01), o[0]);
+      o[1] = fmaf(zk, __high2float(h01), o[1]);
+      o[2] = fmaf(zk, __low2float(h23), o[2]);
+      o[3] = fmaf(zk, __high2float(h23), o[3]);
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i) z[i] = o[i];
+  }
+
+  __nv_bfloat162 o01 = __floats2bfloat162_rn(z[0], z[1]);
+  __nv_bfloat162 o23 = __floats2bfloat162_rn(z[2], z[3]);
+  uint2 v;
+  v.x = *reinterpret_cast<uint32_t*>(&o01);
+  v.y = *reinterpret_cast<uint32_t*>(&o23);
+  *dst = v;
+}
+
+}  // namespace
+
+cudaError_t launch_pool(const Params& p, cudaStream_t s) {
+  if (p.n_out <= 0) return cudaSuccess;
+  pool_kernel<<<p.n_out, p.D / 4, 0, s>>>(p);
+  return cudaGetLastError();
+}
+
+}  // namespace cmp

@@ -1,0 +1,101 @@
+// Varlen scheduler: turns cu_seqlens / start_pos into the per-sequence metadata
+// the projection and pooling kernels read (validated token offsets, start
+// positions and first output rows). It runs on the device so a call needs no
+// host synchronisation; this is the role the value-dependent AICPU scheduler
+// plays on "NPU DeepSeek-V4 Ascend C 融合算子优化" (AICPU Scheduler).
+//
+// Output-row layout ("CANN PyPTO 算子实战", 返回值说明 fixes only the row count
+// min(T, T//ratio + B)): sequence b reserves cap_b = min(L_b, L_b / ratio + 1)
+// rows after those of sequences 0..b-1. A sequence covering positions [s, e)
+// completes e/ratio - s/ratio <= cap_b windows, and sum(cap_b) <= the row count.
+#include "cmp_internal.cuh"
+
+namespace cmp {
+namespace {
+
+constexpr int kThreads = 1024;
+
+__device__ __forceinline__ int block_exclusive_scan(int v, int* warp_tot, int* total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int inc = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int n = __shfl_up_sync(0xffffffffu, inc, o);
+    if (lane >= o) inc += n;
+  }
+  if (lane == 31) warp_tot[warp] = inc;
+  __syncthreads();
+  if (warp == 0) {
+    int w = lane < (kThreads / 32) ? warp_tot[lane] : 0;
+    int wi = w;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int n = __shfl_up_sync(0xffffffffu, wi, o);
+      if (lane >= o) wi += n;
+    }
+    warp_tot[lane] = wi - w;  // exclusive prefix of warp totals
+    if (lane == 31) *total = wi;
+  }
+  __syncthreads();
+  const int r = warp_tot[warp] + inc - v;
+  __syncthreads();
+  return r;
+}
+
+__global__ void __launch_bounds__(kThreads) sched_kernel(Params p) {
+  __shared__ int bad;
+  __shared__ int warp_tot[32];
+  __shared__ int chunk_total;
+  if (threadIdx.x == 0) bad = 0;
+  __syncthreads();
+  const int B = p.B;
+  // 1) validate: cu rises from 0 to T, start_pos >= 0, positions fit in int32
+  for (int b = threadIdx.x; b <= B; b += kThreads) {
+    const int c = p.cu_in[b];
+    bool ok = c >= 0 && c <= p.T;
+    if (b == 0) ok = ok && c == 0;
+    if (b == B) ok = ok && c == p.T;
+    if (b < B) {
+      const int c1 = p.cu_in[b + 1];
+      const int s = p.start_pos ? p.start_pos[b] : 0;
+      ok = ok && c1 >= c && s >= 0 && (int64_t)s + (int64_t)(c1 - c) <= (int64_t)INT32_MAX;
+    }
+    if (!ok) atomicOr(&bad, 1);
+  }
+  __syncthreads();
+  const bool rejected = bad != 0;
+  if (rejected && threadIdx.x == 0) atomicOr(p.err, kErrIndex);
+  // 2) metadata; a rejected call gets empty sequences (every output row 0)
+  int carry = 0;
+  for (int base = 0; base < B; base += kThreads) {
+    const int b = base + threadIdx.x;
+    int c = 0, s = 0, cap = 0;
+    if (b < B && !rejected) {
+      c = p.cu_in[b];
+      const int L = p.cu_in[b + 1] - c;
+      s = p.start_pos ? p.start_pos[b] : 0;
+      cap = min(L, L / p.ratio + 1);
+    }
+    const int ex = block_exclusive_scan(cap, warp_tot, &chunk_total);
+    if (b < B) {
+      p.m_cu[b] = c;
+      p.m_s[b] = s;
+      p.m_off[b] = carry + ex;
+    }
+    carry += chunk_total;
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) {
+    p.m_cu[B] = rejected ? 0 : p.T;
+    p.m_off[B] = carry;
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_sched(const Params& p, cudaStream_t s) {
+  sched_kernel<<<1, kThreads, 0, s>>>(p);
+  return cudaGetLastError();
+}
+
+}  // namespace cmp

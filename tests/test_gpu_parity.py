@@ -1,0 +1,245 @@
+"""Parity of the CUDA library with the CPU oracle, on a B200.
+
+Every test runs the library through its C ABI (the ctypes binding) on seeded
+inputs from ``workloads`` and compares with ``oracle`` on the same inputs,
+under the tolerances in tests/gpu_helpers.py.
+"""
+
+import dataclasses
+import json
+import os
+
+import numpy as np
+import pytest
+
+from oracle import run_inputs, window_row_positions
+from workloads import make_chunked, make_config, make_inputs, bf16_bits, sylvester
+from tests.gpu_helpers import (assert_out_close, assert_state_close, bits, dev, run, to_device)
+
+pytestmark = pytest.mark.gpu
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def with_rope(inp):
+    return inp.with_rope(window_row_positions(inp.cu_seqlens, inp.start_pos, inp.ratio))
+
+
+def check(cmp, inp, rows=None):
+    out, kv, sc, err = run(cmp, inp)
+    assert err == 0, f"device error status {err}"
+    res = run_inputs(inp, windows_only=rows)
+    assert_out_close(out, res, rows)
+    if rows is None:
+        assert_state_close(kv, sc, inp, res)
+    return out, kv, sc, res
+
+
+@pytest.fixture(params=[0, 1, 2, 3], ids=["auto", "mma", "tcgen05", "decode"])
+def proj_kernel(request, lib):
+    prev = lib.set_proj_kernel(request.param)
+    yield request.param
+    lib.set_proj_kernel(prev)
+
+
+# ---- the five workloads ----------------------------------------------------
+
+def test_c4li_tiny_prefill(lib, proj_kernel):
+    check(lib, with_rope(make_config("c4li_tiny")))
+
+
+@pytest.mark.slow
+def test_c4a_varlen_prefill(lib):
+    check(lib, with_rope(make_config("c4a_varlen")))
+
+
+def test_c4a_decode(lib, proj_kernel):
+    check(lib, with_rope(make_config("c4a_decode")))
+
+
+@pytest.mark.slow
+def test_c128a_128k_prefill_sampled(lib):
+    inp = with_rope(make_config("c128a_128k"))
+    args = to_device(inp)
+    kv0 = args["kv_state"].clone()
+    sc0 = args["score_state"].clone()
+    out = lib.compressor(**args)
+    assert lib.get_error() == 0
+    o = bits(out)
+    assert o.shape == (1025, 512)
+    rows = [0, 1, 2, 127, 128, 511, 777, 1022, 1023, 1024]
+    res = run_inputs(inp, windows_only=rows)
+    assert_out_close(o, res, rows)
+    assert np.all(o[1024] == 0)
+    # e = 131072 is window aligned: no tail, so no state byte may change
+    import torch
+    assert torch.equal(args["kv_state"], kv0) and torch.equal(args["score_state"], sc0)
+
+
+@pytest.mark.slow
+def test_c4li_chunked_continuation(lib):
+    import torch
+    ch = make_chunked()
+    kv = dev(ch.calls[0].kv_state)
+    sc = dev(ch.calls[0].score_state)
+    okv, osc = ch.calls[0].kv_state, ch.calls[0].score_state
+    per_window = {}
+    for c, call in enumerate(ch.calls):
+        call = dataclasses.replace(with_rope(call), kv_state=okv, score_state=osc)
+        args = to_device(call, kv_state=kv, score_state=sc)
+        out = bits(lib.compressor(**args))
+        assert lib.get_error() == 0
+        res = run_inputs(call)
+        assert_out_close(out, res)
+        assert_state_close(kv.cpu().numpy(), sc.cpu().numpy(), call, res)
+        okv, osc = res.kv_state, res.score_state
+        for row, b, w in res.layout.rows:
+            per_window[(int(ch.order[c][b]), w)] = out[row]
+    one = run_inputs(with_rope(ch.oneshot))
+    got = np.zeros_like(one.out)
+    for row, b, w in one.layout.rows:
+        got[row] = per_window[(b, w)]
+    assert len(per_window) == len(one.layout.rows)
+    assert_out_close(got, one)
+    # the state the chunked calls leave equals the one-shot call's tail
+    m = one.written
+    d = np.abs(kv.cpu().numpy()[m].astype(np.float64) - one.kv_state[m])
+    assert (d <= 1e-4 * np.maximum(np.abs(one.kv_state[m]), 1.0)).all()
+
+
+# ---- the PyPTO example cases and other ratios -------------------------------
+
+@pytest.mark.parametrize("case", json.load(open(os.path.join(GOLDEN, "pypto_example_cases.json")))["cases"],
+                         ids=lambda c: c["name"])
+@pytest.mark.parametrize("shift", [0, -2])
+def test_pypto_example_cases(lib, case, shift):
+    B, S = case["bsz"], case["seq"]
+    coff = 2 if case["ratio"] == 4 else 1
+    sp = max(0, case["start_pos"] + shift)
+    inp = make_inputs(name=case["name"], seed=7, lengths=[S] * B, start_pos=[sp] * B,
+                      H=case["H"], D=case["D"], coff=coff, ratio=case["ratio"],
+                      block_size=case["block_size"], rotate=case["rotate"], lookback=2 * case["ratio"])
+    check(lib, with_rope(inp))
+
+
+@pytest.mark.parametrize("ratio", [2, 8, 16, 32, 64])
+def test_other_ratios(lib, ratio, proj_kernel):
+    rng = np.random.default_rng(ratio)
+    L = rng.integers(0, 5 * ratio, size=5).tolist()
+    sp = rng.integers(0, 3 * ratio, size=5).tolist()
+    inp = make_inputs(name="r", seed=ratio, lengths=L, start_pos=sp, H=1024, D=128, coff=1,
+                      ratio=ratio, block_size=32, rotate=True)
+    check(lib, with_rope(inp))
+
+
+# ---- edges ----------------------------------------------------------------------
+
+EDGE_CASES = {
+    "ragged_tiles": dict(lengths=[1, 129, 300, 0, 77], start_pos=[0, 3, 126, 5, 1], D=512, H=1024,
+                         ratio=4, bs=64),
+    "c128a_partial_windows": dict(lengths=[200, 1, 130], start_pos=[100, 127, 0], D=512, H=1024,
+                                  ratio=128, bs=128),
+    "block_size_1": dict(lengths=[9, 6], start_pos=[2, 0], D=128, H=512, ratio=4, bs=1),
+    "block_size_1024": dict(lengths=[700, 333], start_pos=[1000, 3], D=128, H=512, ratio=4, bs=1024),
+    "far_positions": dict(lengths=[5, 3], start_pos=[(1 << 30) - 3, 2_000_000_001], D=128, H=512,
+                          ratio=4, bs=128, lookback=8),
+    "d128_ratio128": dict(lengths=[260], start_pos=[0], D=128, H=2048, ratio=128, bs=32),
+    "single_token": dict(lengths=[1], start_pos=[3], D=512, H=1024, ratio=4, bs=16),
+    "wide_hidden": dict(lengths=[64, 40], start_pos=[0, 0], D=512, H=16384, ratio=4, bs=128),
+}
+
+
+@pytest.mark.parametrize("name", sorted(EDGE_CASES))
+def test_edge_cases(lib, name):
+    c = dict(EDGE_CASES[name])
+    ratio = c.pop("ratio")
+    bs = c.pop("bs")
+    inp = make_inputs(name=name, seed=11, coff=2 if ratio == 4 else 1, ratio=ratio, block_size=bs,
+                      rotate=c["D"] == 128, **c)
+    check(lib, with_rope(inp))
+
+
+def test_dense_rotation_with_any_matrix(lib):
+    inp = make_inputs(name="rot", seed=3, lengths=[40, 21], start_pos=[0, 6], H=1024, D=128,
+                      coff=2, ratio=4, block_size=16, rotate=True)
+    rng = np.random.default_rng(1)
+    inp = dataclasses.replace(inp, hadamard=bf16_bits(rng.standard_normal((128, 128)).astype(np.float32) / 11))
+    check(lib, with_rope(inp))
+
+
+def test_empty_and_noop_calls(lib):
+    import torch
+    inp = with_rope(make_inputs(name="e", seed=1, lengths=[0, 0], start_pos=[3, 4], H=512, D=128,
+                                coff=2, ratio=4, block_size=16, rotate=False, extra_rows=2))
+    args = to_device(inp)
+    kv0 = args["kv_state"].clone()
+    out = lib.compressor(**args)
+    assert out.shape == (0, 128) and torch.equal(args["kv_state"], kv0)
+    assert lib.get_error() == 0
+
+
+def test_repeat_is_bit_identical_and_idempotent(lib):
+    inp = with_rope(make_inputs(name="d", seed=5, lengths=[333, 91], start_pos=[2, 17], H=2048,
+                                D=512, coff=2, ratio=4, block_size=32, rotate=False))
+    args = to_device(inp)
+    o1 = bits(lib.compressor(**args))
+    kv1, sc1 = args["kv_state"].clone(), args["score_state"].clone()
+    o2 = bits(lib.compressor(**args))   # state already updated: reads only positions < start
+    import torch
+    assert np.array_equal(o1, o2)
+    assert torch.equal(args["kv_state"], kv1) and torch.equal(args["score_state"], sc1)
+
+
+def test_projection_kernels_agree(lib):
+    """All projection kernels give results within the tolerance of the oracle and,
+    for the same kernel, bit-identical repeats."""
+    inp = with_rope(make_inputs(name="k", seed=9, lengths=[40, 7, 1, 16], start_pos=[1, 0, 3, 9],
+                                H=4096, D=512, coff=2, ratio=4, block_size=128, rotate=False))
+    res = run_inputs(inp)
+    outs = {}
+    for k in (1, 2, 3):
+        prev = lib.set_proj_kernel(k)
+        try:
+            o, kv, sc, err = run(lib, inp)
+            o2, _, _, _ = run(lib, inp)
+        finally:
+            lib.set_proj_kernel(prev)
+        assert err == 0
+        assert np.array_equal(o, o2)
+        assert_out_close(o, res)
+        assert_state_close(kv, sc, inp, res)
+        outs[k] = o
+
+
+# ---- faults are reported, never trapped ------------------------------------------
+
+def test_bad_needed_table_entry_sets_error(lib):
+    inp = with_rope(make_inputs(name="bad", seed=2, lengths=[6], start_pos=[9], H=512, D=128,
+                                coff=2, ratio=4, block_size=4, rotate=False))
+    tbl = inp.kv_block_table.copy()
+    tbl[0, 1] = inp.block_num + 5          # block of positions 4..7: the previous window
+    out, kv, sc, err = run(lib, dataclasses.replace(inp, kv_block_table=tbl))
+    assert err == 5                        # CMP_ERR_DEVICE_INDEX
+    assert lib.get_error() == 0            # cleared by the read
+
+
+def test_unneeded_padding_is_not_read(lib):
+    inp = with_rope(make_inputs(name="pad", seed=2, lengths=[6], start_pos=[9], H=512, D=128,
+                                coff=2, ratio=4, block_size=4, rotate=False))
+    tbl = inp.kv_block_table.copy()
+    tbl[0, 0] = -1                         # positions 0..3 are never needed here
+    inp = dataclasses.replace(inp, kv_block_table=tbl, state_block_table=tbl.copy())
+    check(lib, inp)
+
+
+def test_bad_cu_seqlens_rejected_on_device(lib):
+    import torch
+    inp = with_rope(make_inputs(name="cu", seed=2, lengths=[6, 10], start_pos=[0, 0], H=512, D=128,
+                                coff=2, ratio=4, block_size=16, rotate=False))
+    args = to_device(inp)
+    args["cu_seqlens"] = torch.tensor([0, 12, 16], dtype=torch.int32, device="cuda")
+    args["cu_seqlens"][1] = 20             # not rising to T: the call is rejected
+    kv0 = args["kv_state"].clone()
+    out = lib.compressor(**args)
+    assert lib.get_error() == 5
+    assert (bits(out) == 0).all() and torch.equal(args["kv_state"], kv0)
