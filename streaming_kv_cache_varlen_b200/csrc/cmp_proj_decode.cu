@@ -1,10 +1,254 @@
-// Small-T projection that streams the weights at HBM bandwidth.
+// Small-T projection (decode, T <= 64 tokens): the cost is reading the two
+// weight matrices once, so the kernel is built to stream them at HBM bandwidth
+// across the whole GPU.
+//
+//   proj[t][n] = sum_k W[n][k] * x[t][k]  (+ ape on score columns, tail rows to
+//   the paged state), as in the prefill kernels ("compressor torch_extension
+//   API", 计算公式 1-2).
+//
+// Work split: the weight rows are cut into 128-row tiles (MMA M = 128) and the
+// hidden dimension into 8 slices; the 8 CTAs that share a row tile form one
+// thread-block cluster. Each CTA streams its 128 x (H/8) weight slice and the
+// matching x slice with TMA through a 6-stage ring, accumulates a 128 x N
+// partial product in TMEM with tcgen05.mma (N = T rounded up to 16), and parks
+// it in its shared memory. After a cluster barrier, CTA j of the cluster sums
+// rows 16j..16j+15 of the 8 partials, always in cluster-rank order (so the
+// result is bitwise reproducible), reading its peers' shared memory, and writes
+// those rows of proj and of the state tail.
+// (Splitting the head dimension across more cores to raise the number of
+// active cores and the bandwidth in decode is the idea of "NPU DeepSeek-V4
+// Ascend C 融合算子优化", Decode; here the split is over K and the reduction
+// stays on chip.)
+#include <mutex>
+
 #include "cmp_internal.cuh"
+#include "cmp_sm100.cuh"
 
 namespace cmp {
+namespace {
 
-bool proj_decode_supported(const Params&) { return false; }
+using namespace sm100;
+
+constexpr int BM = 128;        // weight rows per cluster
+constexpr int BK = 64;         // K per stage
+constexpr int KSPLIT = 8;      // CTAs per cluster (K slices)
+constexpr int STAGES = 6;
+constexpr int MAX_T = 64;
+constexpr int kThreads = 128;
+
+struct Smem {
+  __nv_bfloat16 w[STAGES][BM * BK];      // 16 KB per stage, 1024-byte aligned
+  __nv_bfloat16 x[STAGES][MAX_T * BK];   // up to 8 KB per stage
+  float part[MAX_T][BM];                 // this CTA's partial product, [token][row]
+  uint64_t full[STAGES];
+  uint64_t empty[STAGES];
+  uint64_t acc_full;
+  uint32_t tmem_base;
+  int abort;
+};
+
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+
+__device__ __forceinline__ void cluster_sync() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::
+                   : "memory");
+}
+
+__device__ __forceinline__ float ld_peer(const float* local, uint32_t peer) {
+  uint32_t a = smem_u32(local), ra;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(ra) : "r"(a), "r"(peer));
+  float v;
+  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(ra) : "memory");
+  return v;
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+    proj_decode_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUtensorMap map_wkv,
+                       const __grid_constant__ CUtensorMap map_wg, Params p, int NT) {
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  Smem& sm = *reinterpret_cast<Smem*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_rank();            // K slice of this CTA
+  const int m0 = blockIdx.y * BM;                  // weight row tile (of the 2C rows)
+  const bool score = m0 >= p.C;
+  const CUtensorMap* wmap = score ? &map_wg : &map_wkv;
+  const int wrow = score ? m0 - p.C : m0;
+  const int kb_total = p.H / BK;
+  const int kb_lo = (int)(rank * kb_total / KSPLIT);
+  const int kb_hi = (int)((rank + 1) * kb_total / KSPLIT);
+  const uint32_t x_bytes = (uint32_t)NT * BK * 2;
+  const uint32_t tmem_cols = NT <= 32 ? 32 : 64;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&sm.full[s], 1);
+      mbar_init(&sm.empty[s], 1);
+    }
+    mbar_init(&sm.acc_full, 1);
+    sm.abort = 0;
+    fence_barrier_init();
+    prefetch_tmap(wmap);
+    prefetch_tmap(&map_x);
+  }
+  if (warp == 1) tmem_alloc(&sm.tmem_base, tmem_cols);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = sm.tmem_base;
+  volatile int* abort = &sm.abort;
+
+  if (warp == 0 && lane == 0) {
+    int stage = 0;
+    uint32_t phase = 0;
+    for (int kb = kb_lo; kb < kb_hi; ++kb) {
+      if (!mbar_wait(&sm.empty[stage], phase ^ 1u, abort)) break;
+      mbar_arrive_expect_tx(&sm.full[stage], BM * BK * 2 + x_bytes);
+      tma_load_2d(sm.w[stage], wmap, &sm.full[stage], kb * BK, wrow);
+      tma_load_2d(sm.x[stage], &map_x, &sm.full[stage], kb * BK, 0);
+      if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+    }
+  } else if (warp == 1 && lane == 0) {
+    int stage = 0;
+    uint32_t phase = 0;
+    const uint32_t idesc = idesc_bf16_f32(BM, NT);
+    bool ok = true;
+    for (int kb = kb_lo; kb < kb_hi; ++kb) {
+      if (!mbar_wait(&sm.full[stage], phase, abort)) { ok = false; break; }
+      tc_fence_after();
+      const uint32_t a0 = smem_u32(sm.w[stage]);
+      const uint32_t b0 = smem_u32(sm.x[stage]);
+#pragma unroll
+      for (int k = 0; k < BK / 16; ++k)
+        mma_bf16(tmem, sw128_kmajor_desc(a0 + k * 32), sw128_kmajor_desc(b0 + k * 32), idesc,
+                 (kb > kb_lo || k > 0) ? 1u : 0u);
+      mma_commit(&sm.empty[stage]);
+      if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+    }
+    if (ok) mma_commit(&sm.acc_full);
+  }
+
+  // every warp: move its 32 accumulator lanes (weight rows) to shared memory
+  const bool have = mbar_wait(&sm.acc_full, 0, abort);
+  if (__all_sync(0xffffffffu, have)) {
+    tc_fence_after();
+    const int row = warp * 32 + lane;
+    for (int c0 = 0; c0 < NT; c0 += 32) {
+      uint32_t r[32];
+      tmem_ld32(tmem + ((uint32_t)(warp * 32) << 16) + c0, r);
+      tmem_ld_wait(r);
+#pragma unroll
+      for (int j = 0; j < 32; ++j)
+        if (c0 + j < NT) sm.part[c0 + j][row] = __uint_as_float(r[j]);
+    }
+  }
+  tc_fence_before();
+  cluster_sync();  // all partials parked; every CTA reaches this on every path
+
+  // CTA `rank` reduces rows 16*rank .. 16*rank+15 of the tile over the 8 slices
+  if (!*abort) {
+    for (int i = threadIdx.x; i < 16 * NT; i += kThreads) {
+      const int tok = i >> 4, r = (int)(rank * 16) + (i & 15);
+      const int t = tok;
+      if (t >= p.T) continue;
+      const int b = upper_index(p.m_cu, p.B, t);
+      if (b >= p.B) continue;
+      float v = 0.f;
+      for (uint32_t q = 0; q < KSPLIT; ++q) v += ld_peer(&sm.part[tok][r], q);
+      const int s = p.m_s[b];
+      const int c0 = p.m_cu[b];
+      const int pos = s + (t - c0);
+      const int e = s + (p.m_cu[b + 1] - c0);
+      const int col = wrow + r;
+      if (score) v += __ldg(p.ape + (int64_t)(pos % p.ratio) * p.C + col);
+      p.proj[(int64_t)t * (2 * p.C) + (score ? p.C : 0) + col] = v;
+      if (pos >= tail_threshold(e, p.ratio, p.coff)) {
+        const int pr = table_row(p, score ? p.sc_tbl : p.kv_tbl, b, pos);
+        if (pr >= 0) (score ? p.score_state : p.kv_state)[((int64_t)pr * p.bs + pos % p.bs) * p.C + col] = v;
+      }
+    }
+  }
+  cluster_sync();  // peers may still be reading this CTA's partial
+
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, tmem_cols);
+  }
+  if (threadIdx.x == 0 && sm.abort) atomicOr(p.err, kErrTimeout);
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*,
+                                  CUtensorMapInterleave, CUtensorMapSwizzle, CUtensorMapL2promotion,
+                                  CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(f);
+  });
+  return fn;
+}
+
+bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows) {
+  EncodeTiledFn f = encode_fn();
+  if (!f) return false;
+  const cuuint64_t dims[2] = {cols, rows};
+  const cuuint64_t strides[1] = {cols * 2};
+  const cuuint32_t box[2] = {(cuuint32_t)BK, box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  return f(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace
+
+bool proj_decode_supported(const Params& p) {
+  return p.T >= 1 && p.T <= MAX_T && (p.H / BK) >= KSPLIT && p.H % BK == 0 && (2 * p.C) % BM == 0 &&
+         encode_fn() != nullptr;
+}
+
 size_t proj_decode_workspace(const Params&) { return 0; }
-cudaError_t launch_proj_decode(const Params&, cudaStream_t) { return cudaErrorNotSupported; }
+
+cudaError_t launch_proj_decode(const Params& p, cudaStream_t s) {
+  const int NT = (p.T + 15) / 16 * 16;
+  CUtensorMap mx, mkv, mg;
+  if (!make_map(&mx, p.x, p.T, p.H, (uint32_t)NT) || !make_map(&mkv, p.wkv, p.C, p.H, BM) ||
+      !make_map(&mg, p.wgate, p.C, p.H, BM))
+    return cudaErrorInvalidValue;
+  const size_t smem = sizeof(Smem) + 1024;
+  static int configured[64] = {0};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev >= 64 || !configured[dev]) {
+    cudaError_t e = cudaFuncSetAttribute(proj_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)smem);
+    if (e != cudaSuccess) return e;
+    if (dev < 64) configured[dev] = 1;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(KSPLIT, (2 * p.C) / BM, 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = KSPLIT;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, proj_decode_kernel, mx, mkv, mg, p, NT);
+}
 
 }  // namespace cmp

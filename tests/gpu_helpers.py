@@ -81,10 +81,13 @@ def assert_out_close(gpu_bits, res, rows=None):
     return float(err.max()) if err.size else 0.0
 
 
-def assert_state_close(gpu_kv, gpu_sc, inp, res):
-    """Written slots within STATE_TOL, untouched slots bit-identical."""
-    for gpu, before, ref, mask in ((gpu_kv, inp.kv_state, res.kv_state, res.written),
-                                   (gpu_sc, inp.score_state, res.score_state, res.written_score)):
+def assert_state_close(gpu_kv, gpu_sc, inp, res, before_kv=None, before_sc=None):
+    """Written slots within STATE_TOL, untouched slots bit-identical to the device
+    state before the call (by default the input's state)."""
+    before_kv = inp.kv_state if before_kv is None else before_kv
+    before_sc = inp.score_state if before_sc is None else before_sc
+    for gpu, before, ref, mask in ((gpu_kv, before_kv, res.kv_state, res.written),
+                                   (gpu_sc, before_sc, res.score_state, res.written_score)):
         untouched = ~mask
         assert np.array_equal(gpu[untouched].view(np.uint32), before[untouched].view(np.uint32)), \
             "a state slot the call must not write changed"

@@ -87,11 +87,12 @@ def test_c4li_chunked_continuation(lib):
     for c, call in enumerate(ch.calls):
         call = dataclasses.replace(with_rope(call), kv_state=okv, score_state=osc)
         args = to_device(call, kv_state=kv, score_state=sc)
+        kv_before, sc_before = kv.cpu().numpy(), sc.cpu().numpy()
         out = bits(lib.compressor(**args))
         assert lib.get_error() == 0
-        res = run_inputs(call)
+        res = run_inputs(call)   # the oracle continues from its own state
         assert_out_close(out, res)
-        assert_state_close(kv.cpu().numpy(), sc.cpu().numpy(), call, res)
+        assert_state_close(kv.cpu().numpy(), sc.cpu().numpy(), call, res, kv_before, sc_before)
         okv, osc = res.kv_state, res.score_state
         for row, b, w in res.layout.rows:
             per_window[(int(ch.order[c][b]), w)] = out[row]
