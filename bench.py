@@ -245,18 +245,14 @@ def traffic_for(kernel_file: str, kernel: str, units_scale: float = 1.0):
     return e["bytes_per_launch"] * units_scale
 
 
-def run_ours(args):
+def bench_prefill(args, ws, local, stream, peaks, peak_src):
+    """Device-resident prefill steps: value, per-kernel times and the roofline."""
     import torch
 
     import streaming_kv_cache_varlen_b200 as cmp
 
-    ws, rank, local = dist_setup()
     device = torch.device("cuda", local)
-    torch.cuda.set_device(device)
-    stream = torch.cuda.current_stream(device)
-    peaks, peak_src = read_peaks()
-
-    # ---------------- prefill: device-resident inputs ----------------
+    rank = int(os.environ.get("RANK", "0"))
     pf = prefill_inputs(device, seed=1234 + rank)
     out = torch.empty((cmp.out_rows(1, PREFILL["T"], PREFILL["ratio"]), PREFILL["D"]),
                       dtype=torch.bfloat16, device=device)
@@ -280,9 +276,7 @@ def run_ours(args):
     launches = cmp.launch_count() - launches0
     assert cmp.get_error() == 0
     ms = max_over_ranks(e0.elapsed_time(e1), ws)
-    ms_step = ms / args.steps
-    tokens = PREFILL["T"] * ws * args.steps
-    value = tokens / (ms / 1e3)
+    value = PREFILL["T"] * ws * args.steps / (ms / 1e3)
 
     # dominant kernel: the projection (a dense bf16 contraction)
     proj_name = max(("proj_tcgen05", "proj_mma_sync", "proj_decode"), key=lambda k: prof[k][0])
@@ -295,21 +289,30 @@ def run_ours(args):
              "proj_decode": "cmp_proj_decode.cu"}[proj_name]
     roofline = {"kernel": proj_name, "bound": "tensor", "achieved": achieved, "peak": peak,
                 "unit": "TFLOP/s", "frac": achieved / peak if achieved else None,
-                "traffic": traffic_for(kfile, proj_name), "peak_source": peak_src + " (burst)",
-                "algorithmic_flops_per_launch": flops,
+                "traffic": traffic_for(kfile, proj_name, T / 131072.0),
+                "peak_source": peak_src + " (burst)", "algorithmic_flops_per_launch": flops,
                 "kernel_ms": {k: (v[0] / v[1] if v[1] else None) for k, v in prof.items()}}
+    return dict(value=value, ms_step=ms / args.steps, launches=launches, roofline=roofline,
+                clocks=clk.summary(), inputs=pf, out=out)
 
-    # ---------------- e2e: host buffers, copies inside the timed region ----------------
+
+def bench_e2e(args, ws, stream, pf, out):
+    """The same metric through the public call with host buffers: per step, H2D of
+    the step's inputs from pinned memory, the call, D2H of the output."""
+    import torch
+
+    import streaming_kv_cache_varlen_b200 as cmp
+
     host_names = ("x", "cu_seqlens", "start_pos", "kv_block_table", "state_block_table", "sin", "cos")
     host = {k: pf[k].cpu().pin_memory() for k in host_names}
     out_host = torch.empty(out.shape, dtype=out.dtype).pin_memory()
     dev_in = {k: torch.empty_like(pf[k]) for k in host_names}
     h2d = sum(v.numel() * v.element_size() for v in host.values())
     d2h = out.numel() * out.element_size()
-    e2e_steps = max(1, min(args.steps, 20))
+    steps = max(1, min(args.steps, 20))
     call = dict(pf)
 
-    def e2e_step():
+    def step():
         for k in host_names:
             dev_in[k].copy_(host[k], non_blocking=True)
             call[k] = dev_in[k]
@@ -317,32 +320,77 @@ def run_ours(args):
         out_host.copy_(out, non_blocking=True)
 
     for _ in range(2):
-        e2e_step()
+        step()
     torch.cuda.synchronize()
     barrier(ws)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
-    for _ in range(e2e_steps):
-        e2e_step()
+    for _ in range(steps):
+        step()
     e1.record(stream)
     torch.cuda.synchronize()
-    e2e_ms = max_over_ranks(e0.elapsed_time(e1), ws)
-    e2e_value = PREFILL["T"] * ws * e2e_steps / (e2e_ms / 1e3)
-    del host, dev_in, call
-    del pf
-    torch.cuda.empty_cache()
+    ms = max_over_ranks(e0.elapsed_time(e1), ws)
+    return {"value": PREFILL["T"] * ws * steps / (ms / 1e3), "unit": "tokens/s",
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": steps}
 
-    # ---------------- decode: microseconds per call, L2 flushed ----------------
+
+def bench_decode(args, ws, local, stream, peaks, peak_src):
+    """C4A 32-request decode, microseconds of device time per call.
+
+    Device time comes from CUDA-graph replays: a graph of N x (256 MB L2 flush,
+    call) minus a graph of N flushes alone, divided by N, so host and binding
+    overhead is excluded and every call starts with a cold L2. The eager time
+    (events around each call from Python, host overhead included) is reported
+    beside it."""
+    import torch
+
+    import streaming_kv_cache_varlen_b200 as cmp
+
+    device = torch.device("cuda", local)
     dec, dec_bytes, dec_inp = decode_inputs(device)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=device)
     dout = torch.empty((cmp.out_rows(dec_inp.B, dec_inp.T, dec_inp.ratio), dec_inp.D),
                        dtype=torch.bfloat16, device=device)
-    for _ in range(max(3, args.warmup)):
-        cmp.compressor(**dec, out=dout)
+    side = torch.cuda.Stream(device)
+    with torch.cuda.stream(side):
+        for _ in range(max(3, args.warmup)):
+            cmp.compressor(**dec, out=dout)
+            flush.fill_(1)
     torch.cuda.synchronize()
-    n_dec = max(20, min(200, args.steps))
+    n = 50
+    g_call, g_flush = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g_call, stream=side):
+        for _ in range(n):
+            flush.fill_(1)
+            cmp.compressor(**dec, out=dout)
+    with torch.cuda.graph(g_flush, stream=side):
+        for _ in range(n):
+            flush.fill_(1)
+    torch.cuda.synchronize()
+
+    def replay(g):
+        best = None
+        for _ in range(5):
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            with torch.cuda.stream(side):  # replay() launches on the current stream
+                a.record(side)
+                g.replay()
+                b.record(side)
+            torch.cuda.synchronize()
+            t = a.elapsed_time(b)
+            best = t if best is None else min(best, t)
+        return best
+
+    barrier(ws)
+    t_call, t_flush = replay(g_call), replay(g_flush)
+    assert cmp.get_error(side) == 0
+    dec_us = max_over_ranks((t_call - t_flush) * 1e3 / n, ws)
+    del g_call, g_flush
+
+    # eager: events around each call from Python (host overhead included)
     times = []
     cmp.profile_start()
-    for _ in range(n_dec):
+    for _ in range(20):
         flush.fill_(1)
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record(stream)
@@ -351,38 +399,54 @@ def run_ours(args):
         times.append((a, b))
     torch.cuda.synchronize()
     dprof = cmp.profile_stop()
-    assert cmp.get_error() == 0
-    us = sorted(a.elapsed_time(b) * 1e3 for a, b in times)
-    dec_us = statistics.median(us)
-    dec_us = max_over_ranks(dec_us, ws)
-    decode = {"workload": "c4a_decode: 32 requests x 1 token, H=4096, D=512, ratio 4",
-              "us_per_call": dec_us, "us_per_call_min": us[0], "calls": n_dec,
-              "l2": "flushed (256 MB write) before every call",
-              "roofline": {"bound": "hbm", "achieved": dec_bytes / (dec_us / 1e6) / 1e9,
-                           "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                           "frac": dec_bytes / (dec_us / 1e6) / 1e9 / peaks["hbm_gbs"],
-                           "algorithmic_bytes_per_call": dec_bytes, "peak_source": peak_src},
-              "kernel_us": {k: (v[0] / v[1] * 1e3 if v[1] else None) for k, v in dprof.items()}}
+    eager = statistics.median(a.elapsed_time(b) * 1e3 for a, b in times)
+    ach = dec_bytes / (dec_us / 1e6) / 1e9
+    return {"workload": "c4a_decode: 32 requests x 1 token, H=4096, D=512, ratio 4",
+            "us_per_call": dec_us, "us_per_call_eager": eager, "calls": n,
+            "timing": "CUDA-graph replay of 50 x (L2 flush + call) minus 50 flushes, / 50",
+            "roofline": {"bound": "hbm", "achieved": ach, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                         "frac": ach / peaks["hbm_gbs"], "algorithmic_bytes_per_call": dec_bytes,
+                         "peak_source": peak_src},
+            "kernel_us_eager": {k: (v[0] / v[1] * 1e3 if v[1] else None) for k, v in dprof.items()}}
 
-    # ---------------- CPU baseline: the oracle on a bounded sample ----------------
+
+def run_ours(args):
+    import torch
+
+    ws, rank, local = dist_setup()
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    stream = torch.cuda.current_stream(device)
+    peaks, peak_src = read_peaks()
+
+    pre = e2e = decode = None
+    if args.only in ("all", "prefill"):
+        pre = bench_prefill(args, ws, local, stream, peaks, peak_src)
+        if args.only == "all":
+            e2e = bench_e2e(args, ws, stream, pre["inputs"], pre["out"])
+        pre.pop("inputs")
+        pre.pop("out")
+        torch.cuda.empty_cache()
+    if args.only in ("all", "decode"):
+        decode = bench_decode(args, ws, local, stream, peaks, peak_src)
     cpu = None
-    if rank == 0 and ws == 1 and not args.no_cpu_baseline:
+    if rank == 0 and ws == 1 and args.only == "all" and not args.no_cpu_baseline:
         cpu = cpu_baseline(args.cpu_tokens)
 
     if rank == 0:
-        line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": ws,
-                "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+        line = {"metric": METRIC, "value": pre["value"] if pre else None, "unit": "tokens/s",
+                "n_gpus": ws, "steps": args.steps, "warmup": args.warmup,
+                "ms_per_step": pre["ms_step"] if pre else None,
                 "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
                 "dtype": "bf16 in, fp32 accumulate / state, bf16 out", "data": "synthetic",
-                "config": {"workload": "c128a_128k: C128A prefill, 1 sequence x 131072 tokens, "
-                                       "H=4096, D=512, ratio=128, coff=1, block_size=128",
+                "config": {"workload": f"c128a_128k: C128A prefill, 1 sequence x {PREFILL['T']} "
+                                       "tokens, H=4096, D=512, ratio=128, coff=1, block_size=128",
                            "global_batch": ws, "seq_len": PREFILL["T"],
                            "parallelism": f"dp{ws} (independent replicas)",
                            "l2": "inputs larger than L2 (x is 1 GiB per step)"},
-                "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d,
-                        "d2h_bytes_per_step": d2h, "steps": e2e_steps},
-                "gpu_launches": launches, "roofline": roofline, "decode": decode,
-                "clocks": clk.summary(), "cpu_baseline": cpu}
+                "e2e": e2e, "gpu_launches": pre["launches"] if pre else None,
+                "roofline": pre["roofline"] if pre else None, "decode": decode,
+                "clocks": pre["clocks"] if pre else None, "cpu_baseline": cpu}
         print(json.dumps(line), flush=True)
     if ws > 1:
         import torch.distributed as dist
@@ -457,9 +521,14 @@ def main():
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--cpu-tokens", type=int, default=8192)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--only", choices=("all", "prefill", "decode"), default="all",
+                    help="run only one part (for profiler captures)")
+    ap.add_argument("--prefill-tokens", type=int, default=PREFILL["T"],
+                    help="tokens of the prefill sequence (smaller cases for profiler captures)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
+    PREFILL["T"] = args.prefill_tokens
     if args.impl == "reference":
         run_reference(args)
     else:

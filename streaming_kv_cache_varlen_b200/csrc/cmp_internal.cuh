@@ -77,6 +77,19 @@ __device__ __forceinline__ int tail_threshold(int e, int ratio, int coff) {
   return (e / ratio - coff + 1) * ratio;
 }
 
+// Raise a kernel's dynamic shared-memory limit once per device (the attribute
+// belongs to the function on the current device).
+template <class K>
+inline cudaError_t smem_attr_once(K* kernel, size_t bytes, int (&done)[64]) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 64 && done[dev]) return cudaSuccess;
+  e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+  if (e == cudaSuccess && dev < 64) done[dev] = 1;
+  return e;
+}
+
 // Kernel launchers (each file defines its own).
 cudaError_t launch_sched(const Params& p, cudaStream_t s);
 cudaError_t launch_proj_mma(const Params& p, cudaStream_t s);

@@ -7,8 +7,9 @@
 //    the window, columns [D, 2D); the first window of a sequence has no
 //    previous rows ("compressor torch_extension API", 计算公式 2-4; "CANN PyPTO
 //    算子实战", 压缩窗口与状态更新: 0 and -inf fill the missing previous window).
-//    A row at a position inside this call comes from the projection buffer,
-//    an earlier one from the paged state;
+//    A row at a position inside this call comes from the projection buffer
+//    (raw score, plus ape[position mod ratio] here), an earlier one from the
+//    paged state (which already holds score + ape);
 //  * per-channel softmax over those rows weighting a sum of the kv rows
 //    (计算公式 3-5), as an online (running max) softmax in fp32;
 //  * RMSNorm, eps 1e-6, times norm_weight; interleaved RoPE on the last
@@ -35,9 +36,22 @@ __device__ __forceinline__ void online(float& m, float& l, float& a, float z, fl
   m = mn;
 }
 
+// Where row j of a window comes from: this call's projection row t (raw score,
+// ape row given) or an earlier call's state rows (score already with ape), or
+// nowhere (masked / bad table entry).
+struct RowSrc {
+  int64_t kv;    // element offset of the row start: proj row (2C wide) or kv_state row (C wide)
+  int64_t sc;    // proj row again, or score_state row
+  int32_t ape;   // ape row for projection rows, -1 for state rows, -2 for skipped rows
+  int32_t half;  // column offset of the half this row contributes (0 or D)
+};
+
+constexpr int kMaxRows = 256;  // coff * ratio <= 256
+
 __global__ void __launch_bounds__(128) pool_kernel(Params p) {
   __shared__ float red[32];
   __shared__ float zs[512];
+  __shared__ RowSrc src[kMaxRows];
   const int n = blockIdx.x;
   const int D = p.D, C = p.C, r = p.ratio;
   const int c = threadIdx.x * 4;
@@ -58,31 +72,67 @@ __global__ void __launch_bounds__(128) pool_kernel(Params p) {
     return;
   }
 
+  // 1) resolve every row of the window (table lookups in parallel)
+  const int rows = p.coff * r;
+  for (int j = threadIdx.x; j < rows; j += blockDim.x) {
+    const bool bhalf = p.coff == 1 || j >= r;
+    const int q = p.coff == 1 ? w * r + j : (j < r ? (w - 1) * r + j : w * r + (j - r));
+    RowSrc rs{0, 0, -2, (p.coff == 2 && bhalf) ? D : 0};
+    if (q >= s) {
+      rs.kv = (int64_t)(cu + (q - s)) * (2 * C);
+      rs.sc = rs.kv + C;
+      rs.ape = q % r;
+    } else if (q >= 0) {  // q < 0: the first window has no previous window
+      const int rk = table_row(p, p.kv_tbl, b, q);
+      const int rv = table_row(p, p.sc_tbl, b, q);
+      if (rk >= 0 && rv >= 0) {
+        rs.kv = ((int64_t)rk * p.bs + q % p.bs) * C;
+        rs.sc = ((int64_t)rv * p.bs + q % p.bs) * C;
+        rs.ape = -1;
+      }
+    }
+    src[j] = rs;
+  }
+  __syncthreads();
+
+  // 2) online softmax over the rows, 8 rows' loads in flight at a time
   float m[4], l[4], a[4];
 #pragma unroll
   for (int i = 0; i < 4; ++i) { m[i] = -INFINITY; l[i] = 0.f; a[i] = 0.f; }
-  const int rows = p.coff * r;
-  for (int j = 0; j < rows; ++j) {
-    const bool bhalf = p.coff == 1 || j >= r;
-    const int q = p.coff == 1 ? w * r + j : (j < r ? (w - 1) * r + j : w * r + (j - r));
-    if (q < 0) continue;  // the first window has no previous window
-    const int col = (p.coff == 2 && bhalf) ? D + c : c;
-    float4 kv, sc;
-    if (q >= s) {
-      const float* row = p.proj + (int64_t)(cu + (q - s)) * (2 * C);
-      kv = ld4(row + col);
-      sc = ld4(row + C + col);
-    } else {
-      const int rk = table_row(p, p.kv_tbl, b, q);
-      const int rs = table_row(p, p.sc_tbl, b, q);
-      if (rk < 0 || rs < 0) continue;
-      kv = ld4(p.kv_state + ((int64_t)rk * p.bs + q % p.bs) * C + col);
-      sc = ld4(p.score_state + ((int64_t)rs * p.bs + q % p.bs) * C + col);
+  for (int j0 = 0; j0 < rows; j0 += 8) {
+    float4 kv[8], sc[8];
+    bool use[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      use[u] = false;
+      if (j0 + u < rows) {
+        const RowSrc rs = src[j0 + u];
+        const int col = rs.half + c;
+        if (rs.ape >= 0) {
+          kv[u] = ld4(p.proj + rs.kv + col);
+          sc[u] = ld4(p.proj + rs.sc + col);
+          const float4 ap = ld4(p.ape + (int64_t)rs.ape * C + col);
+          sc[u].x += ap.x;
+          sc[u].y += ap.y;
+          sc[u].z += ap.z;
+          sc[u].w += ap.w;
+          use[u] = true;
+        } else if (rs.ape == -1) {
+          kv[u] = ld4(p.kv_state + rs.kv + col);
+          sc[u] = ld4(p.score_state + rs.sc + col);
+          use[u] = true;
+        }
+      }
     }
-    online(m[0], l[0], a[0], sc.x, kv.x);
-    online(m[1], l[1], a[1], sc.y, kv.y);
-    online(m[2], l[2], a[2], sc.z, kv.z);
-    online(m[3], l[3], a[3], sc.w, kv.w);
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      if (use[u]) {
+        online(m[0], l[0], a[0], sc[u].x, kv[u].x);
+        online(m[1], l[1], a[1], sc[u].y, kv[u].y);
+        online(m[2], l[2], a[2], sc[u].z, kv[u].z);
+        online(m[3], l[3], a[3], sc[u].w, kv[u].w);
+      }
+    }
   }
   float y[4];
 #pragma unroll

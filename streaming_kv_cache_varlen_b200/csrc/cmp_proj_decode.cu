@@ -2,8 +2,8 @@
 // weight matrices once, so the kernel is built to stream them at HBM bandwidth
 // across the whole GPU.
 //
-//   proj[t][n] = sum_k W[n][k] * x[t][k]  (+ ape on score columns, tail rows to
-//   the paged state), as in the prefill kernels ("compressor torch_extension
+//   proj[t][n] = sum_k W[n][k] * x[t][k]  (raw scores; tail rows, score rows
+//   with ape, to the paged state), as in the prefill kernels ("compressor torch_extension
 //   API", 计算公式 1-2).
 //
 // Work split: the weight rows are cut into 128-row tiles (MMA M = 128) and the
@@ -11,10 +11,11 @@
 // thread-block cluster. Each CTA streams its 128 x (H/8) weight slice and the
 // matching x slice with TMA through a 6-stage ring, accumulates a 128 x N
 // partial product in TMEM with tcgen05.mma (N = T rounded up to 16), and parks
-// it in its shared memory. After a cluster barrier, CTA j of the cluster sums
-// rows 16j..16j+15 of the 8 partials, always in cluster-rank order (so the
-// result is bitwise reproducible), reading its peers' shared memory, and writes
-// those rows of proj and of the state tail.
+// pushes each row of it into the shared memory of the CTA that owns the row
+// (CTA j owns rows 16j..16j+15) through distributed shared memory. After one
+// cluster barrier every CTA sums its 16 rows over the 8 slices, always in
+// slice order (so the result is bitwise reproducible), and writes those rows
+// of proj and of the state tail.
 // (Splitting the head dimension across more cores to raise the number of
 // active cores and the bandwidth in decode is the idea of "NPU DeepSeek-V4
 // Ascend C 融合算子优化", Decode; here the split is over K and the reduction
@@ -36,10 +37,18 @@ constexpr int STAGES = 6;
 constexpr int MAX_T = 64;
 constexpr int kThreads = 128;
 
+struct TokMeta {
+  int32_t valid;     // token belongs to a sequence
+  int32_t ape_row;   // position mod ratio
+  int64_t kv_off;    // element offset of its kv_state row if it is a tail row, else -1
+  int64_t sc_off;    // same for score_state
+};
+
 struct Smem {
   __nv_bfloat16 w[STAGES][BM * BK];      // 16 KB per stage, 1024-byte aligned
   __nv_bfloat16 x[STAGES][MAX_T * BK];   // up to 8 KB per stage
-  float part[MAX_T][BM];                 // this CTA's partial product, [token][row]
+  float recv[KSPLIT][MAX_T][16];         // partials of this CTA's 16 rows, from every K slice
+  TokMeta tok[MAX_T];
   uint64_t full[STAGES];
   uint64_t empty[STAGES];
   uint64_t acc_full;
@@ -58,12 +67,12 @@ __device__ __forceinline__ void cluster_sync() {
                    : "memory");
 }
 
-__device__ __forceinline__ float ld_peer(const float* local, uint32_t peer) {
-  uint32_t a = smem_u32(local), ra;
-  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(ra) : "r"(a), "r"(peer));
-  float v;
-  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(ra) : "memory");
-  return v;
+// Store v into the shared memory of cluster CTA `peer`, at the address `local`
+// has in this CTA.
+__device__ __forceinline__ void st_peer(float* local, uint32_t peer, float v) {
+  uint32_t ra;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(ra) : "r"(smem_u32(local)), "r"(peer));
+  asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(ra), "f"(v) : "memory");
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -132,47 +141,66 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (ok) mma_commit(&sm.acc_full);
   }
 
-  // every warp: move its 32 accumulator lanes (weight rows) to shared memory
+  // while the weights stream in: per-token facts for the epilogue
+  for (int t = threadIdx.x; t < NT; t += kThreads) {
+    TokMeta m{0, 0, -1, -1};
+    if (t < p.T) {
+      const int b = upper_index(p.m_cu, p.B, t);
+      if (b < p.B) {
+        const int s0 = p.m_s[b];
+        const int c0 = p.m_cu[b];
+        const int pos = s0 + (t - c0);
+        const int e = s0 + (p.m_cu[b + 1] - c0);
+        m.valid = 1;
+        m.ape_row = pos % p.ratio;
+        if (pos >= tail_threshold(e, p.ratio, p.coff)) {
+          const int rk = table_row(p, p.kv_tbl, b, pos);
+          const int rs = table_row(p, p.sc_tbl, b, pos);
+          if (rk >= 0) m.kv_off = ((int64_t)rk * p.bs + pos % p.bs) * p.C;
+          if (rs >= 0) m.sc_off = ((int64_t)rs * p.bs + pos % p.bs) * p.C;
+        }
+      }
+    }
+    sm.tok[t] = m;
+  }
+
+  // every warp: its 32 accumulator lanes (weight rows) go to the CTA that owns
+  // them (rows 16j..16j+15 -> cluster rank j), into slot [this K slice]
   const bool have = mbar_wait(&sm.acc_full, 0, abort);
   if (__all_sync(0xffffffffu, have)) {
     tc_fence_after();
     const int row = warp * 32 + lane;
+    const uint32_t owner = (uint32_t)(row >> 4);
     for (int c0 = 0; c0 < NT; c0 += 32) {
       uint32_t r[32];
       tmem_ld32(tmem + ((uint32_t)(warp * 32) << 16) + c0, r);
       tmem_ld_wait(r);
 #pragma unroll
       for (int j = 0; j < 32; ++j)
-        if (c0 + j < NT) sm.part[c0 + j][row] = __uint_as_float(r[j]);
+        if (c0 + j < NT) st_peer(&sm.recv[rank][c0 + j][row & 15], owner, __uint_as_float(r[j]));
     }
   }
   tc_fence_before();
-  cluster_sync();  // all partials parked; every CTA reaches this on every path
+  cluster_sync();  // every CTA reaches this on every path; the pushes are now visible
 
-  // CTA `rank` reduces rows 16*rank .. 16*rank+15 of the tile over the 8 slices
+  // this CTA's rows 16*rank .. 16*rank+15: sum the K slices in a fixed order
   if (!*abort) {
     for (int i = threadIdx.x; i < 16 * NT; i += kThreads) {
-      const int tok = i >> 4, r = (int)(rank * 16) + (i & 15);
-      const int t = tok;
-      if (t >= p.T) continue;
-      const int b = upper_index(p.m_cu, p.B, t);
-      if (b >= p.B) continue;
+      const int t = i >> 4, r = i & 15;
+      const TokMeta m = sm.tok[t];
+      if (t >= p.T || !m.valid) continue;
       float v = 0.f;
-      for (uint32_t q = 0; q < KSPLIT; ++q) v += ld_peer(&sm.part[tok][r], q);
-      const int s = p.m_s[b];
-      const int c0 = p.m_cu[b];
-      const int pos = s + (t - c0);
-      const int e = s + (p.m_cu[b + 1] - c0);
-      const int col = wrow + r;
-      if (score) v += __ldg(p.ape + (int64_t)(pos % p.ratio) * p.C + col);
+#pragma unroll
+      for (int q = 0; q < KSPLIT; ++q) v += sm.recv[q][t][r];
+      const int col = wrow + (int)(rank * 16) + r;
       p.proj[(int64_t)t * (2 * p.C) + (score ? p.C : 0) + col] = v;
-      if (pos >= tail_threshold(e, p.ratio, p.coff)) {
-        const int pr = table_row(p, score ? p.sc_tbl : p.kv_tbl, b, pos);
-        if (pr >= 0) (score ? p.score_state : p.kv_state)[((int64_t)pr * p.bs + pos % p.bs) * p.C + col] = v;
+      const int64_t so = score ? m.sc_off : m.kv_off;
+      if (so >= 0) {
+        if (score) v += __ldg(p.ape + (int64_t)m.ape_row * p.C + col);  // state: score + ape
+        (score ? p.score_state : p.kv_state)[so + col] = v;
       }
     }
   }
-  cluster_sync();  // peers may still be reading this CTA's partial
 
   if (warp == 1) {
     tc_fence_after();
@@ -228,14 +256,8 @@ cudaError_t launch_proj_decode(const Params& p, cudaStream_t s) {
     return cudaErrorInvalidValue;
   const size_t smem = sizeof(Smem) + 1024;
   static int configured[64] = {0};
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (dev >= 64 || !configured[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(proj_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)smem);
-    if (e != cudaSuccess) return e;
-    if (dev < 64) configured[dev] = 1;
-  }
+  const cudaError_t e = smem_attr_once(proj_decode_kernel, smem, configured);
+  if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(KSPLIT, (2 * p.C) / BM, 1);
   cfg.blockDim = dim3(kThreads, 1, 1);

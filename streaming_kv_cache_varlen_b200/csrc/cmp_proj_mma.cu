@@ -1,11 +1,11 @@
 // Dual projection with warp-level mma.sync (bf16 x bf16 -> fp32).
 //
-//   proj[t][n] = sum_k x[t][k] * W[n][k],  W = wkv (n < C) or wgate (n >= C),
-//   plus ape[p mod ratio][n - C] on the score columns
-// ("compressor torch_extension API", 计算公式 1-2), where p is the absolute
-// position of token t. The epilogue also writes the state tail rows
-// (positions p >= (e/ratio - coff + 1)*ratio of their sequence) into the paged
-// fp32 kv_state / score_state.
+//   proj[t][n] = sum_k x[t][k] * W[n][k],  W = wkv (n < C) or wgate (n >= C)
+// ("compressor torch_extension API", 计算公式 1-2). The epilogue also writes
+// the state tail rows (positions p >= (e/ratio - coff + 1)*ratio of their
+// sequence) into the paged fp32 kv_state / score_state, the score rows with
+// ape[p mod ratio] added (the pooling kernel adds ape to the projection rows
+// it reads, so the projection buffer holds raw scores).
 //
 // This is the portable tensor-core path (mma.sync runs on every architecture
 // since sm_80); the sm_100a tcgen05 kernel is the fast prefill path and this one
@@ -57,13 +57,13 @@ __device__ __forceinline__ void store_pair(const Params& p, int t, int n, float 
   }
   const bool score = n >= p.C;
   const int col = score ? n - p.C : n;
-  if (score && seq) {
-    const float2 a = *reinterpret_cast<const float2*>(p.ape + (int64_t)(pos % p.ratio) * p.C + col);
-    v0 += a.x;
-    v1 += a.y;
-  }
   *reinterpret_cast<float2*>(p.proj + (int64_t)t * (2 * p.C) + n) = make_float2(v0, v1);
   if (seq && pos >= thr) {
+    if (score) {  // the state holds score + ape
+      const float2 a = *reinterpret_cast<const float2*>(p.ape + (int64_t)(pos % p.ratio) * p.C + col);
+      v0 += a.x;
+      v1 += a.y;
+    }
     const int r = table_row(p, score ? p.sc_tbl : p.kv_tbl, b, pos);
     if (r >= 0) {
       float* st = score ? p.score_state : p.kv_state;
@@ -162,13 +162,9 @@ __global__ void __launch_bounds__(kThreads) proj_mma_kernel(Params p) {
 
 cudaError_t launch_proj_mma(const Params& p, cudaStream_t s) {
   const size_t smem = (size_t)STAGES * (BM + BN) * LDS * sizeof(__nv_bfloat16);
-  static bool configured = false;  // attribute is per function, same on every device
-  if (!configured) {
-    cudaError_t e = cudaFuncSetAttribute(proj_mma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)smem);
-    if (e != cudaSuccess) return e;
-    configured = true;
-  }
+  static int configured[64] = {0};
+  const cudaError_t e = smem_attr_once(proj_mma_kernel, smem, configured);
+  if (e != cudaSuccess) return e;
   dim3 grid((p.T + BM - 1) / BM, (2 * p.C) / BN);
   proj_mma_kernel<<<grid, kThreads, smem, s>>>(p);
   return cudaGetLastError();

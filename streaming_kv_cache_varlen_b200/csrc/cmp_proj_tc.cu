@@ -2,10 +2,10 @@
 // tcgen05.mma -> TMEM -> epilogue.
 //
 //   proj[t][n] = sum_k W[n][k] * x[t][k]   (W = wkv for n < C, wgate for n >= C)
-//   + ape[p mod ratio][n - C] on the score columns
-// ("compressor torch_extension API", 计算公式 1-2), and the state tail rows
-// (positions p >= (e/ratio - coff + 1)*ratio of their sequence) go straight
-// into the paged fp32 kv_state / score_state from the epilogue.
+// ("compressor torch_extension API", 计算公式 1-2), raw scores (the pooling
+// kernel adds ape[p mod ratio]); the state tail rows (positions
+// p >= (e/ratio - coff + 1)*ratio of their sequence, score rows with ape) go
+// straight into the paged fp32 kv_state / score_state from the epilogue.
 //
 // Layout of the contraction: the weight rows are the MMA's M side (128 rows of
 // wkv or wgate per tile) and the tokens its N side (256 per tile), so an
@@ -16,7 +16,7 @@
 //   warp 0     TMA producer: W tile 128x64 and x tile 256x64 per stage (48 KB)
 //   warp 1     owns TMEM (512 columns = two 256-column fp32 accumulators) and
 //              issues tcgen05.mma (M=128, N=256, K=16) from one thread
-//   warps 2-5  epilogue: tcgen05.ld, + ape, fp32 stores, tail-state stores
+//   warps 2-5  epilogue: tcgen05.ld, fp32 stores, tail-state stores (+ ape)
 // Four shared-memory stages; the two accumulators let the epilogue of one
 // tile overlap the main loop of the next. Every wait is bounded: a role that
 // gives up raises the CTA's abort flag and the device error word, and all
@@ -41,7 +41,7 @@ constexpr uint32_t kStageBytesB = BN * BK * 2;  // 32 KB
 constexpr uint32_t kIdesc = idesc_bf16_f32(BM, BN);
 
 struct TokInfo {
-  int32_t ape_row;   // position mod ratio, or -1 if the token belongs to no sequence
+  int32_t ape_row;   // position mod ratio (used on tail rows only)
   int32_t pad;
   int64_t kv_off;    // element offset of the token's kv_state row, or -1 (not a tail row)
   int64_t sc_off;    // element offset of the token's score_state row, or -1
@@ -52,6 +52,7 @@ struct Smem {
   __nv_bfloat16 a[STAGES][BM * BK];
   __nv_bfloat16 b[STAGES][BN * BK];
   TokInfo tok[2][BN];
+  uint32_t tail_mask[2][BN / 32];  // per 32-token chunk: which tokens are state tail rows
   uint64_t full[STAGES];
   uint64_t empty[STAGES];
   uint64_t acc_full[2];
@@ -62,9 +63,12 @@ struct Smem {
 
 __device__ __forceinline__ void epi_bar() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
 
-__device__ void fill_tok_info(const Params& p, TokInfo* info, int n0, int e_tid) {
+// Per-token facts of one tile, computed by the 128 epilogue threads while the
+// tile's main loop runs: which tokens are state tail rows and where they go.
+__device__ void fill_tok_info(const Params& p, TokInfo* info, uint32_t* tail_mask, int n0, int e_tid) {
   for (int j = e_tid; j < BN; j += 128) {
-    TokInfo ti{-1, 0, -1, -1};
+    TokInfo ti{0, 0, -1, -1};
+    bool tail = false;
     const int t = n0 + j;
     if (t < p.T) {
       const int b = upper_index(p.m_cu, p.B, t);
@@ -73,16 +77,19 @@ __device__ void fill_tok_info(const Params& p, TokInfo* info, int n0, int e_tid)
         const int c0 = p.m_cu[b];
         const int pos = s + (t - c0);
         const int e = s + (p.m_cu[b + 1] - c0);
-        ti.ape_row = pos % p.ratio;
         if (pos >= tail_threshold(e, p.ratio, p.coff)) {
+          ti.ape_row = pos % p.ratio;
           const int rk = table_row(p, p.kv_tbl, b, pos);
           const int rs = table_row(p, p.sc_tbl, b, pos);
           if (rk >= 0) ti.kv_off = ((int64_t)rk * p.bs + pos % p.bs) * p.C;
           if (rs >= 0) ti.sc_off = ((int64_t)rs * p.bs + pos % p.bs) * p.C;
+          tail = true;
         }
       }
     }
     info[j] = ti;
+    const unsigned m = __ballot_sync(0xffffffffu, tail);  // j = e_tid + 128 i: one warp = one chunk
+    if ((j & 31) == 0) tail_mask[j >> 5] = m;
   }
 }
 
@@ -181,7 +188,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int m0 = (tile % n_m) * BM;
       const int n0 = (tile / n_m) * BN;
       TokInfo* info = sm.tok[local & 1];
-      fill_tok_info(p, info, n0, e_tid);
+      uint32_t* tmask = sm.tail_mask[local & 1];
+      fill_tok_info(p, info, tmask, n0, e_tid);
       epi_bar();
       const int acc = local & 1;
       const uint32_t acc_phase = (local >> 1) & 1;
@@ -192,23 +200,30 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int col = (score ? m0 - p.C : m0) + row;  // channel within kv or score
       float* proj_col = p.proj + (score ? p.C : 0) + col;
       float* state = score ? p.score_state : p.kv_state;
-      const float* ape_col = p.ape + col;
       const uint32_t taddr = tmem + ((uint32_t)(quad * 32) << 16) + acc * BN;
 #pragma unroll 1
       for (int c = 0; c < BN / 32; ++c) {
         uint32_t r[32];
         tmem_ld32(taddr + c * 32, r);
         tmem_ld_wait(r);
+        const int t0 = n0 + c * 32;
+        const int jmax = p.T - t0;  // tokens past T are padding
+        float* dst = proj_col + (int64_t)t0 * (2 * p.C);
 #pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          const TokInfo ti = info[c * 32 + j];
-          if (ti.ape_row < 0) continue;  // past T, or the call was rejected
-          float v = __uint_as_float(r[j]);
-          if (score) v += __ldg(ape_col + (int64_t)ti.ape_row * p.C);
-          const int64_t t = n0 + c * 32 + j;
-          proj_col[t * (2 * p.C)] = v;
-          const int64_t so = score ? ti.sc_off : ti.kv_off;
-          if (so >= 0) state[so + col] = v;
+        for (int j = 0; j < 32; ++j)
+          if (j < jmax) dst[(int64_t)j * (2 * p.C)] = __uint_as_float(r[j]);
+        const uint32_t m = tmask[c];
+        if (m) {  // rare: state tail rows (score rows carry ape in the state)
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            if (m & (1u << j)) {
+              const TokInfo ti = info[c * 32 + j];
+              const int64_t so = score ? ti.sc_off : ti.kv_off;
+              float v = __uint_as_float(r[j]);
+              if (score) v += __ldg(p.ape + (int64_t)ti.ape_row * p.C + col);
+              if (so >= 0) state[so + col] = v;
+            }
+          }
         }
       }
       tc_fence_before();
@@ -279,13 +294,8 @@ cudaError_t launch_proj_tc(const Params& p, cudaStream_t s) {
     return cudaErrorInvalidValue;
   const size_t smem = sizeof(Smem) + 1024;
   static int configured[64] = {0};
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (dev >= 64 || !configured[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(proj_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    if (dev < 64) configured[dev] = 1;
-  }
+  const cudaError_t e = smem_attr_once(proj_tc_kernel, smem, configured);
+  if (e != cudaSuccess) return e;
   const int n_tiles = ((2 * p.C) / BM) * ((p.T + BN - 1) / BN);
   const int grid = n_tiles < sm_count() ? n_tiles : sm_count();
   proj_tc_kernel<<<grid, kThreads, smem, s>>>(mx, mkv, mg, p);
