@@ -161,6 +161,33 @@ CMP_API int cmp_compressor(const cmp_bf16* x, float* kv_state, float* score_stat
                    int32_t ratio, int32_t rope_head_dim, bool rotate, cmp_bf16* out,
                    void* stream, const cmp_dims* dims);
 
+/* No counterpart on the pages: an entry point for callers that must not
+ * allocate device memory at call time (for example a serving engine that
+ * reserves all device memory at start-up, or a caller running with the GPU
+ * nearly full, where a cudaMalloc could fail or synchronise the device).
+ *
+ * Same arguments and results as cmp_compressor, for decode-sized calls:
+ * T <= 64 tokens, and the call's scratch (error word, per-sequence metadata,
+ * fp32 projection rows: about 12*B + 8*T*coff*D bytes) must fit a fixed
+ * 1 MiB array in device memory that the library image carries; larger calls
+ * return CMP_ERR_INVALID before launching anything. It never calls cudaMalloc,
+ * cudaFree or any allocating routine.
+ *
+ * The first call on each device (with that device current) looks up the
+ * array's device address once (cudaGetSymbolAddress); make that first call
+ * before any stream capture. All calls on a device share the array, so calls
+ * that overlap on the GPU race and must be ordered by the caller (one stream,
+ * or events). The array keeps the last call's contents; each call clears the
+ * part that must start at zero. Device-side index errors of this variant are
+ * not reported through cmp_get_error. */
+CMP_API int cmp_compressor_noalloc(const cmp_bf16* x, float* kv_state, float* score_state,
+                                   const int32_t* kv_block_table, const int32_t* state_block_table,
+                                   const cmp_bf16* sin, const cmp_bf16* cos, const cmp_bf16* wkv,
+                                   const cmp_bf16* wgate, const float* ape, const cmp_bf16* norm_weight,
+                                   const cmp_bf16* hadamard, const int32_t* start_pos,
+                                   const int32_t* cu_seqlens, int32_t ratio, int32_t rope_head_dim,
+                                   bool rotate, cmp_bf16* out, void* stream, const cmp_dims* dims);
+
 /* Synchronises stream, then returns and clears the error word the kernels of
  * the current device set: CMP_OK, CMP_ERR_DEVICE_INDEX or CMP_ERR_TIMEOUT
  * (CMP_ERR_CUDA if the synchronisation itself fails). */

@@ -45,6 +45,8 @@ def _load() -> ctypes.CDLL:
         "cmp_out_row_layout": (ctypes.c_int, [P, P, I32, I32, I64, P, P]),
         "cmp_compressor": (ctypes.c_int, [P] * 14 + [I32, I32, ctypes.c_bool, P, P,
                                                    ctypes.POINTER(cmp_dims)]),
+        "cmp_compressor_noalloc": (ctypes.c_int, [P] * 14 + [I32, I32, ctypes.c_bool, P, P,
+                                                           ctypes.POINTER(cmp_dims)]),
         "cmp_get_error": (ctypes.c_int, [P]),
         "cmp_workspace_size": (SZ, [ctypes.POINTER(cmp_dims), I32]),
         "cmp_release_workspaces": (ctypes.c_int, []),
