@@ -70,13 +70,22 @@ def barrier(ws):
 
 
 def max_over_ranks(v: float, ws: int) -> float:
+    """The max of v over all ranks (the job's time is its slowest rank's)."""
     if ws == 1:
         return v
     import torch
     import torch.distributed as dist
-    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([v], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def job_throughput(units_per_rank: float, ws: int, ms_this_rank: float) -> float:
+    """Whole-job units per second: every rank processes units_per_rank in the timed
+    region (weak scaling), the region lasts as long as the slowest rank."""
+    ms = max_over_ranks(ms_this_rank, ws)
+    return units_per_rank * ws / (ms / 1e3)
 
 
 # ----------------------------------------------------------------------------
@@ -279,14 +288,15 @@ def bench_prefill(args, ws, local, stream, peaks, peak_src):
     value = PREFILL["T"] * ws * args.steps / (ms / 1e3)
 
     # dominant kernel: the projection (a dense bf16 contraction)
-    proj_name = max(("proj_tcgen05", "proj_mma_sync", "proj_decode"), key=lambda k: prof[k][0])
+    proj_name = max(("proj_tcgen05", "proj_mma_sync", "proj_decode", "fused_tcgen05"),
+                    key=lambda k: prof[k][0])
     p_ms, p_n = prof[proj_name]
     T, H, C = PREFILL["T"], PREFILL["H"], PREFILL["D"]
     flops = 2.0 * T * H * 2 * C
     achieved = flops / (p_ms / p_n / 1e3) / 1e12 if p_n else None
     peak = peaks["bf16_tflops"]
     kfile = {"proj_tcgen05": "cmp_proj_tc.cu", "proj_mma_sync": "cmp_proj_mma.cu",
-             "proj_decode": "cmp_proj_decode.cu"}[proj_name]
+             "proj_decode": "cmp_proj_decode.cu", "fused_tcgen05": "cmp_fused_tc.cu"}[proj_name]
     roofline = {"kernel": proj_name, "bound": "tensor", "achieved": achieved, "peak": peak,
                 "unit": "TFLOP/s", "frac": achieved / peak if achieved else None,
                 "traffic": traffic_for(kfile, proj_name, T / 131072.0),

@@ -125,8 +125,10 @@ CMP_API int cmp_out_row_layout(const int32_t* cu_seqlens, const int32_t* start_p
  *  hadamard           device bf16 [D, D] (out = out @ hadamard); NULL iff !rotate
  *  start_pos          device int32 [B]; NULL means every sequence starts at 0
  *  cu_seqlens         device int32 [B+1], rising from 0 to T
- *  ratio              tokens per window: 2, 4, 8, 16, 32, 64 or 128;
- *                     coff = 2 for ratio 4, else 1
+ *  ratio              tokens per window: 1, 2, 4, 8, 16, 32, 64 or 128;
+ *                     coff = 2 for ratio 4, else 1 (ratio 1: every token is
+ *                     its own window, so only projection and normalisation
+ *                     remain, as the Triton-Ascend Compressor article notes)
  *  rope_head_dim      64 (the only value the pages support)
  *  rotate             apply the hadamard product
  *  out                device bf16 [n_out, D], n_out = cmp_out_rows(B, T, ratio);
@@ -213,7 +215,9 @@ enum {
   CMP_KERNEL_PROJ_MMA = 2,     /* projection, warp-level mma.sync */
   CMP_KERNEL_PROJ_DECODE = 3,  /* small-T projection streaming the weights */
   CMP_KERNEL_POOL = 4,         /* pooling + RMSNorm + RoPE + Hadamard + store */
-  CMP_KERNEL_COUNT = 5
+  CMP_KERNEL_FUSED = 5,        /* prefill projection with the pooling in its epilogue */
+  CMP_KERNEL_FINISH = 6,       /* fused path: merge halves + RMSNorm + RoPE + Hadamard */
+  CMP_KERNEL_COUNT = 7
 };
 
 /* Name of a kernel id (NULL if out of range). */
@@ -231,10 +235,12 @@ CMP_API int cmp_profile_start(void);
  * launches[CMP_KERNEL_COUNT] (host arrays; either may be NULL). */
 CMP_API int cmp_profile_stop(double* ms, int64_t* launches);
 
-/* Testing knob: which projection kernel prefill calls use. 0 = automatic
- * (tcgen05 kernel for large T, weight-streaming kernel for small T), 1 = force
- * the mma.sync kernel, 2 = force the tcgen05 kernel, 3 = force the
- * weight-streaming kernel. Returns the previous value, or -1 if out of range. */
+/* Testing knob: which path calls take. 0 = automatic (weight streaming for
+ * T <= 64; the fused tcgen05 pooling kernel for long sequences, T >= 1024 and
+ * T >= 256*B; else the tcgen05 projection + pooling kernel), 1 = force the
+ * mma.sync projection, 2 = the tcgen05 projection, 3 = weight streaming,
+ * 4 = the fused path. A forced path a call cannot take falls back to 1.
+ * Returns the previous value, or -1 if out of range. */
 CMP_API int cmp_set_proj_kernel(int which);
 
 #ifdef __cplusplus

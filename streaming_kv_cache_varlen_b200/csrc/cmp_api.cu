@@ -25,10 +25,12 @@ using cmp::Params;
 // ---- workspace ---------------------------------------------------------------
 
 struct WsLayout {
-  size_t err, m_cu, m_s, m_off, proj, total;
+  size_t err, m_cu, m_s, m_off, m_tile, proj, ystat, ylse, total;
 };
 
-WsLayout ws_layout(int64_t B, int64_t T, int64_t C) {
+// fused: the pooled-halves buffers of the fused path instead of the fp32
+// projection rows of the other paths.
+WsLayout ws_layout(int64_t B, int64_t T, int64_t C, int64_t n_out, bool fused) {
   WsLayout L{};
   size_t o = 0;
   auto take = [&](size_t n) {
@@ -40,9 +42,40 @@ WsLayout ws_layout(int64_t B, int64_t T, int64_t C) {
   L.m_cu = take(sizeof(int32_t) * (B + 1));
   L.m_s = take(sizeof(int32_t) * std::max<int64_t>(B, 1));
   L.m_off = take(sizeof(int32_t) * (B + 1));
-  L.proj = take(sizeof(float) * (size_t)T * 2 * C);
+  L.m_tile = take(fused ? sizeof(int32_t) * (B + 1) : 0);
+  L.proj = take(fused ? 0 : sizeof(float) * (size_t)T * 2 * C);
+  L.ystat = take(fused ? sizeof(float) * (size_t)std::max<int64_t>(n_out, 1) * C : 0);
+  L.ylse = take(fused ? sizeof(float) * (size_t)std::max<int64_t>(n_out, 1) * C : 0);
   L.total = o;
   return L;
+}
+
+// Which projection path a call takes: 1 mma.sync, 2 tcgen05 (+ pooling kernel),
+// 3 small-T weight streaming (+ pooling kernel), 4 fused tcgen05 pooling
+// (+ finish kernel).
+int choose_path(const Params& p, int forced) {
+  int which = forced;
+  if (which == 0) {
+    if (cmp::proj_decode_supported(p)) which = 3;
+    else if (cmp::fused_supported(p) && p.T >= 1024 && (int64_t)p.T >= 256LL * p.B) which = 4;
+    else if (cmp::proj_tc_supported(p)) which = 2;
+    else which = 1;
+  }
+  if (which == 2 && !cmp::proj_tc_supported(p)) which = 1;
+  if (which == 3 && !cmp::proj_decode_supported(p)) which = 1;
+  if (which == 4 && !cmp::fused_supported(p)) which = 1;
+  return which;
+}
+
+int sm_count_cached() {
+  static int counts[64] = {0};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 64 && counts[dev]) return counts[dev];
+  int n = 148;
+  cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+  if (dev < 64) counts[dev] = n;
+  return n;
 }
 
 struct Workspace {
@@ -134,7 +167,7 @@ int get_workspace(cudaStream_t s, size_t need, unsigned char** out) {
 }
 
 bool valid_ratio(int r) {
-  return r == 2 || r == 4 || r == 8 || r == 16 || r == 32 || r == 64 || r == 128;
+  return r == 1 || r == 2 || r == 4 || r == 8 || r == 16 || r == 32 || r == 64 || r == 128;
 }
 
 bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
@@ -188,7 +221,6 @@ int cmp_out_row_layout(const int32_t* cu_seqlens, const int32_t* start_pos, int3
 size_t cmp_workspace_size(const cmp_dims* dims, int32_t ratio) {
   if (check_dims(dims) != CMP_OK || !valid_ratio(ratio)) return 0;
   const int coff = ratio == 4 ? 2 : 1;
-  size_t base = ws_layout(dims->B, dims->T, (int64_t)coff * dims->D).total;
   Params p{};
   p.B = dims->B;
   p.T = dims->T;
@@ -197,7 +229,9 @@ size_t cmp_workspace_size(const cmp_dims* dims, int32_t ratio) {
   p.C = coff * dims->D;
   p.coff = coff;
   p.ratio = ratio;
-  return base + cmp::proj_decode_workspace(p);
+  const int which = choose_path(p, g_proj_kernel.load());
+  return ws_layout(dims->B, dims->T, p.C, cmp_out_rows(p.B, p.T, ratio), which == 4).total +
+         cmp::proj_decode_workspace(p);
 }
 
 int cmp_release_workspaces(void) {
@@ -274,7 +308,9 @@ int cmp_compressor(const cmp_bf16* x, float* kv_state, float* score_state,
   p.stride = dims->table_stride;
   p.n_out = (int)cmp_out_rows(p.B, p.T, ratio);
 
-  const WsLayout L = ws_layout(p.B, p.T, p.C);
+  const int which = choose_path(p, g_proj_kernel.load());
+  const bool fused = which == 4;
+  const WsLayout L = ws_layout(p.B, p.T, p.C, p.n_out, fused);
   const size_t extra = cmp::proj_decode_workspace(p);
   unsigned char* ws = nullptr;
   rc = get_workspace(s, L.total + extra, &ws);
@@ -283,20 +319,23 @@ int cmp_compressor(const cmp_bf16* x, float* kv_state, float* score_state,
   p.m_cu = reinterpret_cast<int32_t*>(ws + L.m_cu);
   p.m_s = reinterpret_cast<int32_t*>(ws + L.m_s);
   p.m_off = reinterpret_cast<int32_t*>(ws + L.m_off);
-  p.proj = reinterpret_cast<float*>(ws + L.proj);
+  p.m_tile = fused ? reinterpret_cast<int32_t*>(ws + L.m_tile) : nullptr;
+  p.proj = fused ? nullptr : reinterpret_cast<float*>(ws + L.proj);
+  p.ystat = fused ? reinterpret_cast<float*>(ws + L.ystat) : nullptr;
+  p.ylse = fused ? reinterpret_cast<float*>(ws + L.ylse) : nullptr;
 
   // ---- kernels ----
   if (launch(CMP_KERNEL_SCHED, s, [&] { return cmp::launch_sched(p, s); }) != cudaSuccess)
     return CMP_ERR_CUDA;
-  int which = g_proj_kernel.load();
-  if (which == 0) {
-    if (cmp::proj_decode_supported(p)) which = 3;
-    else if (cmp::proj_tc_supported(p)) which = 2;
-    else which = 1;
-  }
-  if (which == 2 && !cmp::proj_tc_supported(p)) which = 1;
-  if (which == 3 && !cmp::proj_decode_supported(p)) which = 1;
   cudaError_t e;
+  if (fused) {
+    const int sms = sm_count_cached();
+    e = launch(CMP_KERNEL_FUSED, s, [&] { return cmp::launch_fused(p, s, sms); });
+    if (e != cudaSuccess) return CMP_ERR_CUDA;
+    if (launch(CMP_KERNEL_FINISH, s, [&] { return cmp::launch_finish(p, s); }) != cudaSuccess)
+      return CMP_ERR_CUDA;
+    return CMP_OK;
+  }
   if (which == 2)
     e = launch(CMP_KERNEL_PROJ_TC, s, [&] { return cmp::launch_proj_tc(p, s); });
   else if (which == 3)
@@ -350,8 +389,9 @@ const char* cmp_status_string(int status) {
 }
 
 const char* cmp_kernel_name(int kernel) {
-  static const char* names[CMP_KERNEL_COUNT] = {"sched", "proj_tcgen05", "proj_mma_sync",
-                                                "proj_decode", "pool_epilogue"};
+  static const char* names[CMP_KERNEL_COUNT] = {"sched",         "proj_tcgen05", "proj_mma_sync",
+                                                "proj_decode",   "pool_epilogue", "fused_tcgen05",
+                                                "finish"};
   return (kernel >= 0 && kernel < CMP_KERNEL_COUNT) ? names[kernel] : nullptr;
 }
 
@@ -392,7 +432,7 @@ int cmp_profile_stop(double* ms, int64_t* launches) {
 }
 
 int cmp_set_proj_kernel(int which) {
-  if (which < 0 || which > 3) return -1;
+  if (which < 0 || which > 4) return -1;
   return g_proj_kernel.exchange(which);
 }
 

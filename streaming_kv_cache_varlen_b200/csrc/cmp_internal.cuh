@@ -5,6 +5,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <utility>
+
 #include "cmp.h"
 
 namespace cmp {
@@ -41,7 +43,10 @@ struct Params {
   int32_t* m_cu;   // [B+1] validated token offsets (all 0 when the call is rejected)
   int32_t* m_s;    // [B]   start positions
   int32_t* m_off;  // [B+1] first output row of each sequence
-  float* proj;     // [T, 2C]: kv in columns [0, C), score (with ape) in [C, 2C)
+  float* proj;     // [T, 2C]: kv in columns [0, C), raw score in [C, 2C) (non-fused paths)
+  int32_t* m_tile; // [B+1] first fused work tile of each sequence (fused path), else null
+  float* ystat;    // [n_out, coff, D] pooled halves (fused path)
+  float* ylse;     // [n_out, coff, D] log-sum-exp of each half's scores (fused path, coff = 2)
 };
 
 // Largest b in [0, n] with a[b] <= v, for a non-decreasing a[0..n] with a[0] <= v.
@@ -77,6 +82,44 @@ __device__ __forceinline__ int tail_threshold(int e, int ratio, int coff) {
   return (e / ratio - coff + 1) * ratio;
 }
 
+// Programmatic dependent launch. A kernel launched with launch_chained may start
+// while the kernel before it in the stream is still running; it must call
+// pdl_wait() before it touches anything that kernel (or an earlier one of the
+// same call) writes, and may read the call's inputs before that. pdl_trigger()
+// lets the next kernel of the chain be scheduled early. Without the launch
+// attribute both are no-ops.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// Launch `kernel` on `s` as a programmatic dependent of the previous launch in
+// the stream, optionally as clusters of cluster_x CTAs.
+template <class... KArgs, class... Args>
+inline cudaError_t launch_chained(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                                  cudaStream_t s, int cluster_x, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[2];
+  int n = 0;
+  attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[n].val.programmaticStreamSerializationAllowed = 1;
+  ++n;
+  if (cluster_x > 1) {
+    attr[n].id = cudaLaunchAttributeClusterDimension;
+    attr[n].val.clusterDim.x = cluster_x;
+    attr[n].val.clusterDim.y = 1;
+    attr[n].val.clusterDim.z = 1;
+    ++n;
+  }
+  cfg.attrs = attr;
+  cfg.numAttrs = n;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
 // Raise a kernel's dynamic shared-memory limit once per device (the attribute
 // belongs to the function on the current device).
 template <class K>
@@ -94,5 +137,9 @@ inline cudaError_t smem_attr_once(K* kernel, size_t bytes, int (&done)[64]) {
 cudaError_t launch_sched(const Params& p, cudaStream_t s);
 cudaError_t launch_proj_mma(const Params& p, cudaStream_t s);
 cudaError_t launch_pool(const Params& p, cudaStream_t s);
+cudaError_t launch_finish(const Params& p, cudaStream_t s);
+cudaError_t launch_fused(const Params& p, cudaStream_t s, int sm_count);
+bool fused_supported(const Params& p);
+constexpr int kFusedTile = 256;  // positions per fused work tile
 
 }  // namespace cmp

@@ -75,7 +75,7 @@ int scratch_address(unsigned char** out) {
   return CMP_OK;
 }
 
-bool ratio_ok(int r) { return r == 2 || r == 4 || r == 8 || r == 16 || r == 32 || r == 64 || r == 128; }
+bool ratio_ok(int r) { return r == 1 || r == 2 || r == 4 || r == 8 || r == 16 || r == 32 || r == 64 || r == 128; }
 
 bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 

@@ -19,11 +19,10 @@
 //  * bf16 round-to-nearest-even store. Rows that hold no window are stored as 0
 //    ("CANN PyPTO 算子实战", 返回值说明).
 #include "cmp_internal.cuh"
+#include "cmp_rowpost.cuh"
 
 namespace cmp {
 namespace {
-
-constexpr float kRmsEps = 1e-6f;
 
 __device__ __forceinline__ float4 ld4(const float* p) { return *reinterpret_cast<const float4*>(p); }
 
@@ -47,17 +46,33 @@ struct RowSrc {
 };
 
 constexpr int kMaxRows = 256;  // coff * ratio <= 256
+constexpr int kMaxStagedSeqs = 256;
 
 __global__ void __launch_bounds__(128) pool_kernel(Params p) {
   __shared__ float red[32];
   __shared__ float zs[512];
   __shared__ RowSrc src[kMaxRows];
+  __shared__ int32_t off_s[kMaxStagedSeqs + 1];
   const int n = blockIdx.x;
   const int D = p.D, C = p.C, r = p.ratio;
   const int c = threadIdx.x * 4;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
+  pdl_wait();  // everything below reads what the earlier kernels of the call wrote
 
-  const int b = upper_index(p.m_off, p.B, n);
+  // which sequence owns row n (search the row offsets; staged when B is small)
+  int b;
+  if (p.B <= kMaxStagedSeqs) {
+    for (int i = threadIdx.x; i <= p.B; i += blockDim.x) off_s[i] = p.m_off[i];
+    __syncthreads();
+    int lo = 0, hi = p.B;
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (off_s[mid] <= n) lo = mid; else hi = mid - 1;
+    }
+    b = lo;
+  } else {
+    b = upper_index(p.m_off, p.B, n);
+  }
   int w = -1, s = 0, cu = 0;
   if (b < p.B) {
     s = p.m_s[b];
@@ -138,71 +153,14 @@ __global__ void __launch_bounds__(128) pool_kernel(Params p) {
 #pragma unroll
   for (int i = 0; i < 4; ++i) y[i] = l[i] > 0.f ? a[i] / l[i] : 0.f;
 
-  // RMSNorm over the D channels of the row
-  float ss = y[0] * y[0] + y[1] * y[1] + y[2] * y[2] + y[3] * y[3];
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-  if (lane == 0) red[warp] = ss;
-  __syncthreads();
-  float tot = 0.f;
-  for (int i = 0; i < nwarps; ++i) tot += red[i];
-  const float inv = rsqrtf(tot / (float)D + kRmsEps);
-  const uint2 wraw = *reinterpret_cast<const uint2*>(p.norm_w + c);
-  const __nv_bfloat162 w01 = *reinterpret_cast<const __nv_bfloat162*>(&wraw.x);
-  const __nv_bfloat162 w23 = *reinterpret_cast<const __nv_bfloat162*>(&wraw.y);
-  float z[4] = {y[0] * inv * __low2float(w01), y[1] * inv * __high2float(w01),
-                y[2] * inv * __low2float(w23), y[3] * inv * __high2float(w23)};
-
-  // interleaved RoPE on the last rope channels
-  const int r0 = D - p.rope;
-  if (c >= r0) {
-    const int half = p.rope / 2;
-    const __nv_bfloat16* cs = p.cos + (int64_t)n * p.rope;
-    const __nv_bfloat16* sn = p.sin + (int64_t)n * p.rope;
-#pragma unroll
-    for (int i = 0; i < 4; i += 2) {
-      const int j = (c + i - r0) >> 1;
-      const float ce = __bfloat162float(cs[j]), se = __bfloat162float(sn[j]);
-      const float co = __bfloat162float(cs[half + j]), so = __bfloat162float(sn[half + j]);
-      const float ev = z[i], od = z[i + 1];
-      z[i] = ev * ce - od * se;
-      z[i + 1] = od * co + ev * so;
-    }
-  }
-
-  if (p.rotate) {  // out = z @ hadamard (dense product, any D x D matrix)
-#pragma unroll
-    for (int i = 0; i < 4; ++i) zs[c + i] = z[i];
-    __syncthreads();
-    float o[4] = {0.f, 0.f, 0.f, 0.f};
-    for (int k = 0; k < D; ++k) {
-      const float zk = zs[k];
-      const uint2 hr = *reinterpret_cast<const uint2*>(p.had + (int64_t)k * D + c);
-      const __nv_bfloat162 h01 = *reinterpret_cast<const __nv_bfloat162*>(&hr.x);
-      const __nv_bfloat162 h23 = *reinterpret_cast<const __nv_bfloat162*>(&hr.y);
-      o[0] = fmaf(zk, __low2float(h01), o[0]);
-      o[1] = fmaf(zk, __high2float(h01), o[1]);
-      o[2] = fmaf(zk, __low2float(h23), o[2]);
-      o[3] = fmaf(zk, __high2float(h23), o[3]);
-    }
-#pragma unroll
-    for (int i = 0; i < 4; ++i) z[i] = o[i];
-  }
-
-  __nv_bfloat162 o01 = __floats2bfloat162_rn(z[0], z[1]);
-  __nv_bfloat162 o23 = __floats2bfloat162_rn(z[2], z[3]);
-  uint2 v;
-  v.x = *reinterpret_cast<uint32_t*>(&o01);
-  v.y = *reinterpret_cast<uint32_t*>(&o23);
-  *dst = v;
+  finish_row(p, n, c, y, red, zs);
 }
 
 }  // namespace
 
 cudaError_t launch_pool(const Params& p, cudaStream_t s) {
   if (p.n_out <= 0) return cudaSuccess;
-  pool_kernel<<<p.n_out, p.D / 4, 0, s>>>(p);
-  return cudaGetLastError();
+  return launch_chained(pool_kernel, dim3(p.n_out), dim3(p.D / 4), 0, s, 1, p);
 }
 
 }  // namespace cmp

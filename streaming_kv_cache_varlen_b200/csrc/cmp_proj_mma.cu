@@ -75,6 +75,8 @@ __device__ __forceinline__ void store_pair(const Params& p, int t, int n, float 
 
 __global__ void __launch_bounds__(kThreads) proj_mma_kernel(Params p) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
+  pdl_wait();
+  pdl_trigger();
   __nv_bfloat16* As = reinterpret_cast<__nv_bfloat16*>(smem_raw);
   __nv_bfloat16* Bs = As + STAGES * BM * LDS;
 
@@ -166,8 +168,7 @@ cudaError_t launch_proj_mma(const Params& p, cudaStream_t s) {
   const cudaError_t e = smem_attr_once(proj_mma_kernel, smem, configured);
   if (e != cudaSuccess) return e;
   dim3 grid((p.T + BM - 1) / BM, (2 * p.C) / BN);
-  proj_mma_kernel<<<grid, kThreads, smem, s>>>(p);
-  return cudaGetLastError();
+  return launch_chained(proj_mma_kernel, grid, dim3(kThreads), smem, s, 1, p);
 }
 
 }  // namespace cmp

@@ -127,9 +127,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = sm.tmem_base;
   volatile int* abort = &sm.abort;
+  pdl_trigger();
 
   if (warp == 0) {
-    // ---------------- TMA producer ----------------
+    // ---------------- TMA producer (x and the weights are call inputs) ----------------
     if (lane == 0) {
       int stage = 0;
       uint32_t phase = 0;
@@ -180,6 +181,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {
     // ---------------- epilogue (warps 2..5) ----------------
+    pdl_wait();  // reads the scheduler's metadata, writes proj and the state
     const int e_tid = threadIdx.x - 64;
     const int quad = warp & 3;            // TMEM lanes this warp may access
     const int row = quad * 32 + lane;     // weight row within the tile = TMEM lane
@@ -298,8 +300,7 @@ cudaError_t launch_proj_tc(const Params& p, cudaStream_t s) {
   if (e != cudaSuccess) return e;
   const int n_tiles = ((2 * p.C) / BM) * ((p.T + BN - 1) / BN);
   const int grid = n_tiles < sm_count() ? n_tiles : sm_count();
-  proj_tc_kernel<<<grid, kThreads, smem, s>>>(mx, mkv, mg, p);
-  return cudaGetLastError();
+  return launch_chained(proj_tc_kernel, dim3(grid), dim3(kThreads), smem, s, 1, mx, mkv, mg, p);
 }
 
 }  // namespace cmp

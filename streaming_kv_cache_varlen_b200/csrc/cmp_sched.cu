@@ -46,6 +46,7 @@ __global__ void __launch_bounds__(kThreads) sched_kernel(Params p) {
   __shared__ int bad;
   __shared__ int warp_tot[32];
   __shared__ int chunk_total;
+  pdl_trigger();  // the projection kernel may start streaming its inputs now
   if (threadIdx.x == 0) bad = 0;
   __syncthreads();
   const int B = p.B;
@@ -65,29 +66,37 @@ __global__ void __launch_bounds__(kThreads) sched_kernel(Params p) {
   __syncthreads();
   const bool rejected = bad != 0;
   if (rejected && threadIdx.x == 0) atomicOr(p.err, kErrIndex);
-  // 2) metadata; a rejected call gets empty sequences (every output row 0)
-  int carry = 0;
+  // 2) metadata; a rejected call gets empty sequences (every output row 0).
+  // Fused path: sequence b's work tiles cover positions from its first
+  // window's start (start_pos rounded down to the ratio) to its end.
+  int carry = 0, tcarry = 0;
   for (int base = 0; base < B; base += kThreads) {
     const int b = base + threadIdx.x;
-    int c = 0, s = 0, cap = 0;
+    int c = 0, s = 0, cap = 0, tiles = 0;
     if (b < B && !rejected) {
       c = p.cu_in[b];
       const int L = p.cu_in[b + 1] - c;
       s = p.start_pos ? p.start_pos[b] : 0;
       cap = min(L, L / p.ratio + 1);
+      if (L > 0) tiles = (s + L - (s / p.ratio) * p.ratio + kFusedTile - 1) / kFusedTile;
     }
     const int ex = block_exclusive_scan(cap, warp_tot, &chunk_total);
+    const int cap_total = chunk_total;
+    const int tex = block_exclusive_scan(tiles, warp_tot, &chunk_total);
     if (b < B) {
       p.m_cu[b] = c;
       p.m_s[b] = s;
       p.m_off[b] = carry + ex;
+      if (p.m_tile) p.m_tile[b] = tcarry + tex;
     }
-    carry += chunk_total;
+    carry += cap_total;
+    tcarry += chunk_total;
     __syncthreads();
   }
   if (threadIdx.x == 0) {
     p.m_cu[B] = rejected ? 0 : p.T;
     p.m_off[B] = carry;
+    if (p.m_tile) p.m_tile[B] = tcarry;
   }
 }
 

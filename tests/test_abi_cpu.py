@@ -122,5 +122,5 @@ def test_workspace_size(cmp):
     small = cmp.workspace_size(1, 64, 1024, 128, 4, 16, 4, 4)
     big = cmp.workspace_size(1, 131072, 4096, 512, 1024, 128, 1024, 128)
     assert 0 < small < big
-    assert big >= 131072 * 2 * 512 * 4          # fp32 projection rows of one call
+    assert big >= 1025 * 512 * 4                # at least the pooled rows of one call
     assert cmp.workspace_size(1, 64, 1000, 128, 4, 16, 4, 4) == 0

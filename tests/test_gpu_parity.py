@@ -35,7 +35,7 @@ def check(cmp, inp, rows=None):
     return out, kv, sc, res
 
 
-@pytest.fixture(params=[0, 1, 2, 3], ids=["auto", "mma", "tcgen05", "decode"])
+@pytest.fixture(params=[0, 1, 2, 3, 4], ids=["auto", "mma", "tcgen05", "decode", "fused"])
 def proj_kernel(request, lib):
     prev = lib.set_proj_kernel(request.param)
     yield request.param
@@ -123,7 +123,7 @@ def test_pypto_example_cases(lib, case, shift):
     check(lib, with_rope(inp))
 
 
-@pytest.mark.parametrize("ratio", [2, 8, 16, 32, 64])
+@pytest.mark.parametrize("ratio", [1, 2, 8, 16, 32, 64])
 def test_other_ratios(lib, ratio, proj_kernel):
     rng = np.random.default_rng(ratio)
     L = rng.integers(0, 5 * ratio, size=5).tolist()
@@ -150,13 +150,35 @@ EDGE_CASES = {
 }
 
 
+@pytest.fixture(params=[0, 4], ids=["auto", "fused"])
+def auto_or_fused(request, lib):
+    prev = lib.set_proj_kernel(request.param)
+    yield request.param
+    lib.set_proj_kernel(prev)
+
+
 @pytest.mark.parametrize("name", sorted(EDGE_CASES))
-def test_edge_cases(lib, name):
+def test_edge_cases(lib, name, auto_or_fused):
     c = dict(EDGE_CASES[name])
     ratio = c.pop("ratio")
     bs = c.pop("bs")
     inp = make_inputs(name=name, seed=11, coff=2 if ratio == 4 else 1, ratio=ratio, block_size=bs,
                       rotate=c["D"] == 128, **c)
+    check(lib, with_rope(inp))
+
+
+@pytest.mark.parametrize("ratio", [4, 128])
+def test_fused_path_history_and_tails(lib, ratio, auto_or_fused):
+    """Windows that straddle start_pos (rows from the paged state), tails, zero-length
+    sequences and several sequences per tile row, on the fused path."""
+    rng = np.random.default_rng(ratio + 5)
+    B = 6
+    L = [int(v) for v in rng.integers(ratio, 3 * 256, size=B)]
+    L[2] = 0
+    sp = [int(v) for v in rng.integers(0, 2 * ratio, size=B)]
+    inp = make_inputs(name="fh", seed=ratio, lengths=L, start_pos=sp, H=1024,
+                      D=512 if ratio == 128 else 128, coff=2 if ratio == 4 else 1, ratio=ratio,
+                      block_size=64, rotate=ratio == 4)
     check(lib, with_rope(inp))
 
 
@@ -198,7 +220,7 @@ def test_projection_kernels_agree(lib):
                                 H=4096, D=512, coff=2, ratio=4, block_size=128, rotate=False))
     res = run_inputs(inp)
     outs = {}
-    for k in (1, 2, 3):
+    for k in (1, 2, 3, 4):
         prev = lib.set_proj_kernel(k)
         try:
             o, kv, sc, err = run(lib, inp)

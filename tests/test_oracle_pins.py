@@ -193,6 +193,18 @@ def test_one_dominant_score_selects_its_row(ratio):
         assert np.allclose(res.pooled[row], ref, rtol=1e-12, atol=1e-12)
 
 
+def test_ratio1_pools_each_token_alone():
+    # r = 1: every token is its own window, the one-row softmax weight is 1, so the
+    # pooled row is the token's kv row ("Triton-Ascend Compressor": with r = 1 only
+    # the feature projection and the normalisation remain)
+    inp = tiny([5, 3], [7, 0], ratio=1, D=8, H=16)
+    res = run_inputs(inp)
+    kv, _ = oracle.compressor.project(inp.x, inp.wkv, inp.wgate, inp.ape, [7, 8, 9, 10, 11, 0, 1, 2], 1)
+    assert [r for r, _, _ in res.layout.rows] == list(range(8))
+    assert np.array_equal(res.pooled, kv.astype(np.float64))
+    assert not res.written.any()            # nothing is left for a later call
+
+
 def test_first_c4a_window_ignores_previous_half():
     inp, cols, _ = _equal_score_case(4, 8)
     res = run_inputs(inp)
