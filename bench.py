@@ -369,14 +369,20 @@ def bench_decode(args, ws, local, stream, peaks, peak_src):
     torch.cuda.synchronize()
     n = 50
     g_call, g_flush = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
-    with torch.cuda.graph(g_call, stream=side):
-        for _ in range(n):
-            flush.fill_(1)
-            cmp.compressor(**dec, out=dout)
-    with torch.cuda.graph(g_flush, stream=side):
-        for _ in range(n):
-            flush.fill_(1)
-    torch.cuda.synchronize()
+    try:
+        with torch.cuda.graph(g_call, stream=side):
+            for _ in range(n):
+                flush.fill_(1)
+                cmp.compressor(**dec, out=dout)
+        with torch.cuda.graph(g_flush, stream=side):
+            for _ in range(n):
+                flush.fill_(1)
+        torch.cuda.synchronize()
+        graphs = True
+    except Exception as exc:  # noqa: BLE001 - report eager timing instead
+        torch.cuda.synchronize()
+        graphs = False
+        graph_error = str(exc).splitlines()[0][:200]
 
     def replay(g):
         best = None
@@ -392,9 +398,10 @@ def bench_decode(args, ws, local, stream, peaks, peak_src):
         return best
 
     barrier(ws)
-    t_call, t_flush = replay(g_call), replay(g_flush)
-    assert cmp.get_error(side) == 0
-    dec_us = max_over_ranks((t_call - t_flush) * 1e3 / n, ws)
+    if graphs:
+        t_call, t_flush = replay(g_call), replay(g_flush)
+        assert cmp.get_error(side) == 0
+        dec_us = max_over_ranks((t_call - t_flush) * 1e3 / n, ws)
     del g_call, g_flush
 
     # eager: events around each call from Python (host overhead included)
@@ -410,10 +417,15 @@ def bench_decode(args, ws, local, stream, peaks, peak_src):
     torch.cuda.synchronize()
     dprof = cmp.profile_stop()
     eager = statistics.median(a.elapsed_time(b) * 1e3 for a, b in times)
+    if graphs:
+        timing = "CUDA-graph replay of 50 x (L2 flush + call) minus 50 flushes, / 50"
+    else:
+        dec_us = max_over_ranks(eager, ws)
+        timing = f"eager events around each call (graph capture failed: {graph_error})"
     ach = dec_bytes / (dec_us / 1e6) / 1e9
     return {"workload": "c4a_decode: 32 requests x 1 token, H=4096, D=512, ratio 4",
             "us_per_call": dec_us, "us_per_call_eager": eager, "calls": n,
-            "timing": "CUDA-graph replay of 50 x (L2 flush + call) minus 50 flushes, / 50",
+            "timing": timing,
             "roofline": {"bound": "hbm", "achieved": ach, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                          "frac": ach / peaks["hbm_gbs"], "algorithmic_bytes_per_call": dec_bytes,
                          "peak_source": peak_src},

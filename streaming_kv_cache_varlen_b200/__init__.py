@@ -20,7 +20,7 @@ CMP_OK = 0
 STATUS = {0: "CMP_OK", 1: "CMP_ERR_NULLPTR", 2: "CMP_ERR_INVALID", 3: "CMP_ERR_UNSUPPORTED",
           4: "CMP_ERR_CUDA", 5: "CMP_ERR_DEVICE_INDEX", 6: "CMP_ERR_TIMEOUT"}
 KERNELS = ("sched", "proj_tcgen05", "proj_mma_sync", "proj_decode", "pool_epilogue",
-           "fused_tcgen05", "finish")
+           "fused_tcgen05", "finish", "decode_fused")
 
 
 class CmpError(RuntimeError):
@@ -217,5 +217,6 @@ def profile_stop() -> Dict[str, Tuple[float, int]]:
 
 
 def set_proj_kernel(which: int) -> int:
-    """0 auto, 1 mma.sync, 2 tcgen05, 3 weight streaming, 4 fused. Returns the previous value."""
+    """0 auto, 1 mma.sync, 2 tcgen05, 3 weight streaming, 4 fused, 5 one-kernel decode.
+    Returns the previous value."""
     return int(lib.cmp_set_proj_kernel(which))

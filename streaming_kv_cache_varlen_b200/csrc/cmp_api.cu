@@ -16,6 +16,9 @@ cudaError_t launch_proj_decode(const Params& p, cudaStream_t s);
 bool proj_tc_supported(const Params& p);
 bool proj_decode_supported(const Params& p);
 size_t proj_decode_workspace(const Params& p);
+bool decode_fused_supported(const Params& p);
+size_t decode_fused_workspace(const Params& p);
+cudaError_t launch_decode_fused(const Params& p, float* part, void* bar, cudaStream_t s);
 }  // namespace cmp
 
 namespace {
@@ -24,13 +27,17 @@ using cmp::Params;
 
 // ---- workspace ---------------------------------------------------------------
 
+// The first 256 bytes (zeroed when the workspace is created) hold the error
+// word at offset 0 and the decode kernel's grid-barrier words at offset 64.
+constexpr size_t kGridBarOffset = 64;
+
 struct WsLayout {
-  size_t err, m_cu, m_s, m_off, m_tile, proj, ystat, ylse, total;
+  size_t err, m_cu, m_s, m_off, m_tile, proj, ystat, ylse, part, total;
 };
 
 // fused: the pooled-halves buffers of the fused path instead of the fp32
 // projection rows of the other paths.
-WsLayout ws_layout(int64_t B, int64_t T, int64_t C, int64_t n_out, bool fused) {
+WsLayout ws_layout(int64_t B, int64_t T, int64_t C, int64_t n_out, bool fused, size_t part_bytes) {
   WsLayout L{};
   size_t o = 0;
   auto take = [&](size_t n) {
@@ -46,17 +53,19 @@ WsLayout ws_layout(int64_t B, int64_t T, int64_t C, int64_t n_out, bool fused) {
   L.proj = take(fused ? 0 : sizeof(float) * (size_t)T * 2 * C);
   L.ystat = take(fused ? sizeof(float) * (size_t)std::max<int64_t>(n_out, 1) * C : 0);
   L.ylse = take(fused ? sizeof(float) * (size_t)std::max<int64_t>(n_out, 1) * C : 0);
+  L.part = take(part_bytes);
   L.total = o;
   return L;
 }
 
 // Which projection path a call takes: 1 mma.sync, 2 tcgen05 (+ pooling kernel),
 // 3 small-T weight streaming (+ pooling kernel), 4 fused tcgen05 pooling
-// (+ finish kernel).
+// (+ finish kernel), 5 decode in one cooperative kernel.
 int choose_path(const Params& p, int forced) {
   int which = forced;
   if (which == 0) {
-    if (cmp::proj_decode_supported(p)) which = 3;
+    if (cmp::decode_fused_supported(p)) which = 5;
+    else if (cmp::proj_decode_supported(p)) which = 3;
     else if (cmp::fused_supported(p) && p.T >= 1024 && (int64_t)p.T >= 256LL * p.B) which = 4;
     else if (cmp::proj_tc_supported(p)) which = 2;
     else which = 1;
@@ -64,6 +73,7 @@ int choose_path(const Params& p, int forced) {
   if (which == 2 && !cmp::proj_tc_supported(p)) which = 1;
   if (which == 3 && !cmp::proj_decode_supported(p)) which = 1;
   if (which == 4 && !cmp::fused_supported(p)) which = 1;
+  if (which == 5 && !cmp::decode_fused_supported(p)) which = 1;
   return which;
 }
 
@@ -229,8 +239,10 @@ size_t cmp_workspace_size(const cmp_dims* dims, int32_t ratio) {
   p.C = coff * dims->D;
   p.coff = coff;
   p.ratio = ratio;
+  p.n_out = (int)cmp_out_rows(p.B, p.T, ratio);
   const int which = choose_path(p, g_proj_kernel.load());
-  return ws_layout(dims->B, dims->T, p.C, cmp_out_rows(p.B, p.T, ratio), which == 4).total +
+  return ws_layout(dims->B, dims->T, p.C, p.n_out, which == 4,
+                   which == 5 ? cmp::decode_fused_workspace(p) : 0).total +
          cmp::proj_decode_workspace(p);
 }
 
@@ -310,7 +322,8 @@ int cmp_compressor(const cmp_bf16* x, float* kv_state, float* score_state,
 
   const int which = choose_path(p, g_proj_kernel.load());
   const bool fused = which == 4;
-  const WsLayout L = ws_layout(p.B, p.T, p.C, p.n_out, fused);
+  const WsLayout L = ws_layout(p.B, p.T, p.C, p.n_out, fused,
+                               which == 5 ? cmp::decode_fused_workspace(p) : 0);
   const size_t extra = cmp::proj_decode_workspace(p);
   unsigned char* ws = nullptr;
   rc = get_workspace(s, L.total + extra, &ws);
@@ -325,6 +338,14 @@ int cmp_compressor(const cmp_bf16* x, float* kv_state, float* score_state,
   p.ylse = fused ? reinterpret_cast<float*>(ws + L.ylse) : nullptr;
 
   // ---- kernels ----
+  if (which == 5) {  // decode: one cooperative kernel, no scheduler launch
+    float* part = reinterpret_cast<float*>(ws + L.part);
+    void* bar = ws + L.err + kGridBarOffset;
+    if (launch(CMP_KERNEL_DECODE_FUSED, s, [&] { return cmp::launch_decode_fused(p, part, bar, s); }) !=
+        cudaSuccess)
+      return CMP_ERR_CUDA;
+    return CMP_OK;
+  }
   if (launch(CMP_KERNEL_SCHED, s, [&] { return cmp::launch_sched(p, s); }) != cudaSuccess)
     return CMP_ERR_CUDA;
   cudaError_t e;
@@ -367,6 +388,10 @@ int cmp_get_error(void* stream) {
       if (cudaMemcpy(&v, it->second.ptr, sizeof(v), cudaMemcpyDeviceToHost) != cudaSuccess)
         return CMP_ERR_CUDA;
       if (v && cudaMemset(it->second.ptr, 0, sizeof(v)) != cudaSuccess) return CMP_ERR_CUDA;
+      // a wait that gave up may have left the grid barrier's count behind
+      if ((v & cmp::kErrTimeout) &&
+          cudaMemset(it->second.ptr + kGridBarOffset, 0, 2 * sizeof(unsigned)) != cudaSuccess)
+        return CMP_ERR_CUDA;
       word |= v;
     }
   }
@@ -389,9 +414,9 @@ const char* cmp_status_string(int status) {
 }
 
 const char* cmp_kernel_name(int kernel) {
-  static const char* names[CMP_KERNEL_COUNT] = {"sched",         "proj_tcgen05", "proj_mma_sync",
+  static const char* names[CMP_KERNEL_COUNT] = {"sched",         "proj_tcgen05",  "proj_mma_sync",
                                                 "proj_decode",   "pool_epilogue", "fused_tcgen05",
-                                                "finish"};
+                                                "finish",        "decode_fused"};
   return (kernel >= 0 && kernel < CMP_KERNEL_COUNT) ? names[kernel] : nullptr;
 }
 
@@ -432,7 +457,7 @@ int cmp_profile_stop(double* ms, int64_t* launches) {
 }
 
 int cmp_set_proj_kernel(int which) {
-  if (which < 0 || which > 4) return -1;
+  if (which < 0 || which > 5) return -1;
   return g_proj_kernel.exchange(which);
 }
 

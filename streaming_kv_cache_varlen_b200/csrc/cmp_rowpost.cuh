@@ -11,22 +11,28 @@ namespace cmp {
 
 constexpr float kRmsEps = 1e-6f;
 
-// A CTA of D/4 threads; thread i holds the pooled values y of channels
-// c = 4i .. 4i+3 of output row n. red: >= D/128 floats of shared memory,
-// zs: >= D floats of shared memory. Every thread of the CTA must call it.
+// Threads 0 .. D/4-1 of the CTA hold the pooled values y of channels
+// c = 4i .. 4i+3 of output row n (thread i); any further threads only take part
+// in the barriers. red: >= D/128 floats of shared memory, zs: >= D floats of
+// shared memory. Every thread of the CTA must call it.
 __device__ __forceinline__ void finish_row(const Params& p, int n, int c, const float (&y)[4], float* red,
                                            float* zs) {
   const int D = p.D;
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = D / 128;
+  const bool active = (int)threadIdx.x < D / 4;
   // RMSNorm over the D channels of the row
-  float ss = y[0] * y[0] + y[1] * y[1] + y[2] * y[2] + y[3] * y[3];
+  float ss = active ? y[0] * y[0] + y[1] * y[1] + y[2] * y[2] + y[3] * y[3] : 0.f;
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-  if (lane == 0) red[warp] = ss;
+  if (lane == 0 && warp < nwarps) red[warp] = ss;
   __syncthreads();
   float tot = 0.f;
   for (int i = 0; i < nwarps; ++i) tot += red[i];
   const float inv = rsqrtf(tot / (float)D + kRmsEps);
+  if (!active) {
+    if (p.rotate) __syncthreads();  // the Hadamard product's barrier
+    return;
+  }
   const uint2 wraw = *reinterpret_cast<const uint2*>(p.norm_w + c);
   const __nv_bfloat162 w01 = *reinterpret_cast<const __nv_bfloat162*>(&wraw.x);
   const __nv_bfloat162 w23 = *reinterpret_cast<const __nv_bfloat162*>(&wraw.y);

@@ -40,7 +40,7 @@ def test_status_and_kernel_names(cmp):
     for k, name in enumerate(cmp.KERNELS):
         assert cmp.lib.cmp_kernel_name(k).decode() == name
     assert cmp.lib.cmp_kernel_name(99) is None
-    assert cmp.set_proj_kernel(0) == 0 and cmp.set_proj_kernel(7) == -1
+    assert cmp.set_proj_kernel(0) == 0 and cmp.set_proj_kernel(9) == -1
 
 
 def test_out_rows(cmp):

@@ -35,7 +35,7 @@ def check(cmp, inp, rows=None):
     return out, kv, sc, res
 
 
-@pytest.fixture(params=[0, 1, 2, 3, 4], ids=["auto", "mma", "tcgen05", "decode", "fused"])
+@pytest.fixture(params=[0, 1, 2, 3, 4, 5], ids=["auto", "mma", "tcgen05", "decode", "fused", "decode1k"])
 def proj_kernel(request, lib):
     prev = lib.set_proj_kernel(request.param)
     yield request.param
@@ -220,7 +220,7 @@ def test_projection_kernels_agree(lib):
                                 H=4096, D=512, coff=2, ratio=4, block_size=128, rotate=False))
     res = run_inputs(inp)
     outs = {}
-    for k in (1, 2, 3, 4):
+    for k in (1, 2, 3, 4, 5):
         prev = lib.set_proj_kernel(k)
         try:
             o, kv, sc, err = run(lib, inp)
