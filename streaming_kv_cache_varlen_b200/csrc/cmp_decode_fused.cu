@@ -40,11 +40,16 @@ using namespace sm100;
 
 constexpr int BM = 128;
 constexpr int BK = 64;
-constexpr int STAGES = 4;
-constexpr int kThreads = 128;
+constexpr int kThreads = 192;        // warps 0-3: TMEM quadrants; warps 4-5: call metadata
 constexpr int kMaxSeqs = 256;
 constexpr int kMaxRowsPerWindow = 256;
-constexpr int kHistRows = 8;  // state rows of a window prefetched into shared memory
+constexpr int kHistRows = 8;         // state rows of a window prefetched into shared memory
+
+template <int MAXT>
+struct Stages {
+  // enough stages that a C4A-sized CTA requests its whole weight slice at once
+  static constexpr int value = MAXT <= 32 ? 8 : 6;
+};
 
 struct TokInfo {
   int32_t b;        // sequence, or -1
@@ -55,8 +60,11 @@ struct TokInfo {
 
 template <int MAXT>
 struct Smem {
-  __nv_bfloat16 w[STAGES][BM * BK];     // 16 KB per stage
-  __nv_bfloat16 x[STAGES][MAXT * BK];   // MAXT * 128 bytes per stage
+  static constexpr int S = Stages<MAXT>::value;
+  __nv_bfloat16 w[S][BM * BK];     // 16 KB per stage
+  __nv_bfloat16 x[S][MAXT * BK];   // MAXT * 128 bytes per stage
+  alignas(16) float hist_kv[kHistRows][512];  // the window's state rows (float4 access)
+  alignas(16) float hist_sc[kHistRows][512];
   TokInfo tok[MAXT];
   int32_t cu[kMaxSeqs + 1];
   int32_t sp[kMaxSeqs];
@@ -64,22 +72,19 @@ struct Smem {
   int32_t src_t[kMaxRowsPerWindow];     // per window row: token (>= 0), -1 (state row) or INT32_MIN (skip)
   int64_t src_kv[kMaxRowsPerWindow];
   int64_t src_sc[kMaxRowsPerWindow];
-  alignas(16) float hist_kv[kHistRows][512];  // the window's state rows, prefetched before the grid barrier
-  alignas(16) float hist_sc[kHistRows][512];  // (read and written as float4: 16-byte aligned)
   int32_t row_w;                        // window of this CTA's output row, or -1
-  int32_t row_b;
-  int32_t row_s;
-  int32_t row_cu;
-  int32_t hist_ok;                      // every state row of the window is in hist_*
+  int32_t nhist;                        // state rows 0..nhist-1 of the window are in hist_*, or -1
   float red[32];
   float zs[512];
-  uint64_t full[STAGES];
-  uint64_t empty[STAGES];
+  uint64_t full[S];
+  uint64_t empty[S];
   uint64_t acc_full;
   uint32_t tmem_base;
   int abort;
   int rejected;
   int grid_ok;
+  uint32_t bar_gen;   // generation seen at arrival (thread 0)
+  int bar_last;       // this CTA released the barrier
 };
 
 static_assert(offsetof(Smem<32>, hist_kv) % 16 == 0 && offsetof(Smem<32>, hist_sc) % 16 == 0,
@@ -88,44 +93,45 @@ static_assert(offsetof(Smem<64>, hist_kv) % 16 == 0 && offsetof(Smem<64>, hist_s
               "float4 shared-memory rows must be 16-byte aligned");
 static_assert(offsetof(Smem<32>, x) % 1024 == 0 && offsetof(Smem<64>, x) % 1024 == 0,
               "TMA swizzled tiles must be 1024-byte aligned");
+static_assert(sizeof(Smem<32>) + 1024 <= 232448 && sizeof(Smem<64>) + 1024 <= 232448,
+              "shared memory per CTA");
 
 struct GridBar {
   unsigned count;
+  unsigned pad0[31];  // count and generation on different 128-byte lines
   unsigned gen;
 };
 
-// Grid-wide barrier for a cooperative launch. Thread 0 of each CTA arrives;
-// the last arrival resets the count and bumps the generation. Waiting is
-// bounded: after ~1 s the CTA records a timeout and goes on without the data.
-__device__ bool grid_barrier(GridBar* bar, unsigned nblocks, unsigned* err, int* ok_s) {
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    int ok = 1;
-    unsigned g;
-    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(g) : "l"(&bar->gen) : "memory");
+// Split grid barrier for a cooperative launch. grid_arrive: thread 0 of each
+// CTA, after the CTA's stores; the last arrival resets the count and bumps the
+// generation. grid_wait: thread 0 waits (bounded: ~1 s, then a timeout is
+// recorded and the CTA goes on without the data) for the generation to move.
+__device__ __forceinline__ void grid_arrive(GridBar* bar, unsigned nblocks, uint32_t* gen_seen, int* last) {
+  unsigned g;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(g) : "l"(&bar->gen) : "memory");
+  __threadfence();
+  *gen_seen = g;
+  *last = 0;
+  if (atomicAdd(&bar->count, 1u) == nblocks - 1) {
+    atomicExch(&bar->count, 0u);
     __threadfence();
-    if (atomicAdd(&bar->count, 1u) == nblocks - 1) {
-      atomicExch(&bar->count, 0u);
-      __threadfence();
-      asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(&bar->gen), "r"(g + 1) : "memory");
-    } else {
-      const uint64_t t0 = globaltimer();
-      for (;;) {
-        unsigned now;
-        asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(now) : "l"(&bar->gen) : "memory");
-        if (now != g) break;
-        if (globaltimer() - t0 > 1000000000ull) {
-          ok = 0;
-          atomicOr(err, kErrTimeout);
-          break;
-        }
-        __nanosleep(64);
-      }
-    }
-    *ok_s = ok;
+    asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(&bar->gen), "r"(g + 1) : "memory");
+    *last = 1;
   }
-  __syncthreads();
-  return *ok_s != 0;
+}
+
+__device__ __forceinline__ bool grid_wait(GridBar* bar, uint32_t g, unsigned* err) {
+  const uint64_t t0 = globaltimer();
+  for (;;) {
+    unsigned now;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(now) : "l"(&bar->gen) : "memory");
+    if (now != g) return true;
+    if (globaltimer() - t0 > 1000000000ull) {
+      atomicOr(err, kErrTimeout);
+      return false;
+    }
+    __nanosleep(32);
+  }
 }
 
 // sum over the K slices of part[q][t][col .. col+3], in slice order, with up to
@@ -157,13 +163,140 @@ struct DecodeArgs {
   int ks;           // K slices
 };
 
+// Window row j of window w: its absolute position.
+__device__ __forceinline__ int window_pos(int w, int j, int r, int coff) {
+  return coff == 1 ? w * r + j : (j < r ? (w - 1) * r + j : w * r + (j - r));
+}
+
+// Warps 4-5: validate the call, output-row offsets, per-token facts, and the
+// sources of this CTA's output row (what the varlen scheduler kernel does on
+// the other paths), while warps 0-3 stream and multiply.
+template <int MAXT>
+__device__ void call_metadata(const Params& p, Smem<MAXT>& sm, int NT) {
+  const int et = threadIdx.x - 128;  // 0..63
+  const int B = p.B;
+  bool bad = false;
+  for (int i = et; i <= B; i += 64) {
+    const int c = p.cu_in[i];
+    const int c1 = i < B ? p.cu_in[i + 1] : c;
+    const int s = (i < B && p.start_pos) ? p.start_pos[i] : 0;
+    sm.cu[i] = c;
+    if (i < B) sm.sp[i] = s;
+    bool ok = c >= 0 && c <= p.T && (i != 0 || c == 0) && (i != B || c == p.T);
+    if (i < B) ok = ok && c1 >= c && s >= 0 && (int64_t)s + (c1 - c) <= (int64_t)INT32_MAX;
+    bad = bad || !ok;
+  }
+  if (bad) atomicOr(&sm.rejected, 1);
+  asm volatile("bar.sync 2, 64;" ::: "memory");
+  const bool rejected = sm.rejected != 0;
+  if (et < 32) {  // output-row offsets: sequence b reserves min(L, L/ratio + 1) rows
+    int carry = 0;
+    for (int b0 = 0; b0 < B; b0 += 32) {
+      const int b = b0 + et;
+      int cap = 0;
+      if (b < B && !rejected) {
+        const int L = sm.cu[b + 1] - sm.cu[b];
+        cap = min(L, L / p.ratio + 1);
+      }
+      int inc = cap;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int v = __shfl_up_sync(0xffffffffu, inc, o);
+        if (et >= o) inc += v;
+      }
+      if (b < B) sm.off[b] = carry + inc - cap;
+      carry += __shfl_sync(0xffffffffu, inc, 31);
+    }
+    if (et == 0) {
+      sm.off[B] = carry;
+      if (rejected) atomicOr(p.err, kErrIndex);
+    }
+  }
+  asm volatile("bar.sync 2, 64;" ::: "memory");
+  if (rejected) {
+    for (int i = et; i <= B; i += 64) sm.cu[i] = 0;
+    asm volatile("bar.sync 2, 64;" ::: "memory");
+  }
+  for (int t = et; t < NT; t += 64) {
+    TokInfo ti{-1, 0, -1, -1};
+    if (t < p.T && !rejected) {
+      int lo = 0, hi = B;
+      while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (sm.cu[mid] <= t) lo = mid; else hi = mid - 1;
+      }
+      if (lo < B) {
+        const int s = sm.sp[lo];
+        const int pos = s + (t - sm.cu[lo]);
+        const int e = s + (sm.cu[lo + 1] - sm.cu[lo]);
+        ti.b = lo;
+        ti.pos = pos;
+        if (pos >= tail_threshold(e, p.ratio, p.coff)) {
+          const int rk = table_row(p, p.kv_tbl, lo, pos);
+          const int rs = table_row(p, p.sc_tbl, lo, pos);
+          if (rk >= 0) ti.kv_off = ((int64_t)rk * p.bs + pos % p.bs) * p.C;
+          if (rs >= 0) ti.sc_off = ((int64_t)rs * p.bs + pos % p.bs) * p.C;
+        }
+      }
+    }
+    sm.tok[t] = ti;
+  }
+  // this CTA's output row: its window and where each window row comes from
+  if ((int)blockIdx.x < p.n_out) {
+    const int n = blockIdx.x, r = p.ratio;
+    int lo = 0, hi = B;
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (sm.off[mid] <= n) lo = mid; else hi = mid - 1;
+    }
+    int w = -1, s = 0, cu = 0;
+    if (lo < B && !rejected) {
+      s = sm.sp[lo];
+      cu = sm.cu[lo];
+      const int e = s + (sm.cu[lo + 1] - cu);
+      const int k = n - sm.off[lo];
+      if (k < e / r - s / r) w = s / r + k;
+    }
+    const int rows = p.coff * r;
+    int nh = 0;
+    if (w >= 0) {
+      for (int j = et; j < rows; j += 64) {
+        const int q = window_pos(w, j, r, p.coff);
+        int st = INT32_MIN;
+        int64_t okv = 0, osc = 0;
+        if (q >= s) {
+          st = cu + (q - s);
+        } else if (q >= 0) {
+          const int rk = table_row(p, p.kv_tbl, lo, q);
+          const int rs = table_row(p, p.sc_tbl, lo, q);
+          if (rk >= 0 && rs >= 0) {
+            st = -1;
+            okv = ((int64_t)rk * p.bs + q % p.bs) * p.C;
+            osc = ((int64_t)rs * p.bs + q % p.bs) * p.C;
+          }
+        }
+        sm.src_t[j] = st;
+        sm.src_kv[j] = okv;
+        sm.src_sc[j] = osc;
+      }
+      for (int j = 0; j < rows; ++j)
+        if (window_pos(w, j, r, p.coff) < s) nh = j + 1;  // state rows are the window's first rows
+    }
+    if (et == 0) {
+      sm.row_w = w;
+      sm.nhist = (w >= 0 && nh <= kHistRows && p.D <= 512) ? nh : -1;
+    }
+  }
+}
+
 template <int MAXT>
 __global__ void __launch_bounds__(kThreads, 1)
     decode_fused_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUtensorMap map_wkv,
                         const __grid_constant__ CUtensorMap map_wg, Params p, DecodeArgs a, int NT) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
-  using S = Smem<MAXT>;
-  S& sm = *reinterpret_cast<S*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  using SM = Smem<MAXT>;
+  constexpr int STAGES = SM::S;
+  SM& sm = *reinterpret_cast<SM*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int tile = blockIdx.x / a.ks, ks = blockIdx.x % a.ks;
   const int m0 = tile * BM;  // first of the 128 weight rows (of the 2C)
@@ -184,6 +317,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(&sm.acc_full, 1);
     sm.abort = 0;
     sm.rejected = 0;
+    sm.row_w = -1;
+    sm.nhist = -1;
     fence_barrier_init();
     prefetch_tmap(wmap);
     prefetch_tmap(&map_x);
@@ -195,7 +330,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem = sm.tmem_base;
   volatile int* abort = &sm.abort;
 
-  // ---- 1) stream + MMA (warps 0, 1) / call metadata (warps 2, 3) ----
+  // ---- 1) stream + MMA (warps 0, 1) / call metadata (warps 4, 5) ----
   if (warp == 0 && lane == 0) {
     int stage = 0;
     uint32_t phase = 0;
@@ -224,152 +359,65 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (++stage == STAGES) { stage = 0; phase ^= 1u; }
     }
     if (ok) mma_commit(&sm.acc_full);
-  } else if (warp >= 2) {
-    const int et = threadIdx.x - 64;  // 64 threads
-    const int B = p.B;
-    bool bad = false;
-    for (int i = et; i <= B; i += 64) {
-      const int c = p.cu_in[i];
-      sm.cu[i] = c;
-      bool ok = c >= 0 && c <= p.T && (i != 0 || c == 0) && (i != B || c == p.T);
-      if (i < B) {
-        const int c1 = p.cu_in[i + 1];
-        const int s = p.start_pos ? p.start_pos[i] : 0;
-        sm.sp[i] = s;
-        ok = ok && c1 >= c && s >= 0 && (int64_t)s + (c1 - c) <= (int64_t)INT32_MAX;
-      }
-      bad = bad || !ok;
-    }
-    if (bad) atomicOr(&sm.rejected, 1);
-    asm volatile("bar.sync 2, 64;" ::: "memory");
-    const bool rejected = sm.rejected != 0;
-    if (et == 0) {  // output-row offsets: sequence b reserves min(L, L/ratio + 1) rows
-      int acc = 0;
-      for (int b = 0; b < B; ++b) {
-        sm.off[b] = acc;
-        const int L = rejected ? 0 : sm.cu[b + 1] - sm.cu[b];
-        acc += min(L, L / p.ratio + 1);
-      }
-      sm.off[B] = acc;
-      if (rejected) {
-        for (int b = 0; b <= B; ++b) sm.cu[b] = 0;
-        atomicOr(p.err, kErrIndex);
-      }
-    }
-    asm volatile("bar.sync 2, 64;" ::: "memory");
-    for (int t = et; t < NT; t += 64) {
-      TokInfo ti{-1, 0, -1, -1};
-      if (t < p.T && !rejected) {
-        int lo = 0, hi = B;
-        while (lo < hi) {
-          const int mid = (lo + hi + 1) >> 1;
-          if (sm.cu[mid] <= t) lo = mid; else hi = mid - 1;
-        }
-        if (lo < B) {
-          const int s = sm.sp[lo];
-          const int pos = s + (t - sm.cu[lo]);
-          const int e = s + (sm.cu[lo + 1] - sm.cu[lo]);
-          ti.b = lo;
-          ti.pos = pos;
-          if (pos >= tail_threshold(e, p.ratio, p.coff)) {
-            const int rk = table_row(p, p.kv_tbl, lo, pos);
-            const int rs = table_row(p, p.sc_tbl, lo, pos);
-            if (rk >= 0) ti.kv_off = ((int64_t)rk * p.bs + pos % p.bs) * p.C;
-            if (rs >= 0) ti.sc_off = ((int64_t)rs * p.bs + pos % p.bs) * p.C;
-          }
-        }
-      }
-      sm.tok[t] = ti;
-    }
-    // this CTA's output row (CTAs 0 .. n_out-1 build one row each after the
-    // barrier): find its window, resolve where each window row comes from and
-    // fetch the rows written by earlier calls now, while the weights stream
-    if ((int)blockIdx.x < p.n_out) {
-      const int n = blockIdx.x, r = p.ratio;
-      int lo = 0, hi = B;
-      while (lo < hi) {
-        const int mid = (lo + hi + 1) >> 1;
-        if (sm.off[mid] <= n) lo = mid; else hi = mid - 1;
-      }
-      int w = -1, s = 0, cu = 0;
-      if (lo < B && !rejected) {
-        s = sm.sp[lo];
-        cu = sm.cu[lo];
-        const int e = s + (sm.cu[lo + 1] - cu);
-        const int k = n - sm.off[lo];
-        if (k < e / r - s / r) w = s / r + k;
-      }
-      if (et == 0) {
-        sm.row_w = w;
-        sm.row_b = lo;
-        sm.row_s = s;
-        sm.row_cu = cu;
-      }
-      int nhist = 0;
-      if (w >= 0) {
-        const int rows = p.coff * r;
-        for (int j = et; j < rows; j += 64) {
-          const int q = p.coff == 1 ? w * r + j : (j < r ? (w - 1) * r + j : w * r + (j - r));
-          int st = INT32_MIN;
-          int64_t okv = 0, osc = 0;
-          if (q >= s) {
-            st = cu + (q - s);
-          } else if (q >= 0) {
-            const int rk = table_row(p, p.kv_tbl, lo, q);
-            const int rs = table_row(p, p.sc_tbl, lo, q);
-            if (rk >= 0 && rs >= 0) {
-              st = -1;
-              okv = ((int64_t)rk * p.bs + q % p.bs) * p.C;
-              osc = ((int64_t)rs * p.bs + q % p.bs) * p.C;
-            }
-          }
-          sm.src_t[j] = st;
-          sm.src_kv[j] = okv;
-          sm.src_sc[j] = osc;
-        }
-        // state rows can only be the window's first rows; prefetch them if few
-        nhist = 0;
-        for (int j = 0; j < rows; ++j) {
-          const int q = p.coff == 1 ? w * r + j : (j < r ? (w - 1) * r + j : w * r + (j - r));
-          if (q < s) nhist = j + 1;
-        }
-      }
-      asm volatile("bar.sync 2, 64;" ::: "memory");
-      const bool fits = w >= 0 && nhist <= kHistRows && p.D <= 512;
-      if (fits) {
-        for (int i = et; i < nhist * (p.D / 4); i += 64) {
-          const int j = i / (p.D / 4), c = (i % (p.D / 4)) * 4;
-          if (sm.src_t[j] != -1) continue;
-          const int col = ((p.coff == 2 && j >= r) ? p.D : 0) + c;
-          *reinterpret_cast<float4*>(&sm.hist_kv[j][c]) =
-              *reinterpret_cast<const float4*>(p.kv_state + sm.src_kv[j] + col);
-          *reinterpret_cast<float4*>(&sm.hist_sc[j][c]) =
-              *reinterpret_cast<const float4*>(p.score_state + sm.src_sc[j] + col);
-        }
-      }
-      if (et == 0) sm.hist_ok = fits ? nhist : -1;
-    }
+  } else if (warp >= 4) {
+    call_metadata<MAXT>(p, sm, NT);
   }
 
-  // partial product of this CTA's 128 rows -> part[ks][t][m0 + row]
-  const bool have = mbar_wait(&sm.acc_full, 0, abort);
-  if (__all_sync(0xffffffffu, have)) {
-    tc_fence_after();
-    const int row = warp * 32 + lane;
-    float* dst = a.part + (int64_t)ks * p.T * C2 + m0 + row;
-    for (int c0 = 0; c0 < NT; c0 += 32) {
-      uint32_t r[32];
-      tmem_ld32(tmem + ((uint32_t)(warp * 32) << 16) + c0, r);
-      tmem_ld_wait(r);
+  if (warp < 4) {
+    // the partial product of this CTA's 128 rows -> part[ks][t][m0 + row]
+    const bool have = mbar_wait(&sm.acc_full, 0, abort);
+    if (__all_sync(0xffffffffu, have)) {
+      tc_fence_after();
+      const int row = warp * 32 + lane;
+      float* dst = a.part + (int64_t)ks * p.T * C2 + m0 + row;
+      for (int c0 = 0; c0 < NT; c0 += 32) {
+        uint32_t r[32];
+        tmem_ld32(tmem + ((uint32_t)(warp * 32) << 16) + c0, r);
+        tmem_ld_wait(r);
 #pragma unroll
-      for (int j = 0; j < 32; ++j)
-        if (c0 + j < p.T) dst[(int64_t)(c0 + j) * C2] = __uint_as_float(r[j]);
+        for (int j = 0; j < 32; ++j)
+          if (c0 + j < p.T) dst[(int64_t)(c0 + j) * C2] = __uint_as_float(r[j]);
+      }
+    }
+    tc_fence_before();
+    asm volatile("bar.sync 1, 128;" ::: "memory");  // all partial stores of the CTA issued
+    if (threadIdx.x == 0) grid_arrive(a.bar, gridDim.x, &sm.bar_gen, &sm.bar_last);
+  }
+  __syncthreads();  // metadata (warps 4-5) done
+
+  // ---- 2) while the other CTAs arrive: this CTA's window rows from the state ----
+  const int nh = sm.nhist;
+  if ((int)blockIdx.x < p.n_out && nh > 0) {
+    const int q4 = p.D / 4;
+    for (int i0 = threadIdx.x; i0 < nh * q4; i0 += 2 * kThreads) {
+      float4 kv[2], sc[2];
+      bool use[2];
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {  // two rows' loads in flight per thread
+        const int i = i0 + u * kThreads;
+        const int j = i / q4;
+        use[u] = i < nh * q4 && sm.src_t[j] == -1;
+        if (use[u]) {
+          const int c = (i % q4) * 4;
+          const int col = ((p.coff == 2 && j >= p.ratio) ? p.D : 0) + c;
+          kv[u] = *reinterpret_cast<const float4*>(p.kv_state + sm.src_kv[j] + col);
+          sc[u] = *reinterpret_cast<const float4*>(p.score_state + sm.src_sc[j] + col);
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+        if (use[u]) {
+          const int i = i0 + u * kThreads;
+          const int j = i / q4, c = (i % q4) * 4;
+          *reinterpret_cast<float4*>(&sm.hist_kv[j][c]) = kv[u];
+          *reinterpret_cast<float4*>(&sm.hist_sc[j][c]) = sc[u];
+        }
+      }
     }
   }
-  tc_fence_before();
-
-  // ---- 2) every CTA's partials are in L2 ----
-  const bool ok = grid_barrier(a.bar, gridDim.x, p.err, &sm.grid_ok) && !*abort;
+  if (threadIdx.x == 0) sm.grid_ok = sm.bar_last ? 1 : (grid_wait(a.bar, sm.bar_gen, p.err) ? 1 : 0);
+  __syncthreads();
+  const bool ok = sm.grid_ok && !*abort;
 
   // ---- 3) output rows / state tails ----
   const int n_out = p.n_out;
@@ -384,7 +432,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (active) *reinterpret_cast<uint2*>(p.out + (int64_t)n * D + c) = make_uint2(0u, 0u);
     } else {
       const int rows = p.coff * r;
-      const int nhist = sm.hist_ok;  // >= 0: state rows 0..nhist-1 are in shared memory
       float y[4] = {0.f, 0.f, 0.f, 0.f};
       if (active) {
         float m[4], l[4], ac[4];
@@ -396,7 +443,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int col = ((p.coff == 2 && j >= r) ? D : 0) + c;
           float4 kv, sc;
           if (st >= 0) {  // this call's token: the K-slice partials plus ape
-            const int q = p.coff == 1 ? w * r + j : (j < r ? (w - 1) * r + j : w * r + (j - r));
+            const int q = window_pos(w, j, r, p.coff);
             kv = sum_slices(a.part, KS, slice, (int64_t)st * C2 + col);
             sc = sum_slices(a.part, KS, slice, (int64_t)st * C2 + p.C + col);
             const float4 ap = *reinterpret_cast<const float4*>(p.ape + (int64_t)(q % r) * p.C + col);
@@ -404,7 +451,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             sc.y += ap.y;
             sc.z += ap.z;
             sc.w += ap.w;
-          } else if (j < nhist) {
+          } else if (j < nh) {
             kv = *reinterpret_cast<const float4*>(&sm.hist_kv[j][c]);
             sc = *reinterpret_cast<const float4*>(&sm.hist_sc[j][c]);
           } else {
