@@ -217,8 +217,10 @@ enum {
   CMP_KERNEL_POOL = 4,         /* pooling + RMSNorm + RoPE + Hadamard + store */
   CMP_KERNEL_FUSED = 5,        /* prefill projection with the pooling in its epilogue */
   CMP_KERNEL_FINISH = 6,       /* fused path: merge halves + RMSNorm + RoPE + Hadamard */
-  CMP_KERNEL_DECODE_FUSED = 7, /* decode (T <= 64) in one cooperative kernel */
-  CMP_KERNEL_COUNT = 8
+  CMP_KERNEL_DECODE_FUSED = 7, /* decode (T <= 64) in one cooperative kernel, K-split grid */
+  CMP_KERNEL_DECODE_CP = 8,    /* decode (T <= 64) in one cooperative kernel of 4-CTA clusters
+                                  that each own 16 channels */
+  CMP_KERNEL_COUNT = 9
 };
 
 /* Name of a kernel id (NULL if out of range). */
@@ -237,12 +239,14 @@ CMP_API int cmp_profile_start(void);
 CMP_API int cmp_profile_stop(double* ms, int64_t* launches);
 
 /* Testing knob: which path calls take. 0 = automatic (for T <= 64 the
- * one-kernel cooperative decode, else the weight-streaming projection +
- * pooling kernel; the fused tcgen05 pooling kernel for long sequences,
- * T >= 1024 and T >= 256*B; else the tcgen05 projection + pooling kernel),
- * 1 = force the mma.sync projection, 2 = the tcgen05 projection, 3 = weight
- * streaming, 4 = the fused path, 5 = the one-kernel decode. A forced path a
- * call cannot take falls back to 1.
+ * channel-group decode kernel, or without it (rotate, or a device that cannot
+ * hold its clusters) the K-split one-kernel decode, else the weight-streaming
+ * projection + pooling kernel; the fused tcgen05 pooling kernel for long
+ * sequences, T >= 1024 and T >= 256*B; else the tcgen05 projection + pooling
+ * kernel), 1 = force the mma.sync projection, 2 = the tcgen05 projection,
+ * 3 = weight streaming, 4 = the fused path, 5 = the K-split one-kernel decode,
+ * 6 = the channel-group decode. A forced path a call cannot take falls back
+ * to 1.
  * Returns the previous value, or -1 if out of range. */
 CMP_API int cmp_set_proj_kernel(int which);
 

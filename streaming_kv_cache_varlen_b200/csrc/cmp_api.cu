@@ -19,6 +19,9 @@ size_t proj_decode_workspace(const Params& p);
 bool decode_fused_supported(const Params& p);
 size_t decode_fused_workspace(const Params& p);
 cudaError_t launch_decode_fused(const Params& p, float* part, void* bar, cudaStream_t s);
+bool decode_cp_supported(const Params& p);
+size_t decode_cp_workspace(const Params& p);
+cudaError_t launch_decode_cp(const Params& p, float* ss, void* bar, cudaStream_t s);
 }  // namespace cmp
 
 namespace {
@@ -27,9 +30,12 @@ using cmp::Params;
 
 // ---- workspace ---------------------------------------------------------------
 
-// The first 256 bytes (zeroed when the workspace is created) hold the error
-// word at offset 0 and the decode kernel's grid-barrier words at offset 64.
+// The first kHeaderBytes (zeroed when the workspace is created) hold the error
+// word at offset 0, the K-split decode kernel's grid-barrier words at offset 64
+// and the channel-group decode kernel's barrier counters at offset 256.
+constexpr size_t kHeaderBytes = 2048;
 constexpr size_t kGridBarOffset = 64;
+constexpr size_t kGridBar2Offset = 256;
 
 struct WsLayout {
   size_t err, m_cu, m_s, m_off, m_tile, proj, ystat, ylse, part, total;
@@ -45,7 +51,7 @@ WsLayout ws_layout(int64_t B, int64_t T, int64_t C, int64_t n_out, bool fused, s
     o += (n + 255) & ~size_t(255);
     return r;
   };
-  L.err = take(16);
+  L.err = take(kHeaderBytes);
   L.m_cu = take(sizeof(int32_t) * (B + 1));
   L.m_s = take(sizeof(int32_t) * std::max<int64_t>(B, 1));
   L.m_off = take(sizeof(int32_t) * (B + 1));
@@ -60,11 +66,13 @@ WsLayout ws_layout(int64_t B, int64_t T, int64_t C, int64_t n_out, bool fused, s
 
 // Which projection path a call takes: 1 mma.sync, 2 tcgen05 (+ pooling kernel),
 // 3 small-T weight streaming (+ pooling kernel), 4 fused tcgen05 pooling
-// (+ finish kernel), 5 decode in one cooperative kernel.
+// (+ finish kernel), 5 decode in one cooperative kernel (K-split grid),
+// 6 decode in one cooperative kernel of channel-group clusters.
 int choose_path(const Params& p, int forced) {
   int which = forced;
   if (which == 0) {
-    if (cmp::decode_fused_supported(p)) which = 5;
+    if (cmp::decode_cp_supported(p)) which = 6;
+    else if (cmp::decode_fused_supported(p)) which = 5;
     else if (cmp::proj_decode_supported(p)) which = 3;
     else if (cmp::fused_supported(p) && p.T >= 1024 && (int64_t)p.T >= 256LL * p.B) which = 4;
     else if (cmp::proj_tc_supported(p)) which = 2;
@@ -74,6 +82,7 @@ int choose_path(const Params& p, int forced) {
   if (which == 3 && !cmp::proj_decode_supported(p)) which = 1;
   if (which == 4 && !cmp::fused_supported(p)) which = 1;
   if (which == 5 && !cmp::decode_fused_supported(p)) which = 1;
+  if (which == 6 && !cmp::decode_cp_supported(p)) which = 1;
   return which;
 }
 
@@ -138,7 +147,12 @@ cudaError_t launch(int kernel, cudaStream_t s, F&& f) {
   if (prof) {
     cudaEventRecord(t.b, s);
     std::lock_guard<std::mutex> lk(g_prof_mu);
-    g_timed.push_back(t);
+    if (e == cudaSuccess) {
+      g_timed.push_back(t);
+    } else {  // nothing ran: no timing record
+      g_event_pool.push_back(t.a);
+      g_event_pool.push_back(t.b);
+    }
   }
   if (e == cudaSuccess) g_launches.fetch_add(1, std::memory_order_relaxed);
   return e;
@@ -166,7 +180,7 @@ int get_workspace(cudaStream_t s, size_t need, unsigned char** out) {
   const size_t bytes = std::max(need, size_t(1) << 20);
   void* p = nullptr;
   if (cudaMalloc(&p, bytes) != cudaSuccess) return CMP_ERR_CUDA;
-  if (cudaMemset(p, 0, 256) != cudaSuccess) {
+  if (cudaMemset(p, 0, kHeaderBytes) != cudaSuccess) {
     cudaFree(p);
     return CMP_ERR_CUDA;
   }
@@ -174,6 +188,13 @@ int get_workspace(cudaStream_t s, size_t need, unsigned char** out) {
   w.bytes = bytes;
   *out = w.ptr;
   return CMP_OK;
+}
+
+// Extra workspace of the one-kernel decode paths.
+size_t decode_part_bytes(const Params& p, int which) {
+  if (which == 5) return cmp::decode_fused_workspace(p);
+  if (which == 6) return cmp::decode_cp_workspace(p);
+  return 0;
 }
 
 bool valid_ratio(int r) {
@@ -189,6 +210,68 @@ int check_dims(const cmp_dims* d) {
   if (d->H < 512 || d->H > 16384 || d->H % 512) return CMP_ERR_INVALID;
   if (d->block_size < 1 || d->block_size > 1024) return CMP_ERR_INVALID;
   if (d->block_num < 1 || d->table_stride < 1) return CMP_ERR_INVALID;
+  return CMP_OK;
+}
+
+// Returned by run_path when the device refused a launch form before anything
+// ran (the path is then disabled on that device): the caller picks again.
+constexpr int kRetryOtherPath = -1000;
+
+// Workspace and launches of one call on path `which`.
+int run_path(Params& p, int which, cudaStream_t s) {
+  int rc;
+  const bool fused = which == 4;
+  const WsLayout L = ws_layout(p.B, p.T, p.C, p.n_out, fused, decode_part_bytes(p, which));
+  const size_t extra = cmp::proj_decode_workspace(p);
+  unsigned char* ws = nullptr;
+  rc = get_workspace(s, L.total + extra, &ws);
+  if (rc != CMP_OK) return rc;
+  p.err = reinterpret_cast<unsigned*>(ws + L.err);
+  p.m_cu = reinterpret_cast<int32_t*>(ws + L.m_cu);
+  p.m_s = reinterpret_cast<int32_t*>(ws + L.m_s);
+  p.m_off = reinterpret_cast<int32_t*>(ws + L.m_off);
+  p.m_tile = fused ? reinterpret_cast<int32_t*>(ws + L.m_tile) : nullptr;
+  p.proj = fused ? nullptr : reinterpret_cast<float*>(ws + L.proj);
+  p.ystat = fused ? reinterpret_cast<float*>(ws + L.ystat) : nullptr;
+  p.ylse = fused ? reinterpret_cast<float*>(ws + L.ylse) : nullptr;
+
+  // ---- kernels ----
+  if (which == 6) {  // decode: one cooperative kernel of clusters, no scheduler launch
+    float* ss = reinterpret_cast<float*>(ws + L.part);
+    void* bar = ws + L.err + kGridBar2Offset;
+    const cudaError_t e =
+        launch(CMP_KERNEL_DECODE_CP, s, [&] { return cmp::launch_decode_cp(p, ss, bar, s); });
+    if (e == cudaErrorNotSupported) return kRetryOtherPath;
+    return e == cudaSuccess ? CMP_OK : CMP_ERR_CUDA;
+  }
+  if (which == 5) {  // decode: one cooperative kernel, no scheduler launch
+    float* part = reinterpret_cast<float*>(ws + L.part);
+    void* bar = ws + L.err + kGridBarOffset;
+    if (launch(CMP_KERNEL_DECODE_FUSED, s, [&] { return cmp::launch_decode_fused(p, part, bar, s); }) !=
+        cudaSuccess)
+      return CMP_ERR_CUDA;
+    return CMP_OK;
+  }
+  if (launch(CMP_KERNEL_SCHED, s, [&] { return cmp::launch_sched(p, s); }) != cudaSuccess)
+    return CMP_ERR_CUDA;
+  cudaError_t e;
+  if (fused) {
+    const int sms = sm_count_cached();
+    e = launch(CMP_KERNEL_FUSED, s, [&] { return cmp::launch_fused(p, s, sms); });
+    if (e != cudaSuccess) return CMP_ERR_CUDA;
+    if (launch(CMP_KERNEL_FINISH, s, [&] { return cmp::launch_finish(p, s); }) != cudaSuccess)
+      return CMP_ERR_CUDA;
+    return CMP_OK;
+  }
+  if (which == 2)
+    e = launch(CMP_KERNEL_PROJ_TC, s, [&] { return cmp::launch_proj_tc(p, s); });
+  else if (which == 3)
+    e = launch(CMP_KERNEL_PROJ_DECODE, s, [&] { return cmp::launch_proj_decode(p, s); });
+  else
+    e = launch(CMP_KERNEL_PROJ_MMA, s, [&] { return cmp::launch_proj_mma(p, s); });
+  if (e != cudaSuccess) return CMP_ERR_CUDA;
+  if (launch(CMP_KERNEL_POOL, s, [&] { return cmp::launch_pool(p, s); }) != cudaSuccess)
+    return CMP_ERR_CUDA;
   return CMP_OK;
 }
 
@@ -241,8 +324,7 @@ size_t cmp_workspace_size(const cmp_dims* dims, int32_t ratio) {
   p.ratio = ratio;
   p.n_out = (int)cmp_out_rows(p.B, p.T, ratio);
   const int which = choose_path(p, g_proj_kernel.load());
-  return ws_layout(dims->B, dims->T, p.C, p.n_out, which == 4,
-                   which == 5 ? cmp::decode_fused_workspace(p) : 0).total +
+  return ws_layout(dims->B, dims->T, p.C, p.n_out, which == 4, decode_part_bytes(p, which)).total +
          cmp::proj_decode_workspace(p);
 }
 
@@ -320,54 +402,15 @@ int cmp_compressor(const cmp_bf16* x, float* kv_state, float* score_state,
   p.stride = dims->table_stride;
   p.n_out = (int)cmp_out_rows(p.B, p.T, ratio);
 
-  const int which = choose_path(p, g_proj_kernel.load());
-  const bool fused = which == 4;
-  const WsLayout L = ws_layout(p.B, p.T, p.C, p.n_out, fused,
-                               which == 5 ? cmp::decode_fused_workspace(p) : 0);
-  const size_t extra = cmp::proj_decode_workspace(p);
-  unsigned char* ws = nullptr;
-  rc = get_workspace(s, L.total + extra, &ws);
-  if (rc != CMP_OK) return rc;
-  p.err = reinterpret_cast<unsigned*>(ws + L.err);
-  p.m_cu = reinterpret_cast<int32_t*>(ws + L.m_cu);
-  p.m_s = reinterpret_cast<int32_t*>(ws + L.m_s);
-  p.m_off = reinterpret_cast<int32_t*>(ws + L.m_off);
-  p.m_tile = fused ? reinterpret_cast<int32_t*>(ws + L.m_tile) : nullptr;
-  p.proj = fused ? nullptr : reinterpret_cast<float*>(ws + L.proj);
-  p.ystat = fused ? reinterpret_cast<float*>(ws + L.ystat) : nullptr;
-  p.ylse = fused ? reinterpret_cast<float*>(ws + L.ylse) : nullptr;
-
-  // ---- kernels ----
-  if (which == 5) {  // decode: one cooperative kernel, no scheduler launch
-    float* part = reinterpret_cast<float*>(ws + L.part);
-    void* bar = ws + L.err + kGridBarOffset;
-    if (launch(CMP_KERNEL_DECODE_FUSED, s, [&] { return cmp::launch_decode_fused(p, part, bar, s); }) !=
-        cudaSuccess)
-      return CMP_ERR_CUDA;
-    return CMP_OK;
+  for (int attempt = 0; attempt < 2; ++attempt) {
+    const int r2 = run_path(p, choose_path(p, g_proj_kernel.load()), s);
+    // the device refused the channel-group decode's launch form (nothing ran):
+    // the path is now disabled there and the next choice is taken
+    if (r2 != kRetryOtherPath) return r2;
   }
-  if (launch(CMP_KERNEL_SCHED, s, [&] { return cmp::launch_sched(p, s); }) != cudaSuccess)
-    return CMP_ERR_CUDA;
-  cudaError_t e;
-  if (fused) {
-    const int sms = sm_count_cached();
-    e = launch(CMP_KERNEL_FUSED, s, [&] { return cmp::launch_fused(p, s, sms); });
-    if (e != cudaSuccess) return CMP_ERR_CUDA;
-    if (launch(CMP_KERNEL_FINISH, s, [&] { return cmp::launch_finish(p, s); }) != cudaSuccess)
-      return CMP_ERR_CUDA;
-    return CMP_OK;
-  }
-  if (which == 2)
-    e = launch(CMP_KERNEL_PROJ_TC, s, [&] { return cmp::launch_proj_tc(p, s); });
-  else if (which == 3)
-    e = launch(CMP_KERNEL_PROJ_DECODE, s, [&] { return cmp::launch_proj_decode(p, s); });
-  else
-    e = launch(CMP_KERNEL_PROJ_MMA, s, [&] { return cmp::launch_proj_mma(p, s); });
-  if (e != cudaSuccess) return CMP_ERR_CUDA;
-  if (launch(CMP_KERNEL_POOL, s, [&] { return cmp::launch_pool(p, s); }) != cudaSuccess)
-    return CMP_ERR_CUDA;
-  return CMP_OK;
+  return CMP_ERR_CUDA;
 }
+
 
 int cmp_get_error(void* stream) {
   cudaStream_t s = static_cast<cudaStream_t>(stream);
@@ -390,7 +433,7 @@ int cmp_get_error(void* stream) {
       if (v && cudaMemset(it->second.ptr, 0, sizeof(v)) != cudaSuccess) return CMP_ERR_CUDA;
       // a wait that gave up may have left the grid barrier's count behind
       if ((v & cmp::kErrTimeout) &&
-          cudaMemset(it->second.ptr + kGridBarOffset, 0, 2 * sizeof(unsigned)) != cudaSuccess)
+          cudaMemset(it->second.ptr + kGridBarOffset, 0, kHeaderBytes - kGridBarOffset) != cudaSuccess)
         return CMP_ERR_CUDA;
       word |= v;
     }
@@ -416,7 +459,7 @@ const char* cmp_status_string(int status) {
 const char* cmp_kernel_name(int kernel) {
   static const char* names[CMP_KERNEL_COUNT] = {"sched",         "proj_tcgen05",  "proj_mma_sync",
                                                 "proj_decode",   "pool_epilogue", "fused_tcgen05",
-                                                "finish",        "decode_fused"};
+                                                "finish",        "decode_fused",  "decode_cp"};
   return (kernel >= 0 && kernel < CMP_KERNEL_COUNT) ? names[kernel] : nullptr;
 }
 
@@ -457,7 +500,7 @@ int cmp_profile_stop(double* ms, int64_t* launches) {
 }
 
 int cmp_set_proj_kernel(int which) {
-  if (which < 0 || which > 5) return -1;
+  if (which < 0 || which > 6) return -1;
   return g_proj_kernel.exchange(which);
 }
 

@@ -13,6 +13,16 @@ __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
 
+// The first 1024-byte aligned address at or after `raw` (dynamic shared memory)
+// as a T. The offset is added to the shared array itself (not to an integer
+// copy of its address), so that accesses through the result stay shared-memory
+// accesses for the compiler instead of generic ones.
+template <class T>
+__device__ __forceinline__ T& smem_align1024(unsigned char* raw) {
+  const uint32_t a = smem_u32(raw);
+  return *reinterpret_cast<T*>(raw + (((a + 1023u) & ~1023u) - a));
+}
+
 __device__ __forceinline__ uint64_t globaltimer() {
   uint64_t t;
   asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));

@@ -35,7 +35,8 @@ def check(cmp, inp, rows=None):
     return out, kv, sc, res
 
 
-@pytest.fixture(params=[0, 1, 2, 3, 4, 5], ids=["auto", "mma", "tcgen05", "decode", "fused", "decode1k"])
+@pytest.fixture(params=[0, 1, 2, 3, 4, 5, 6],
+                ids=["auto", "mma", "tcgen05", "decode", "fused", "decode1k", "decodecp"])
 def proj_kernel(request, lib):
     prev = lib.set_proj_kernel(request.param)
     yield request.param
@@ -220,7 +221,7 @@ def test_projection_kernels_agree(lib):
                                 H=4096, D=512, coff=2, ratio=4, block_size=128, rotate=False))
     res = run_inputs(inp)
     outs = {}
-    for k in (1, 2, 3, 4, 5):
+    for k in (1, 2, 3, 4, 5, 6):
         prev = lib.set_proj_kernel(k)
         try:
             o, kv, sc, err = run(lib, inp)
@@ -232,6 +233,53 @@ def test_projection_kernels_agree(lib):
         assert_out_close(o, res)
         assert_state_close(kv, sc, inp, res)
         outs[k] = o
+
+
+# ---- the channel-group decode kernel -------------------------------------------------
+
+DECODE_CP_CASES = {
+    # name: lengths, start_pos, D, H, ratio, block_size
+    "c4a_32way": ([1] * 32, [4 * k + 3 for k in range(32)], 512, 4096, 4, 128),
+    "c4a_mixed_starts": ([1] * 24, [k for k in range(24)], 512, 4096, 4, 16),
+    "c4a_first_window": ([1, 1, 2, 3], [3, 0, 2, 1], 512, 1024, 4, 8),
+    "t64_multi_window": ([30, 17, 9, 8], [2, 0, 5, 61], 512, 2048, 4, 32),
+    "t48_ragged": ([20, 0, 27, 1], [6, 3, 0, 9], 128, 1024, 4, 4),
+    "ratio1": ([3, 5, 1], [0, 7, 2], 128, 512, 1, 8),
+    "ratio2": ([9, 4], [1, 6], 512, 1024, 2, 16),
+    "ratio8_tails": ([13, 2, 31], [5, 6, 3], 128, 2048, 8, 16),
+    "ratio64": ([1] * 6, [63, 127, 0, 64, 191, 5], 512, 1024, 64, 64),
+    "ratio128_overflow": ([1] * 8, [128 * k + 127 for k in range(8)], 512, 1024, 128, 128),
+    "single_token": ([1], [3], 512, 1024, 4, 16),
+    "wide_hidden": ([16, 5], [3, 0], 512, 16384, 4, 128),
+    "many_sequences": ([1] * 64, [4 * k + 3 - (k % 3) for k in range(64)], 128, 512, 4, 8),
+}
+
+
+@pytest.mark.parametrize("name", sorted(DECODE_CP_CASES))
+def test_decode_cp_cases(lib, name):
+    """Path 6 on windows that straddle start_pos, the first window (no previous
+    block), several windows per sequence, tails of every ratio, history rows past
+    the prefetch capacity (ratio 128, 8 x 127 state rows), T from 1 to 64."""
+    L, sp, D, H, ratio, bs = DECODE_CP_CASES[name]
+    inp = with_rope(make_inputs(name=name, seed=13, lengths=L, start_pos=sp, H=H, D=D,
+                                coff=2 if ratio == 4 else 1, ratio=ratio, block_size=bs,
+                                rotate=False, lookback=2 * ratio))
+    prev = lib.set_proj_kernel(6)
+    try:
+        lib.profile_start()
+        check(lib, inp)
+        launched = lib.profile_stop()
+    finally:
+        lib.set_proj_kernel(prev)
+    assert launched["decode_cp"][1] == 1, launched
+
+
+def test_decode_cp_is_the_automatic_decode_path(lib):
+    inp = with_rope(make_config("c4a_decode"))
+    lib.profile_start()
+    check(lib, inp)
+    launched = lib.profile_stop()
+    assert launched["decode_cp"][1] == 1 and sum(n for _, n in launched.values()) == 1, launched
 
 
 # ---- faults are reported, never trapped ------------------------------------------
