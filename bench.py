@@ -93,39 +93,84 @@ def job_throughput(units_per_rank: float, ws: int, ms_this_rank: float) -> float
 # ----------------------------------------------------------------------------
 
 class ClockSampler:
+    """SM clock, max clock and clock-event reasons sampled every 5 ms while the
+    timed region runs, read through NVML (read-only queries), or through
+    `nvidia-smi -lms 50` when NVML cannot be loaded."""
+
+    REASONS = (("hw_slowdown", 0x8), ("hw_thermal_slowdown", 0x40), ("sw_thermal_slowdown", 0x20),
+               ("sw_power_cap", 0x4))
     FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
               "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
               "clocks_event_reasons.sw_power_cap")
 
     def __init__(self, device_index: int):
-        self.samples = []
+        self.samples = []   # (sm_mhz, max_mhz, set of active reason names)
         self.proc = None
+        self.nvml = None
         self.dev = device_index
+        self.stop = threading.Event()
 
-    def __enter__(self):
+    def _uuid(self):
         try:
             import torch
             uuid = str(torch.cuda.get_device_properties(self.dev).uuid)
-            sel = ["-i", uuid if uuid.startswith("GPU-") else "GPU-" + uuid]
+            return uuid if uuid.startswith("GPU-") else "GPU-" + uuid
         except Exception:  # noqa: BLE001
-            sel = []
+            return None
+
+    def __enter__(self):
+        uuid = self._uuid()
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            h = pynvml.nvmlDeviceGetHandleByUUID(uuid) if uuid else pynvml.nvmlDeviceGetHandleByIndex(0)
+            self.nvml = (pynvml, h)
+            self.thread = threading.Thread(target=self._poll_nvml, daemon=True)
+            self.thread.start()
+            return self
+        except Exception:  # noqa: BLE001 - fall back to nvidia-smi
+            self.nvml = None
         try:
             self.proc = subprocess.Popen(
-                ["nvidia-smi", *sel, f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-lms", "50"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-            self.thread = threading.Thread(target=self._read, daemon=True)
+                ["nvidia-smi", *(["-i", uuid] if uuid else []), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "50"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read_smi, daemon=True)
             self.thread.start()
         except OSError:
             self.proc = None
         return self
 
-    def _read(self):
+    def _poll_nvml(self):
+        nv, h = self.nvml
+        while not self.stop.is_set():
+            try:
+                sm = nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)
+                mx = nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM)
+                bits = nv.nvmlDeviceGetCurrentClocksEventReasons(h)
+                self.samples.append((float(sm), float(mx), {n for n, b in self.REASONS if bits & b}))
+            except Exception:  # noqa: BLE001
+                pass
+            self.stop.wait(0.005)
+
+    def _read_smi(self):
+        names = [n for n, _ in self.REASONS]
         for line in self.proc.stdout:
             parts = [p.strip() for p in line.split(",")]
-            if len(parts) == 7:
-                self.samples.append(parts)
+            if len(parts) != 7:
+                continue
+            num = lambda v: float(v) if v.replace(".", "", 1).isdigit() else None
+            self.samples.append((num(parts[0]), num(parts[1]),
+                                 {names[i] for i in range(4) if parts[3 + i].lower() == "active"}))
 
     def __exit__(self, *a):
+        self.stop.set()
+        if self.nvml:
+            self.thread.join(timeout=2)
+            try:
+                self.nvml[0].nvmlShutdown()
+            except Exception:  # noqa: BLE001
+                pass
         if self.proc:
             self.proc.terminate()
             try:
@@ -134,17 +179,14 @@ class ClockSampler:
                 self.proc.kill()
 
     def summary(self):
-        if not self.samples:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
-        num = lambda v: float(v) if v.replace(".", "", 1).isdigit() else None
-        sm = [num(s[0]) for s in self.samples if num(s[0]) is not None]
-        mx = [num(s[1]) for s in self.samples if num(s[1]) is not None]
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({names[i] for s in self.samples for i in range(4)
-                          if s[3 + i].lower() == "active"})
-        return {"sm_mhz": statistics.median(sm) if sm else None,
-                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
-                "samples": len(self.samples)}
+        sm = [s[0] for s in self.samples if s[0] is not None]
+        mx = [s[1] for s in self.samples if s[1] is not None]
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"], "samples": 0}
+        reasons = sorted(set().union(*[s[2] for s in self.samples]))
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(self.samples),
+                "source": "nvml" if self.nvml else "nvidia-smi"}
 
 
 # ----------------------------------------------------------------------------
@@ -294,16 +336,23 @@ def bench_prefill(args, ws, local, stream, peaks, peak_src):
     T, H, C = PREFILL["T"], PREFILL["H"], PREFILL["D"]
     flops = 2.0 * T * H * 2 * C
     achieved = flops / (p_ms / p_n / 1e3) / 1e12 if p_n else None
-    peak = peaks["bf16_tflops"]
+    clocks = clk.summary()
+    # burst peak for a short timed region; the sustained (power-capped) one when
+    # the clocks show the power cap during it
+    sustained = "sw_power_cap" in clocks.get("reasons", []) and "bf16_tflops_sustained" in peaks
+    peak = peaks["bf16_tflops_sustained"] if sustained else peaks["bf16_tflops"]
     kfile = {"proj_tcgen05": "cmp_proj_tc.cu", "proj_mma_sync": "cmp_proj_mma.cu",
              "proj_decode": "cmp_proj_decode.cu", "fused_tcgen05": "cmp_fused_tc.cu"}[proj_name]
     roofline = {"kernel": proj_name, "bound": "tensor", "achieved": achieved, "peak": peak,
                 "unit": "TFLOP/s", "frac": achieved / peak if achieved else None,
                 "traffic": traffic_for(kfile, proj_name, T / 131072.0),
-                "peak_source": peak_src + " (burst)", "algorithmic_flops_per_launch": flops,
+                "peak_source": peak_src + (" (sustained: sw_power_cap during the timed region)"
+                                           if sustained else " (burst)"),
+                "frac_of_burst": achieved / peaks["bf16_tflops"] if achieved else None,
+                "algorithmic_flops_per_launch": flops,
                 "kernel_ms": {k: (v[0] / v[1] if v[1] else None) for k, v in prof.items()}}
     return dict(value=value, ms_step=ms / args.steps, launches=launches, roofline=roofline,
-                clocks=clk.summary(), inputs=pf, out=out)
+                clocks=clocks, inputs=pf, out=out)
 
 
 def bench_e2e(args, ws, stream, pf, out):

@@ -21,7 +21,7 @@ size_t decode_fused_workspace(const Params& p);
 cudaError_t launch_decode_fused(const Params& p, float* part, void* bar, cudaStream_t s);
 bool decode_cp_supported(const Params& p);
 size_t decode_cp_workspace(const Params& p);
-cudaError_t launch_decode_cp(const Params& p, float* ss, void* bar, cudaStream_t s);
+cudaError_t launch_decode_cp(const Params& p, float* ss, void* counter, cudaStream_t s);
 }  // namespace cmp
 
 namespace {
@@ -30,12 +30,15 @@ using cmp::Params;
 
 // ---- workspace ---------------------------------------------------------------
 
-// The first kHeaderBytes (zeroed when the workspace is created) hold the error
-// word at offset 0, the K-split decode kernel's grid-barrier words at offset 64
-// and the channel-group decode kernel's barrier counters at offset 256.
+// The first kHeaderBytes (zeroed when the workspace is created, and after a
+// timeout) hold the error word at offset 0, the K-split decode kernel's
+// grid-barrier words at offset 64 and the channel-group decode kernel's
+// barrier counter at offset 256; only those kernels write there.
 constexpr size_t kHeaderBytes = 2048;
 constexpr size_t kGridBarOffset = 64;
-constexpr size_t kGridBar2Offset = 256;
+constexpr size_t kCounterOffset = 256;
+
+size_t zeroed_bytes() { return kHeaderBytes; }
 
 struct WsLayout {
   size_t err, m_cu, m_s, m_off, m_tile, proj, ystat, ylse, part, total;
@@ -51,7 +54,7 @@ WsLayout ws_layout(int64_t B, int64_t T, int64_t C, int64_t n_out, bool fused, s
     o += (n + 255) & ~size_t(255);
     return r;
   };
-  L.err = take(kHeaderBytes);
+  L.err = take(zeroed_bytes());
   L.m_cu = take(sizeof(int32_t) * (B + 1));
   L.m_s = take(sizeof(int32_t) * std::max<int64_t>(B, 1));
   L.m_off = take(sizeof(int32_t) * (B + 1));
@@ -180,7 +183,7 @@ int get_workspace(cudaStream_t s, size_t need, unsigned char** out) {
   const size_t bytes = std::max(need, size_t(1) << 20);
   void* p = nullptr;
   if (cudaMalloc(&p, bytes) != cudaSuccess) return CMP_ERR_CUDA;
-  if (cudaMemset(p, 0, kHeaderBytes) != cudaSuccess) {
+  if (cudaMemset(p, 0, zeroed_bytes()) != cudaSuccess) {
     cudaFree(p);
     return CMP_ERR_CUDA;
   }
@@ -238,9 +241,9 @@ int run_path(Params& p, int which, cudaStream_t s) {
   // ---- kernels ----
   if (which == 6) {  // decode: one cooperative kernel of clusters, no scheduler launch
     float* ss = reinterpret_cast<float*>(ws + L.part);
-    void* bar = ws + L.err + kGridBar2Offset;
+    void* counter = ws + L.err + kCounterOffset;
     const cudaError_t e =
-        launch(CMP_KERNEL_DECODE_CP, s, [&] { return cmp::launch_decode_cp(p, ss, bar, s); });
+        launch(CMP_KERNEL_DECODE_CP, s, [&] { return cmp::launch_decode_cp(p, ss, counter, s); });
     if (e == cudaErrorNotSupported) return kRetryOtherPath;
     return e == cudaSuccess ? CMP_OK : CMP_ERR_CUDA;
   }
@@ -433,7 +436,7 @@ int cmp_get_error(void* stream) {
       if (v && cudaMemset(it->second.ptr, 0, sizeof(v)) != cudaSuccess) return CMP_ERR_CUDA;
       // a wait that gave up may have left the grid barrier's count behind
       if ((v & cmp::kErrTimeout) &&
-          cudaMemset(it->second.ptr + kGridBarOffset, 0, kHeaderBytes - kGridBarOffset) != cudaSuccess)
+          cudaMemset(it->second.ptr + kGridBarOffset, 0, zeroed_bytes() - kGridBarOffset) != cudaSuccess)
         return CMP_ERR_CUDA;
       word |= v;
     }

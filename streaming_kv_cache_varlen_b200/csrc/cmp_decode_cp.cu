@@ -59,8 +59,7 @@ constexpr int kMaxWinRows = 128;  // coff * ratio
 constexpr int KPS = 2;            // 64-column K blocks per TMA copy (pipeline stage)
 constexpr int kTileA = 8192;      // one K block of A: 2 matrices x 2 halves x 16 rows x 128 B
 constexpr int kSlackA = 16384 - kTileA;  // the 128-row window the MMA reads past the last tile
-constexpr int kPartStride = 68;   // floats per token row of the TMEM copy (64 rows + pad)
-constexpr int kReplicas = 4;      // copies of the sum-of-squares partials (spread the readers)
+constexpr int kReplicas = 16;     // copies of the sum-of-squares partials (spread the readers)
 
 template <int MAXT>
 struct Cfg {
@@ -91,8 +90,7 @@ struct Smem {
   alignas(1024) unsigned char a[S][KPS * kTileA];
   unsigned char a_slack[kSlackA];
   alignas(1024) __nv_bfloat16 x[S][KPS * MAXT * BK];
-  alignas(16) float recv[KQ][4][MAXT][OWN];   // partials pushed by the cluster's CTAs
-  alignas(16) float own[4][MAXT][OWN];        // complete projections [kind][token][channel]
+  alignas(16) float recv[KQ][4 * MAXT * OWN]; // partials from each CTA of the cluster: [kind][token][channel]
   alignas(16) float hist[kHistRows][2 * OWN];  // state rows: kv c0..c3, score c0..c3
   alignas(16) float ape[kMaxWinRows][OWN];     // ape of window row j (half * ratio + residue)
   alignas(16) float rope[kMaxOut][8];          // per pair: cos even, cos odd, sin even, sin odd
@@ -110,11 +108,12 @@ struct Smem {
   uint64_t full[S];
   uint64_t empty[S];
   uint64_t acc_full;
+  uint64_t recv_full;   // the four partial blocks have landed in recv
   uint32_t tmem_base;
   int abort;
   int rejected;
-  int grid_ok;
   uint32_t bar_target;
+  int grid_ok;
 };
 
 static_assert(offsetof(Smem<32>, x) % 1024 == 0 && offsetof(Smem<64>, x) % 1024 == 0,
@@ -123,14 +122,13 @@ static_assert(offsetof(Smem<32>, a_slack) == sizeof(Smem<32>::a) &&
                   offsetof(Smem<64>, a_slack) == sizeof(Smem<64>::a),
               "the MMA's 128-row window past the last stage must stay inside the slack");
 static_assert(offsetof(Smem<32>, recv) % 16 == 0 && offsetof(Smem<64>, recv) % 16 == 0 &&
-                  offsetof(Smem<32>, own) % 16 == 0 && offsetof(Smem<64>, own) % 16 == 0 &&
                   offsetof(Smem<32>, hist) % 16 == 0 && offsetof(Smem<64>, hist) % 16 == 0 &&
                   offsetof(Smem<32>, ape) % 16 == 0 && offsetof(Smem<64>, ape) % 16 == 0 &&
                   offsetof(Smem<32>, ybuf) % 16 == 0 && offsetof(Smem<64>, ybuf) % 16 == 0,
               "float4 shared-memory rows must be 16-byte aligned");
-static_assert(64 * kPartStride * 4 <= Cfg<64>::stages * KPS * kTileA &&
-                  32 * kPartStride * 4 <= Cfg<32>::stages * KPS * kTileA,
-              "the TMEM copy must fit in the stage buffers");
+static_assert(KQ * 4 * 64 * OWN * 4 <= Cfg<64>::stages * KPS * kTileA &&
+                  KQ * 4 * 32 * OWN * 4 <= Cfg<32>::stages * KPS * kTileA,
+              "the outgoing partial blocks must fit in the stage buffers");
 static_assert(sizeof(Smem<32>) + 1024 <= 232448 && sizeof(Smem<64>) + 1024 <= 232448,
               "shared memory per CTA");
 
@@ -145,32 +143,26 @@ static_assert(sizeof(Smem<32>) + 1024 <= 232448 && sizeof(Smem<64>) + 1024 <= 23
 // No reset and no last-arriver step: nothing serializes behind one CTA.
 constexpr uint32_t kQuantum = 1024;
 
-struct GridBar {
-  unsigned count;
-};
-
-__device__ __forceinline__ uint32_t grid_target(const GridBar* bar) {
+__device__ __forceinline__ uint32_t grid_target(const unsigned* counter) {
   uint32_t v;
-  asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(&bar->count) : "memory");
+  asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(counter) : "memory");
   return v - v % kQuantum + kQuantum;
 }
 
-__device__ __forceinline__ void grid_arrive(GridBar* bar, unsigned nblocks) {
-  asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(&bar->count), "r"(kQuantum / nblocks)
-               : "memory");
+__device__ __forceinline__ void grid_arrive(unsigned* counter, unsigned nblocks) {
+  asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(counter), "r"(kQuantum / nblocks) : "memory");
 }
 
-__device__ __forceinline__ bool grid_wait(const GridBar* bar, uint32_t target, unsigned* err) {
+__device__ __forceinline__ bool grid_wait(const unsigned* counter, uint32_t target, unsigned* err) {
   const uint64_t t0 = globaltimer();
   for (;;) {
     uint32_t now;
-    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(now) : "l"(&bar->count) : "memory");
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(now) : "l"(counter) : "memory");
     if ((int32_t)(now - target) >= 0) return true;
     if (globaltimer() - t0 > 1000000000ull) {
       atomicOr(err, kErrTimeout);
       return false;
     }
-    __nanosleep(20);
   }
 }
 
@@ -184,21 +176,33 @@ __device__ __forceinline__ void cluster_arrive_relaxed() {
   asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
 }
 
-__device__ __forceinline__ void cluster_arrive() {
-  asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
-}
-
 __device__ __forceinline__ void cluster_wait() {
   asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
 
-// Store v at `local` in the shared memory of cluster CTA `peer`.
-__device__ __forceinline__ void st_peer_f4(void* local, uint32_t peer, float4 v) {
+// The shared::cluster address of `local` in cluster CTA `peer`.
+__device__ __forceinline__ uint32_t peer_addr(const void* local, uint32_t peer) {
   uint32_t ra;
   asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(ra) : "r"(smem_u32(local)), "r"(peer));
-  asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(ra), "f"(v.x), "f"(v.y), "f"(v.z),
-               "f"(v.w)
-               : "memory");
+  return ra;
+}
+
+// Bulk copy of `bytes` from this CTA's shared memory into a peer's, completing
+// on the peer's mbarrier (both addresses from peer_addr). No multicast.
+__device__ __forceinline__ void bulk_copy_to_peer(uint32_t dst, const void* src, uint32_t bytes, uint32_t mbar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+      "r"(smem_u32(src)), "r"(bytes), "r"(mbar)
+      : "memory");
+}
+
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+
+__device__ __forceinline__ void bulk_wait_read() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+
+// Generic-proxy writes to shared memory before async-proxy reads of it.
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
 // TMA copies of 3-D and 5-D boxes into shared memory, completing on an mbarrier.
@@ -225,8 +229,8 @@ __device__ __forceinline__ float4 add4(float4 a, float4 b) {
 }
 
 struct CpArgs {
-  float* ss;        // [kReplicas][n_out][D/4] each CTA's sum of squares of its channels, per output row
-  GridBar* bar;
+  float* ss;          // [kReplicas][n_out][D/4] each CTA's sum of squares of its channels, per output row
+  unsigned* counter;  // grid-barrier counter (zeroed at creation)
   int kv_first;     // the 4-D weight map holds wkv before wgate (else the other way round)
 };
 
@@ -297,10 +301,7 @@ __device__ void call_metadata(const Params& p, Smem<MAXT>& sm, int NT, int ch0) 
   }
   // these loads are issued: let the weight stream start behind them
   asm volatile("bar.arrive 3, 96;" ::: "memory");
-  // cluster barrier 0 (every CTA of the cluster runs), then barrier 1 at once:
-  // these warps push nothing, so their prefetch overlaps the others' pushes
-  cluster_wait();
-  cluster_arrive_relaxed();
+  cluster_wait();  // cluster barrier 0 (every CTA of the cluster runs)
 #pragma unroll
   for (int u = 0; u < 5; ++u)
     if (et + 64 * u <= B) sm.cu[et + 64 * u] = cuv[u];
@@ -505,6 +506,21 @@ __device__ void call_metadata(const Params& p, Smem<MAXT>& sm, int NT, int ch0) 
   }
 }
 
+// The complete projection of kind k, token t, channel c of this CTA: the four
+// received partial blocks added in rank order.
+template <int MAXT>
+__device__ __forceinline__ float own_value(const Params& p, const Smem<MAXT>& sm, int k, int t, int c) {
+  const int i = (k * p.T + t) * OWN + c;
+  return ((sm.recv[0][i] + sm.recv[1][i]) + sm.recv[2][i]) + sm.recv[3][i];
+}
+
+__device__ __forceinline__ float4 own_value4(const float* r0, const float* r1, const float* r2, const float* r3) {
+  const float4 a = *reinterpret_cast<const float4*>(r0), b = *reinterpret_cast<const float4*>(r1);
+  const float4 c = *reinterpret_cast<const float4*>(r2), d = *reinterpret_cast<const float4*>(r3);
+  return make_float4(((a.x + b.x) + c.x) + d.x, ((a.y + b.y) + c.y) + d.y, ((a.z + b.z) + c.z) + d.z,
+                     ((a.w + b.w) + c.w) + d.w);
+}
+
 // Window row j's kv and score (score + ape for this call's tokens) for channel c.
 template <int MAXT>
 __device__ __forceinline__ void window_row(const Params& p, const Smem<MAXT>& sm, const Win& w, int j, int c,
@@ -516,8 +532,8 @@ __device__ __forceinline__ void window_row(const Params& p, const Smem<MAXT>& sm
     const int r = p.ratio;
     const int half = (p.coff == 2 && j >= r) ? 1 : 0;
     const int t = w.cu + (window_pos(w.w, j, r, p.coff) - w.s);
-    kv = sm.own[half][t][c];
-    z = sm.own[p.coff + half][t][c] + sm.ape[j][c];
+    kv = own_value(p, sm, half, t, c);
+    z = own_value(p, sm, p.coff + half, t, c) + sm.ape[j][c];
   }
 }
 
@@ -537,7 +553,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int nsteps = p.H / (KQ * KPS * BK);   // pipeline steps per CTA (KPS K blocks each)
   const uint32_t bytes = KPS * ((uint32_t)kinds * GCH * BK * 2 + (uint32_t)NT * BK * 2);
   const uint32_t tmem_cols = NT <= 32 ? 32 : 64;
-  float* part = reinterpret_cast<float*>(&sm.a[0][0]);  // [token][kPartStride], after the MMAs
+  // after the MMAs: the outgoing partials, one block per owner CTA [owner][kind][token][channel]
+  float* part = reinterpret_cast<float*>(&sm.a[0][0]);
+  const int blk_floats = kinds * p.T * OWN;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -545,14 +563,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&sm.empty[s], 1);
     }
     mbar_init(&sm.acc_full, 1);
+    mbar_init(&sm.recv_full, 1);
     sm.abort = 0;
     fence_barrier_init();
+    // the four incoming partial blocks (one of them this CTA's own)
+    mbar_arrive_expect_tx(&sm.recv_full, (uint32_t)(KQ * kinds * p.T * OWN * 4));
     prefetch_tmap(&map_w);
     prefetch_tmap(&map_x);
-    sm.bar_target = grid_target(a.bar);
+    sm.bar_target = grid_target(a.counter);
   }
   if (warp == 1) tmem_alloc(&sm.tmem_base, tmem_cols);
-  cluster_arrive_relaxed();  // cluster barrier 0: this CTA runs (the peers may write its shared memory)
+  cluster_arrive_relaxed();  // cluster barrier 0: this CTA runs (its barriers are initialized)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -601,56 +622,58 @@ __global__ void __launch_bounds__(kThreads, 1)
     call_metadata<MAXT>(p, sm, NT, ch0);
   }
 
-  // ---- 2) warps 0-1: TMEM rows -> part[token][row], then push each owner its
-  // channels' partials; everyone then adds the four ----
+  // ---- 2) warps 0-1: TMEM rows -> the owners' blocks, one bulk copy per owner;
+  // every CTA then adds the four blocks it received (in rank order) ----
   if (warp < 2) {
     const bool have = mbar_wait(&sm.acc_full, 0, abort);
     __syncwarp();
     if (__all_sync(0xffffffffu, have) && warp * 32 < kinds * GCH) {
       tc_fence_after();
-      const int row = warp * 32 + lane;
+      // TMEM lane = A row: 16-row block of the tile, channel of the cluster's 16
+      const int row = warp * 32 + lane, b = row / GCH, cg = row % GCH;
+      const int k = a.kv_first ? b : (b + p.coff) % kinds;  // kind of that block
+      float* dst = part + (cg / OWN) * blk_floats + k * p.T * OWN + cg % OWN;
       for (int c0 = 0; c0 < NT; c0 += 32) {
         uint32_t r[32];
         tmem_ld32(tmem + ((uint32_t)(warp * 32) << 16) + c0, r);
         tmem_ld_wait(r);
 #pragma unroll
         for (int j = 0; j < 32; ++j)
-          if (c0 + j < p.T) part[(c0 + j) * kPartStride + row] = __uint_as_float(r[j]);
+          if (c0 + j < p.T) dst[(c0 + j) * OWN] = __uint_as_float(r[j]);
       }
     }
     tc_fence_before();
+    fence_proxy_async_smem();  // the blocks are read by the bulk copies
     asm volatile("bar.sync 1, 64;" ::: "memory");
-    cluster_wait();  // every CTA of the cluster runs
-    for (int i = threadIdx.x; i < KQ * kinds * p.T; i += 64) {
-      const int dst = i / (kinds * p.T), rem = i % (kinds * p.T);
-      const int k = rem / p.T, t = rem % p.T;
-      const int blk = a.kv_first ? k : (k + p.coff) % kinds;  // the kind's 16-row block in the A tile
-      const float4 v = *reinterpret_cast<const float4*>(part + t * kPartStride + blk * GCH + dst * OWN);
-      st_peer_f4(&sm.recv[q][k][t][0], (uint32_t)dst, v);
+    cluster_wait();  // cluster barrier 0: every CTA of the cluster runs, its barriers initialized
+    if (threadIdx.x == 0) {
+      const uint32_t bytes = (uint32_t)blk_floats * 4;
+      for (int o = 0; o < KQ; ++o)
+        bulk_copy_to_peer(peer_addr(&sm.recv[q][0], (uint32_t)o), part + o * blk_floats, bytes,
+                          peer_addr(&sm.recv_full, (uint32_t)o));
+      bulk_commit();
     }
-    cluster_arrive();  // the pushes are performed before barrier 1 completes
   }
-  cluster_wait();
-  __syncthreads();  // and the metadata is complete
+  if (threadIdx.x == 0) {
+    // not cut short by this CTA's abort flag: the peers' copies into this CTA
+    // must land before it goes on (and, at the latest, before it exits)
+    int never = 0;
+    if (!mbar_wait(&sm.recv_full, 0, &never)) atomicOr(p.err, kErrTimeout);
+  }
+  __syncthreads();  // the partials have landed, and the metadata is complete
   const bool mm_ok = !*abort;
-  for (int i = threadIdx.x; i < kinds * p.T; i += kThreads) {
-    const int k = i / p.T, t = i % p.T;
-    float4 acc = *reinterpret_cast<const float4*>(&sm.recv[0][k][t][0]);
-#pragma unroll
-    for (int s = 1; s < KQ; ++s) acc = add4(acc, *reinterpret_cast<const float4*>(&sm.recv[s][k][t][0]));
-    *reinterpret_cast<float4*>(&sm.own[k][t][0]) = acc;
-  }
-  __syncthreads();
 
-  // ---- 3) pooling: warp per window; lane = channel * 8 + row lane ----
+  // ---- 3) pooling: 16 threads per window (4 channels x 4 row lanes), 8 windows at a time ----
   const int r = p.ratio, n_out = p.n_out, rows = p.coff * r, nw = sm.n_win;
   {
-    const int c = lane >> 3, rl = lane & 7;
-    for (int wi = warp; wi < nw; wi += 4) {
-      const int n = sm.wlist[wi];
-      const Win w = sm.win[n];
+    const int c = (threadIdx.x >> 2) & 3, rl = threadIdx.x & 3;
+    for (int wi = threadIdx.x >> 4; wi < nw + 7 - ((nw + 7) % 8); wi += kThreads / 16) {
+      // every lane runs the shuffles; lanes past the last window compute nothing
+      const bool live = wi < nw && mm_ok;
+      const int n = live ? sm.wlist[wi] : 0;
+      Win w = sm.win[n];
       float m = -INFINITY, l = 0.f, acc = 0.f;
-      for (int j = rl; j < rows && mm_ok; j += 8) {
+      for (int j = rl; j < rows && live; j += 4) {
         float kv, z;
         if (j < w.hrows && w.hist < 0) {  // more state rows than the prefetch holds
           const int qp = window_pos(w.w, j, r, p.coff);
@@ -671,9 +694,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         acc = acc * f + e * kv;
         m = mn;
       }
-      // merge the 8 row lanes of each channel (log-sum-exp)
+      // merge the 4 row lanes of each channel (log-sum-exp)
 #pragma unroll
-      for (int o = 1; o < 8; o <<= 1) {
+      for (int o = 1; o < 4; o <<= 1) {
         const float m2 = __shfl_xor_sync(0xffffffffu, m, o);
         const float l2 = __shfl_xor_sync(0xffffffffu, l, o);
         const float a2 = __shfl_xor_sync(0xffffffffu, acc, o);
@@ -684,7 +707,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         acc = acc * f1 + a2 * f2;
         m = mn;
       }
-      if (rl == 0) sm.ybuf[n][c] = l > 0.f ? acc / l : 0.f;
+      if (live && rl == 0) sm.ybuf[n][c] = l > 0.f ? __fdividef(acc, l) : 0.f;
     }
   }
   __syncthreads();
@@ -697,7 +720,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         y.x * y.x + y.y * y.y + y.z * y.z + y.w * y.w;
   }
   __syncthreads();
-  if (threadIdx.x == 0) grid_arrive(a.bar, n_cta);
+  if (threadIdx.x == 0) grid_arrive(a.counter, n_cta);
 
   // ---- while the other CTAs arrive: state tails and rows without a window ----
   for (int i = threadIdx.x; i < kinds * p.T && mm_ok; i += kThreads) {
@@ -707,13 +730,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int64_t so = score ? ti.sc_off : ti.kv_off;
     if (ti.b < 0 || so < 0) continue;
     const int half = score ? k - p.coff : k;
-    float4 v = *reinterpret_cast<const float4*>(&sm.own[k][t][0]);
+    const int e = (k * p.T + t) * OWN;
+    float4 v = own_value4(&sm.recv[0][e], &sm.recv[1][e], &sm.recv[2][e], &sm.recv[3][e]);
     if (score) v = add4(v, *reinterpret_cast<const float4*>(&sm.ape[half * r + ti.pos % r][0]));
     *reinterpret_cast<float4*>((score ? p.score_state : p.kv_state) + so + half * p.D + ch0) = v;
   }
   for (int n = threadIdx.x; n < n_out; n += kThreads)
     if (sm.win[n].w < 0) *reinterpret_cast<uint2*>(p.out + (int64_t)n * p.D + ch0) = make_uint2(0u, 0u);
-  if (threadIdx.x == 0) sm.grid_ok = grid_wait(a.bar, sm.bar_target, p.err) ? 1 : 0;
+  if (threadIdx.x == 0) sm.grid_ok = grid_wait(a.counter, sm.bar_target, p.err) ? 1 : 0;
   __syncthreads();
   const bool ok = sm.grid_ok != 0 && mm_ok;
 
@@ -726,7 +750,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
       for (int u = 0; u < 8; ++u) {
         const int n = sm.wlist[warp + 4 * (u0 + u < mine ? u0 + u : u0)];
-        const float* row = a.ss + (int64_t)(q % kReplicas) * rep_stride + (int64_t)n * n_cta;
+        const float* row = a.ss + (int64_t)(blockIdx.x % kReplicas) * rep_stride + (int64_t)n * n_cta;
         v[u] = lane < nq ? __ldcg(reinterpret_cast<const float4*>(row) + lane) : make_float4(0.f, 0.f, 0.f, 0.f);
       }
       float t[8];
@@ -771,6 +795,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     *reinterpret_cast<uint2*>(p.out + (int64_t)n * p.D + ch0) = v;
   }
 
+  if (threadIdx.x == 0) bulk_wait_read();  // this CTA's outgoing copies have read its blocks
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
@@ -910,14 +935,14 @@ size_t decode_cp_workspace(const Params& p) {
 // Launch. If the device refuses the launch form itself (a cooperative launch of
 // clusters), the path is disabled on this device and cudaErrorNotSupported is
 // returned before anything ran, so that the caller can take another path.
-cudaError_t launch_decode_cp(const Params& p, float* ss, void* bar, cudaStream_t s) {
+cudaError_t launch_decode_cp(const Params& p, float* ss, void* counter, cudaStream_t s) {
   const int NT = (p.T + 15) / 16 * 16;
   CUtensorMap mx, mw;
   CpArgs a;
   if (!make_x_map(&mx, p.x, p.T, p.H, (uint32_t)NT) || !make_w_map(&mw, p, &a.kv_first))
     return cudaErrorInvalidValue;
   a.ss = ss;
-  a.bar = static_cast<GridBar*>(bar);
+  a.counter = static_cast<unsigned*>(counter);
   const int grid = (p.D / GCH) * KQ;
   cudaLaunchAttribute attr[2];
   cudaError_t e;
