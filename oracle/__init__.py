@@ -8,16 +8,21 @@ generators in ``workloads``.
 * ``oracle.compressor`` — the definition in float64 (numpy), step by step.
 * ``oracle.brute`` — a pure-Python restatement from the closed-form formula,
   for tiny inputs, used to pin the former.
+* ``oracle.nsa`` — NsaCompressWithCache (the second workload): the weighted sum
+  of a batch's last compress_block_size cached tokens, written to its slot,
+  with its own brute-force restatement.
 
 Parity status: pinned. No page prints a numeric example of this operator, so
 the pins are brute force on tiny inputs, closed forms (equal scores give the
 window mean, one dominant score selects its row, masked first window, RMSNorm
 unit rms, RoPE identity and pair norms, Hadamard orthogonality) and the
 streaming invariants (token by token, chunked and reordered calls equal one
-call). See tests/test_oracle_pins.py.
+call). See tests/test_oracle_pins.py. ``oracle.nsa`` is pinned by the example
+of its page (a closed form on its all-ones inputs), brute force, the trigger
+rule and closed forms (tests/test_oracle_nsa.py).
 """
 
-from . import brute, compressor  # noqa: F401
+from . import brute, compressor, nsa  # noqa: F401
 from .compressor import (  # noqa: F401
     Layout,
     Result,

@@ -18,3 +18,4 @@ from .synth import (  # noqa: F401
     rope_tables,
     sylvester,
 )
+from .nsa import NsaInputs, make_nsa_inputs  # noqa: F401,E402
