@@ -481,6 +481,83 @@ def bench_decode(args, ws, local, stream, peaks, peak_src):
             "kernel_us_eager": {k: (v[0] / v[1] * 1e3 if v[1] else None) for k, v in dprof.items()}}
 
 
+NSA = dict(B=128, N=24, D=192, page=128, cbs=32, stride=16, max_seq=512)
+
+
+def bench_nsa(args, ws, local, peaks, peak_src):
+    """NsaCompressWithCache, one decode step in which all 128 batches reach a
+    compression step: N=24 heads of D=192 (the shapes of its page's example), bf16,
+    paged cache (page 128), window 32, stride 16. Device time per call from graph
+    replays of 50 x (256 MB L2 flush + call) minus 50 flushes; the algorithmic bytes
+    are the windows read once plus the slots written."""
+    import torch
+
+    import streaming_kv_cache_varlen_b200 as cmp
+
+    c = NSA
+    device = torch.device("cuda", local)
+    g = torch.Generator(device=device).manual_seed(4)
+    per = c["max_seq"] // c["page"]
+    block_num = c["B"] * per
+    bf = torch.bfloat16
+    inp = torch.randn((block_num, c["page"], c["N"], c["D"]), generator=g, device=device).to(bf)
+    weight = (torch.randn((c["cbs"], c["N"]), generator=g, device=device) / c["cbs"] ** 0.5).to(bf)
+    table = torch.randperm(block_num, generator=g, device=device).to(torch.int32).view(c["B"], per)
+    steps = (c["max_seq"] - c["cbs"]) // c["stride"] + 1
+    lens = (c["cbs"] + c["stride"] * torch.randint(0, steps, (c["B"],), generator=g, device=device)).to(torch.int64)
+    result_len = 4 * c["B"]
+    slots = torch.randperm(result_len, generator=g, device=device)[:c["B"]].to(torch.int32)
+    out = torch.zeros((result_len, c["N"], c["D"]), dtype=bf, device=device)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=device)
+
+    def call():
+        cmp.nsa_compress(inp, weight, slots, lens, out, compress_block_size=c["cbs"],
+                         compress_stride=c["stride"], block_table=table, page_block_size=c["page"])
+
+    side = torch.cuda.Stream(device)
+    with torch.cuda.stream(side):
+        for _ in range(max(3, args.warmup)):
+            call()
+            flush.fill_(1)
+    torch.cuda.synchronize()
+    n = 50
+    g_call, g_flush = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g_call, stream=side):
+        for _ in range(n):
+            flush.fill_(1)
+            call()
+    with torch.cuda.graph(g_flush, stream=side):
+        for _ in range(n):
+            flush.fill_(1)
+    torch.cuda.synchronize()
+
+    def replay(gr):
+        best = None
+        for _ in range(5):
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            with torch.cuda.stream(side):
+                a.record(side)
+                gr.replay()
+                b.record(side)
+            torch.cuda.synchronize()
+            best = a.elapsed_time(b) if best is None else min(best, a.elapsed_time(b))
+        return best
+
+    barrier(ws)
+    us = max_over_ranks((replay(g_call) - replay(g_flush)) * 1e3 / n, ws)
+    assert cmp.get_error(side) == 0
+    del g_call, g_flush
+    plane = c["N"] * c["D"] * 2
+    nbytes = c["B"] * (c["cbs"] + 1) * plane + c["cbs"] * c["N"] * 2
+    ach = nbytes / (us / 1e6) / 1e9
+    return {"workload": f"nsa_decode_step: {c['B']} batches on a compression step, N={c['N']}, "
+                        f"D={c['D']}, bf16, paged (page {c['page']}), window {c['cbs']}, stride {c['stride']}",
+            "us_per_call": us, "timing": "CUDA-graph replay of 50 x (L2 flush + call) minus 50 flushes, / 50",
+            "roofline": {"bound": "hbm", "achieved": ach, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                         "frac": ach / peaks["hbm_gbs"], "algorithmic_bytes_per_call": nbytes,
+                         "peak_source": peak_src}}
+
+
 def run_ours(args):
     import torch
 
@@ -500,6 +577,10 @@ def run_ours(args):
         torch.cuda.empty_cache()
     if args.only in ("all", "decode"):
         decode = bench_decode(args, ws, local, stream, peaks, peak_src)
+    nsa = None
+    if args.only in ("all", "nsa"):
+        nsa = bench_nsa(args, ws, local, peaks, peak_src)
+        torch.cuda.empty_cache()
     cpu = None
     if rank == 0 and ws == 1 and args.only == "all" and not args.no_cpu_baseline:
         cpu = cpu_baseline(args.cpu_tokens)
@@ -516,7 +597,7 @@ def run_ours(args):
                            "parallelism": f"dp{ws} (independent replicas)",
                            "l2": "inputs larger than L2 (x is 1 GiB per step)"},
                 "e2e": e2e, "gpu_launches": pre["launches"] if pre else None,
-                "roofline": pre["roofline"] if pre else None, "decode": decode,
+                "roofline": pre["roofline"] if pre else None, "decode": decode, "nsa": nsa,
                 "clocks": pre["clocks"] if pre else None, "cpu_baseline": cpu}
         print(json.dumps(line), flush=True)
     if ws > 1:
@@ -592,7 +673,7 @@ def main():
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--cpu-tokens", type=int, default=8192)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--only", choices=("all", "prefill", "decode"), default="all",
+    ap.add_argument("--only", choices=("all", "prefill", "decode", "nsa"), default="all",
                     help="run only one part (for profiler captures)")
     ap.add_argument("--prefill-tokens", type=int, default=PREFILL["T"],
                     help="tokens of the prefill sequence (smaller cases for profiler captures)")

@@ -207,6 +207,51 @@ CMP_API int cmp_release_workspaces(void);
 /* Static text for a status code. */
 CMP_API const char* cmp_status_string(int status);
 
+/* ---- NsaCompressWithCache (a second workload) ------------------------------
+ * "CANN ops-transformer 算子解析 NsaCompressWithCache" — 计算公式, 算法流程,
+ * 参数说明, 约束说明. For each batch b with s = act_seq_len[b] (per-batch
+ * lengths): if s >= compress_block_size and (s - compress_block_size) %
+ * compress_stride == 0, then for every head n and channel d
+ *   output_cache[slot_mapping[b], n, d] =
+ *     round(sum_{j < compress_block_size} input[token s - compress_block_size + j of b, n, d] * weight[j, n])
+ * with the products and the sum in fp32 and one round-to-nearest-even cast to
+ * the cache dtype. Other slots are not touched. */
+typedef struct {
+  int64_t B;             /* batches: entries of slot_mapping and act_seq_len */
+  int64_t N;             /* heads, 1..64 (even when above 50) */
+  int64_t D;             /* channels per head, a multiple of 16, at most 256 */
+  int64_t tokens;        /* paged: block_num (input rows / page_block_size); packed: T, the input rows */
+  int64_t table_stride;  /* paged: columns of block_table (pages per batch); packed: ignored */
+  int64_t result_len;    /* rows of output_cache */
+} cmp_nsa_dims;
+
+enum { CMP_NSA_FP16 = 0, CMP_NSA_BF16 = 1 };
+enum { CMP_NSA_PAGED = 0, CMP_NSA_PACKED = 1 };
+
+/* input: device, dtype elements, paged [block_num, page_block_size, N, D]
+ *   (a token at position p of batch b is at block block_table[b][p /
+ *   page_block_size], row p % page_block_size) or packed [T, N, D] (batch b's
+ *   tokens follow those of batches < b, in order); 16-byte aligned.
+ * weight: device [compress_block_size, N], same dtype. slot_mapping: device
+ * int32 [B], distinct values in [0, result_len). act_seq_len: device int64 [B].
+ * block_table: device int32 [B, table_stride] (paged; NULL allowed when packed).
+ * output_cache: device [result_len, N, D], same dtype, updated in place;
+ * 16-byte aligned. All memory is the caller's; the call is asynchronous on
+ * `stream` (a cudaStream_t, NULL = default stream).
+ * compress_block_size: a multiple of 16 in [16, 64], >= compress_stride;
+ * compress_stride: 16, 32, 48 or 64; page_block_size: 64 or 128 (paged).
+ * Returns CMP_OK, CMP_ERR_NULLPTR (a required pointer or dims is NULL),
+ * CMP_ERR_INVALID (a size or alignment outside the ranges above),
+ * CMP_ERR_UNSUPPORTED (dtype or layout value), CMP_ERR_CUDA (launch). B == 0
+ * is a no-op. A slot outside [0, result_len), a needed table entry outside
+ * [0, block_num) or packed rows past T set the device error word (the batch is
+ * skipped; cmp_get_error reports CMP_ERR_DEVICE_INDEX). */
+CMP_API int cmp_nsa_compress(const void* input, const void* weight, const int32_t* slot_mapping,
+                             const int64_t* act_seq_len, const int32_t* block_table, int32_t layout,
+                             int32_t dtype, int64_t compress_block_size, int64_t compress_stride,
+                             int64_t page_block_size, void* output_cache, void* stream,
+                             const cmp_nsa_dims* dims);
+
 /* ---- measurement --------------------------------------------------------
  * Kernels of the library, by id: */
 enum {
@@ -220,7 +265,8 @@ enum {
   CMP_KERNEL_DECODE_FUSED = 7, /* decode (T <= 64) in one cooperative kernel, K-split grid */
   CMP_KERNEL_DECODE_CP = 8,    /* decode (T <= 64) in one cooperative kernel of 4-CTA clusters
                                   that each own 16 channels */
-  CMP_KERNEL_COUNT = 9
+  CMP_KERNEL_NSA = 9,          /* NsaCompressWithCache */
+  CMP_KERNEL_COUNT = 10
 };
 
 /* Name of a kernel id (NULL if out of range). */

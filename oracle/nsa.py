@@ -81,7 +81,7 @@ def nsa_compress(input_bits, weight_bits, slot_mapping, act_seq_len, block_table
     uint16 [result_len, N, D] (not modified: the new cache is returned)."""
     if dtype not in ("fp16", "bf16"):
         raise ValueError("dtype is fp16 or bf16")
-    inp = to_f64(input_bits, dtype)
+    inp = np.asarray(input_bits, dtype=np.uint16)   # converted token by token below
     w = to_f64(weight_bits, dtype)
     out = np.array(output_cache_bits, dtype=np.uint16, copy=True)
     result_len, N, D = out.shape
@@ -107,7 +107,7 @@ def nsa_compress(input_bits, weight_bits, slot_mapping, act_seq_len, block_table
                 tok = inp[blk, p % page_block_size]
             else:
                 tok = inp[int(start[b]) + p]
-            acc += tok * w[j][:, None]
+            acc += to_f64(tok, dtype) * w[j][:, None]
         slot = int(slots[b])
         out[slot] = to_bits(acc, dtype)
         sums[slot] = acc

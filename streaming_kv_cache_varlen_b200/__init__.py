@@ -20,7 +20,7 @@ CMP_OK = 0
 STATUS = {0: "CMP_OK", 1: "CMP_ERR_NULLPTR", 2: "CMP_ERR_INVALID", 3: "CMP_ERR_UNSUPPORTED",
           4: "CMP_ERR_CUDA", 5: "CMP_ERR_DEVICE_INDEX", 6: "CMP_ERR_TIMEOUT"}
 KERNELS = ("sched", "proj_tcgen05", "proj_mma_sync", "proj_decode", "pool_epilogue",
-           "fused_tcgen05", "finish", "decode_fused", "decode_cp")
+           "fused_tcgen05", "finish", "decode_fused", "decode_cp", "nsa_compress")
 
 
 class CmpError(RuntimeError):
@@ -33,6 +33,12 @@ class cmp_dims(ctypes.Structure):
     _fields_ = [("B", ctypes.c_int32), ("T", ctypes.c_int32), ("H", ctypes.c_int32),
                 ("D", ctypes.c_int32), ("block_num", ctypes.c_int32),
                 ("block_size", ctypes.c_int32), ("table_stride", ctypes.c_int32)]
+
+
+class cmp_nsa_dims(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int64), ("N", ctypes.c_int64), ("D", ctypes.c_int64),
+                ("tokens", ctypes.c_int64), ("table_stride", ctypes.c_int64),
+                ("result_len", ctypes.c_int64)]
 
 
 def _load() -> ctypes.CDLL:
@@ -57,6 +63,8 @@ def _load() -> ctypes.CDLL:
         "cmp_profile_start": (ctypes.c_int, []),
         "cmp_profile_stop": (ctypes.c_int, [P, P]),
         "cmp_set_proj_kernel": (ctypes.c_int, [ctypes.c_int]),
+        "cmp_nsa_compress": (ctypes.c_int, [P, P, P, P, P, I32, I32, I64, I64, I64, P, P,
+                                            ctypes.POINTER(cmp_nsa_dims)]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -176,6 +184,60 @@ def compressor(x, kv_state, score_state, kv_block_table, state_block_table, sin,
     if st != CMP_OK:
         raise CmpError(st, "cmp_compressor")
     return out
+
+
+def nsa_compress(input, weight, slot_mapping, act_seq_len, output_cache, *, compress_block_size: int,
+                 compress_stride: int, block_table=None, page_block_size: int = 128, stream=None):
+    """NsaCompressWithCache (see cmp_nsa_compress in include/cmp.h); updates and returns
+    ``output_cache``.
+
+    input fp16 / bf16: paged [block_num, page_block_size, N, D] (with ``block_table`` int32
+    [B, pages per batch]) or packed [T, N, D]; weight [compress_block_size, N]; slot_mapping
+    int32 [B]; act_seq_len int64 [B]; output_cache [result_len, N, D]. One CUDA device."""
+    import torch
+    dev = input.device
+    if dev.type != "cuda":
+        raise ValueError("tensors must be on a CUDA device")
+    if input.dtype not in (torch.float16, torch.bfloat16):
+        raise TypeError("input must be float16 or bfloat16")
+    paged = input.dim() == 4
+    if not paged and input.dim() != 3:
+        raise ValueError("input must be [block_num, page_block_size, N, D] or [T, N, D]")
+    _check(input, "input", input.dtype, input.dim(), dev)
+    _check(weight, "weight", input.dtype, 2, dev)
+    _check(output_cache, "output_cache", input.dtype, 3, dev)
+    _check(slot_mapping, "slot_mapping", torch.int32, 1, dev)
+    _check(act_seq_len, "act_seq_len", torch.int64, 1, dev)
+    result_len, N, D = output_cache.shape
+    if tuple(input.shape[-2:]) != (N, D):
+        raise ValueError("input and output_cache must share [N, D]")
+    if tuple(weight.shape) != (compress_block_size, N):
+        raise ValueError("weight must be [compress_block_size, N]")
+    B = slot_mapping.shape[0]
+    if act_seq_len.shape[0] != B:
+        raise ValueError("act_seq_len must be [B]")
+    if paged:
+        if block_table is None:
+            raise ValueError("the paged layout needs block_table")
+        _check(block_table, "block_table", torch.int32, 2, dev)
+        if block_table.shape[0] != B or input.shape[1] != page_block_size:
+            raise ValueError("block_table must be [B, pages]; input [block_num, page_block_size, N, D]")
+        tokens, stride = input.shape[0], block_table.shape[1]
+    else:
+        tokens, stride = input.shape[0], 1
+    dims = cmp_nsa_dims(B, N, D, tokens, stride, result_len)
+    if stream is None:
+        stream = torch.cuda.current_stream(dev)
+    handle = stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+    with torch.cuda.device(dev):
+        st = lib.cmp_nsa_compress(_ptr(input), _ptr(weight), _ptr(slot_mapping), _ptr(act_seq_len),
+                                  _ptr(block_table) if paged else None, 0 if paged else 1,
+                                  1 if input.dtype == torch.bfloat16 else 0, compress_block_size,
+                                  compress_stride, page_block_size if paged else 0,
+                                  _ptr(output_cache), handle, ctypes.byref(dims))
+    if st != CMP_OK:
+        raise CmpError(st, "cmp_nsa_compress")
+    return output_cache
 
 
 def get_error(stream=None) -> int:

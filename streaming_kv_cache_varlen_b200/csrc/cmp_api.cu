@@ -22,6 +22,7 @@ cudaError_t launch_decode_fused(const Params& p, float* part, void* bar, cudaStr
 bool decode_cp_supported(const Params& p);
 size_t decode_cp_workspace(const Params& p);
 cudaError_t launch_decode_cp(const Params& p, float* ss, void* counter, cudaStream_t s);
+cudaError_t launch_nsa(const NsaParams& p, cudaStream_t s);
 }  // namespace cmp
 
 namespace {
@@ -415,6 +416,55 @@ int cmp_compressor(const cmp_bf16* x, float* kv_state, float* score_state,
 }
 
 
+int cmp_nsa_compress(const void* input, const void* weight, const int32_t* slot_mapping,
+                     const int64_t* act_seq_len, const int32_t* block_table, int32_t layout, int32_t dtype,
+                     int64_t compress_block_size, int64_t compress_stride, int64_t page_block_size,
+                     void* output_cache, void* stream, const cmp_nsa_dims* dims) {
+  if (!dims) return CMP_ERR_NULLPTR;
+  if (dtype != CMP_NSA_FP16 && dtype != CMP_NSA_BF16) return CMP_ERR_UNSUPPORTED;
+  if (layout != CMP_NSA_PAGED && layout != CMP_NSA_PACKED) return CMP_ERR_UNSUPPORTED;
+  const cmp_nsa_dims& d = *dims;
+  const int64_t cbs = compress_block_size, st = compress_stride;
+  const bool paged = layout == CMP_NSA_PAGED;
+  if (d.B < 0 || d.N < 1 || d.N > 64 || (d.N > 50 && d.N % 2) || d.D < 16 || d.D > 256 || d.D % 16 ||
+      d.result_len < 1 || d.tokens < 1 || cbs < 16 || cbs > 64 || cbs % 16 ||
+      (st != 16 && st != 32 && st != 48 && st != 64) || cbs < st ||
+      (paged && (page_block_size != 64 && page_block_size != 128)) || (paged && d.table_stride < 1) ||
+      d.B > INT32_MAX)
+    return CMP_ERR_INVALID;
+  if (d.B == 0) return CMP_OK;
+  if (!input || !weight || !slot_mapping || !act_seq_len || !output_cache || (paged && !block_table))
+    return CMP_ERR_NULLPTR;
+  if (!aligned(input, 16) || !aligned(output_cache, 16) || !aligned(weight, 2) || !aligned(slot_mapping, 4) ||
+      !aligned(act_seq_len, 8) || (paged && !aligned(block_table, 4)))
+    return CMP_ERR_INVALID;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  unsigned char* ws = nullptr;
+  const int rc = get_workspace(s, zeroed_bytes(), &ws);
+  if (rc != CMP_OK) return rc;
+  cmp::NsaParams p{};
+  p.input = static_cast<const uint16_t*>(input);
+  p.weight = static_cast<const uint16_t*>(weight);
+  p.slot = slot_mapping;
+  p.len = act_seq_len;
+  p.table = block_table;
+  p.out = static_cast<uint16_t*>(output_cache);
+  p.err = reinterpret_cast<unsigned*>(ws);
+  p.B = (int)d.B;
+  p.N = (int)d.N;
+  p.D = (int)d.D;
+  p.cbs = (int)cbs;
+  p.stride = (int)st;
+  p.pbs = paged ? (int)page_block_size : 1;
+  p.packed = paged ? 0 : 1;
+  p.bf16 = dtype == CMP_NSA_BF16 ? 1 : 0;
+  p.tokens = d.tokens;
+  p.table_stride = paged ? d.table_stride : 1;
+  p.result_len = d.result_len;
+  if (launch(CMP_KERNEL_NSA, s, [&] { return cmp::launch_nsa(p, s); }) != cudaSuccess) return CMP_ERR_CUDA;
+  return CMP_OK;
+}
+
 int cmp_get_error(void* stream) {
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (cudaStreamSynchronize(s) != cudaSuccess) return CMP_ERR_CUDA;
@@ -462,7 +512,8 @@ const char* cmp_status_string(int status) {
 const char* cmp_kernel_name(int kernel) {
   static const char* names[CMP_KERNEL_COUNT] = {"sched",         "proj_tcgen05",  "proj_mma_sync",
                                                 "proj_decode",   "pool_epilogue", "fused_tcgen05",
-                                                "finish",        "decode_fused",  "decode_cp"};
+                                                "finish",        "decode_fused",  "decode_cp",
+                                                "nsa_compress"};
   return (kernel >= 0 && kernel < CMP_KERNEL_COUNT) ? names[kernel] : nullptr;
 }
 

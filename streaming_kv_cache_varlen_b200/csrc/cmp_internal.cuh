@@ -133,6 +133,19 @@ inline cudaError_t smem_attr_once(K* kernel, size_t bytes, int (&done)[64]) {
   return e;
 }
 
+// One NsaCompressWithCache call (the second workload), device pointers.
+struct NsaParams {
+  const uint16_t* input;   // paged [tokens = block_num, pbs, N, D] or packed [tokens = T, N, D]
+  const uint16_t* weight;  // [cbs, N]
+  const int32_t* slot;     // [B]
+  const int64_t* len;      // [B] per-batch lengths
+  const int32_t* table;    // [B, table_stride] (paged)
+  uint16_t* out;           // [result_len, N, D]
+  unsigned* err;           // device error word
+  int B, N, D, cbs, stride, pbs, packed, bf16;
+  int64_t tokens, table_stride, result_len;
+};
+
 // Kernel launchers (each file defines its own).
 cudaError_t launch_sched(const Params& p, cudaStream_t s);
 cudaError_t launch_proj_mma(const Params& p, cudaStream_t s);

@@ -124,3 +124,38 @@ def test_workspace_size(cmp):
     assert 0 < small < big
     assert big >= 1025 * 512 * 4                # at least the pooled rows of one call
     assert cmp.workspace_size(1, 64, 1000, 128, 4, 16, 4, 4) == 0
+
+
+def _nsa(cmp, dims, layout=0, dtype=1, cbs=32, stride=16, pbs=128, ptr=0x10000, null=None):
+    args = [ptr] * 5 + [ptr]    # input, weight, slot_mapping, act_seq_len, block_table, output_cache
+    names = ["input", "weight", "slot_mapping", "act_seq_len", "block_table", "output_cache"]
+    if null is not None:
+        args[names.index(null)] = None
+    d = None if dims is None else ctypes.byref(dims)
+    return cmp.lib.cmp_nsa_compress(args[0], args[1], args[2], args[3], args[4], layout, dtype, cbs,
+                                    stride, pbs, args[5], None, d)
+
+
+def test_nsa_host_checks_reject_before_launch(cmp):
+    D = cmp.cmp_nsa_dims
+    ok = dict(B=4, N=24, D=192, tokens=16, table_stride=4, result_len=512)
+    assert _nsa(cmp, None) == 1
+    assert _nsa(cmp, D(**ok), dtype=2) == 3
+    assert _nsa(cmp, D(**ok), layout=2) == 3
+    for kw in [dict(cbs=8), dict(cbs=24), dict(cbs=80), dict(stride=24), dict(cbs=16, stride=32),
+               dict(pbs=32), dict(pbs=256)]:
+        assert _nsa(cmp, D(**ok), **kw) == 2, kw
+    for k, v in [("N", 0), ("N", 65), ("N", 51), ("D", 8), ("D", 24), ("D", 272), ("result_len", 0),
+                 ("tokens", 0), ("table_stride", 0), ("B", -1)]:
+        bad = dict(ok)
+        bad[k] = v
+        assert _nsa(cmp, D(**bad)) == 2, (k, v)
+    for name in ["input", "weight", "slot_mapping", "act_seq_len", "block_table", "output_cache"]:
+        assert _nsa(cmp, D(**ok), null=name) == 1, name
+    assert _nsa(cmp, D(**ok), ptr=0x10004) == 2          # input / output not 16-byte aligned
+    # packed layout: no block table needed (still rejected here by the misaligned pointer)
+    assert _nsa(cmp, D(**ok), layout=1, null="block_table", ptr=0x10004) == 2
+    # B == 0: a no-op, no pointer touched
+    z = dict(ok, B=0)
+    assert cmp.lib.cmp_nsa_compress(None, None, None, None, None, 0, 1, 32, 16, 128, None, None,
+                                    ctypes.byref(D(**z))) == 0

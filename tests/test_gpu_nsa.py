@@ -1,0 +1,125 @@
+"""NsaCompressWithCache on a B200 against its oracle (oracle/nsa.py): both
+layouts, both dtypes, the stride / window sizes of the page's constraints, the
+page's example, untouched slots, error reporting."""
+
+import json
+import os
+
+import numpy as np
+import pytest
+
+from oracle.nsa import nsa_compress, to_f64
+from workloads import make_nsa_inputs
+
+pytestmark = pytest.mark.gpu
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def to_dev(i):
+    import torch
+    dt = torch.float16 if i.dtype == "fp16" else torch.bfloat16
+    b16 = lambda a: torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).cuda().view(dt)
+    return dict(input=b16(i.input), weight=b16(i.weight),
+                slot_mapping=torch.from_numpy(i.slot_mapping).cuda(),
+                act_seq_len=torch.from_numpy(i.act_seq_len).cuda(),
+                output_cache=b16(i.output_cache),
+                block_table=torch.from_numpy(i.block_table).cuda() if i.layout == "paged" else None)
+
+
+def gpu_call(cmp, i):
+    import torch
+    a = to_dev(i)
+    cmp.nsa_compress(a["input"], a["weight"], a["slot_mapping"], a["act_seq_len"], a["output_cache"],
+                     compress_block_size=i.compress_block_size, compress_stride=i.compress_stride,
+                     block_table=a["block_table"], page_block_size=i.page_block_size)
+    err = cmp.get_error()
+    return a["output_cache"].view(torch.int16).cpu().numpy().view(np.uint16), err
+
+
+def check(cmp, i):
+    ref = nsa_compress(i.input, i.weight, i.slot_mapping, i.act_seq_len, i.block_table, i.output_cache,
+                       dtype=i.dtype, compress_block_size=i.compress_block_size,
+                       compress_stride=i.compress_stride, page_block_size=i.page_block_size,
+                       layout=i.layout)
+    got, err = gpu_call(cmp, i)
+    assert err == 0
+    w = ref.written
+    # slots not written: bit for bit the cache before the call
+    assert np.array_equal(got[~w], i.output_cache[~w])
+    # written slots: the exact sum rounded once, within one unit of the dtype
+    # (the library sums in fp32, so a sum next to a rounding boundary may round
+    # to the other neighbour)
+    g = to_f64(got[w], i.dtype)
+    e = to_f64(ref.output_cache[w], i.dtype)
+    mant = 10 if i.dtype == "fp16" else 7
+    mag = np.maximum(np.abs(e), np.abs(g))
+    ulp = np.exp2(np.floor(np.log2(np.maximum(mag, 1e-30))) - mant)
+    assert (np.abs(g - e) <= ulp + 1e-5).all()
+    return ref, got
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "fp16"])
+@pytest.mark.parametrize("layout", ["paged", "TND"])
+@pytest.mark.parametrize("cbs,stride,pbs", [(32, 16, 128), (16, 16, 64), (64, 64, 128), (48, 32, 64),
+                                            (64, 16, 64)])
+def test_matches_oracle(lib, dtype, layout, cbs, stride, pbs):
+    i = make_nsa_inputs(name="nsa", seed=cbs * 7 + stride, B=24, N=24, D=192, compress_block_size=cbs,
+                        compress_stride=stride, page_block_size=pbs, dtype=dtype, layout=layout,
+                        max_seq_len=512, trigger_fraction=0.6)
+    ref, _ = check(lib, i)
+    assert ref.written.sum() >= 5
+
+
+@pytest.mark.parametrize("N,D", [(1, 16), (64, 256), (52, 48), (7, 128)])
+def test_head_shapes(lib, N, D):
+    i = make_nsa_inputs(name="shape", seed=N + D, B=9, N=N, D=D, compress_block_size=32,
+                        compress_stride=32, page_block_size=64, max_seq_len=256, trigger_fraction=0.7)
+    check(lib, i)
+
+
+def test_pages_example(lib):
+    c = json.load(open(os.path.join(GOLDEN, "nsa_example_case.json")))
+    import torch
+    B, N, D, pbs = c["batch_size"], c["heads_num"], c["heads_dim"], c["page_block_size"]
+    per = c["max_seq_len"] // pbs
+    h = dict(dtype=torch.float16, device="cuda")
+    out = torch.ones((c["result_len"], N, D), **h)
+    lib.nsa_compress(torch.ones((per * B, pbs, N, D), **h), torch.ones((c["compress_block_size"], N), **h),
+                     torch.tensor(c["slot_mapping"], dtype=torch.int32, device="cuda"),
+                     torch.tensor(c["act_seq_len"], dtype=torch.int64, device="cuda"), out,
+                     compress_block_size=c["compress_block_size"], compress_stride=c["compress_stride"],
+                     block_table=torch.zeros((B, per), dtype=torch.int32, device="cuda"), page_block_size=pbs)
+    assert lib.get_error() == 0
+    flat = out.reshape(-1).float().cpu().numpy()
+    i0 = c["printed_first_index"]
+    assert flat[i0:i0 + len(c["expected_printed_values"])].tolist() == c["expected_printed_values"]
+    assert (flat[:N * D] == 32.0).all() and (flat[N * D:] == 1.0).all()
+
+
+def test_repeat_is_bit_identical(lib):
+    i = make_nsa_inputs(name="rep", seed=3, B=40, N=8, D=64, compress_block_size=64, compress_stride=16,
+                        page_block_size=128, max_seq_len=512, trigger_fraction=1.0)
+    a, _ = gpu_call(lib, i)
+    b, _ = gpu_call(lib, i)
+    assert np.array_equal(a, b)
+
+
+def test_bad_table_entry_and_slot_are_reported(lib):
+    import dataclasses
+    i = make_nsa_inputs(name="bad", seed=4, B=3, N=4, D=32, compress_block_size=32, compress_stride=16,
+                        page_block_size=64, lengths=[48, 32, 64], max_seq_len=128)
+    tbl = i.block_table.copy()
+    tbl[0, 0] = i.input.shape[0] + 3           # batch 0 reads page 0 (positions 16..47)
+    slots = i.slot_mapping.copy()
+    slots[2] = 10_000                          # batch 2's slot is past the cache
+    bad = dataclasses.replace(i, block_table=tbl, slot_mapping=slots)
+    got, err = gpu_call(lib, bad)
+    assert err == 5                            # CMP_ERR_DEVICE_INDEX
+    assert lib.get_error() == 0                # cleared by the read
+    # batch 1 is still written; batches 0 and 2 are skipped
+    ref = nsa_compress(i.input, i.weight, i.slot_mapping, i.act_seq_len, i.block_table, i.output_cache,
+                       dtype=i.dtype, compress_block_size=32, compress_stride=16, page_block_size=64)
+    s0, s1 = i.slot_mapping[0], i.slot_mapping[1]
+    assert np.array_equal(got[s0], i.output_cache[s0])
+    assert np.abs(to_f64(got[s1], i.dtype) - to_f64(ref.output_cache[s1], i.dtype)).max() < 0.05
