@@ -411,6 +411,7 @@ def bench_decode(args, ws, local, stream, peaks, peak_src):
     dout = torch.empty((cmp.out_rows(dec_inp.B, dec_inp.T, dec_inp.ratio), dec_inp.D),
                        dtype=torch.bfloat16, device=device)
     side = torch.cuda.Stream(device)
+    side.wait_stream(torch.cuda.current_stream(device))  # the inputs were made on the current stream
     with torch.cuda.stream(side):
         for _ in range(max(3, args.warmup)):
             cmp.compressor(**dec, out=dout)
@@ -515,6 +516,7 @@ def bench_nsa(args, ws, local, peaks, peak_src):
                          compress_stride=c["stride"], block_table=table, page_block_size=c["page"])
 
     side = torch.cuda.Stream(device)
+    side.wait_stream(torch.cuda.current_stream(device))  # the inputs were made on the current stream
     with torch.cuda.stream(side):
         for _ in range(max(3, args.warmup)):
             call()

@@ -217,10 +217,11 @@ CMP_API const char* cmp_status_string(int status);
  * with the products and the sum in fp32 and one round-to-nearest-even cast to
  * the cache dtype. Other slots are not touched. */
 typedef struct {
-  int64_t B;             /* batches: entries of slot_mapping and act_seq_len */
+  int64_t B;             /* batches: entries of slot_mapping and act_seq_len, at most 65535 */
   int64_t N;             /* heads, 1..64 (even when above 50) */
   int64_t D;             /* channels per head, a multiple of 16, at most 256 */
-  int64_t tokens;        /* paged: block_num (input rows / page_block_size); packed: T, the input rows */
+  int64_t tokens;        /* paged: block_num (input rows / page_block_size); packed: T, the input rows;
+                            input rows at most INT32_MAX */
   int64_t table_stride;  /* paged: columns of block_table (pages per batch); packed: ignored */
   int64_t result_len;    /* rows of output_cache */
 } cmp_nsa_dims;
@@ -242,7 +243,8 @@ enum { CMP_NSA_PAGED = 0, CMP_NSA_PACKED = 1 };
  * compress_stride: 16, 32, 48 or 64; page_block_size: 64 or 128 (paged).
  * Returns CMP_OK, CMP_ERR_NULLPTR (a required pointer or dims is NULL),
  * CMP_ERR_INVALID (a size or alignment outside the ranges above),
- * CMP_ERR_UNSUPPORTED (dtype or layout value), CMP_ERR_CUDA (launch). B == 0
+ * CMP_ERR_UNSUPPORTED (dtype or layout value), CMP_ERR_CUDA (launch, or the driver
+ * cannot describe the cache as a TMA tensor). B == 0
  * is a no-op. A slot outside [0, result_len), a needed table entry outside
  * [0, block_num) or packed rows past T set the device error word (the batch is
  * skipped; cmp_get_error reports CMP_ERR_DEVICE_INDEX). */

@@ -430,7 +430,7 @@ int cmp_nsa_compress(const void* input, const void* weight, const int32_t* slot_
       d.result_len < 1 || d.tokens < 1 || cbs < 16 || cbs > 64 || cbs % 16 ||
       (st != 16 && st != 32 && st != 48 && st != 64) || cbs < st ||
       (paged && (page_block_size != 64 && page_block_size != 128)) || (paged && d.table_stride < 1) ||
-      d.B > INT32_MAX)
+      d.B > 65535 || d.tokens > (paged ? INT32_MAX / page_block_size : INT32_MAX))
     return CMP_ERR_INVALID;
   if (d.B == 0) return CMP_OK;
   if (!input || !weight || !slot_mapping || !act_seq_len || !output_cache || (paged && !block_table))

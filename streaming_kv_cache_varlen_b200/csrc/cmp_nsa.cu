@@ -7,12 +7,15 @@
 // values cast to fp32, multiplied by weight[j, n], summed, cast back to
 // fp16 / bf16 with round-to-nearest-even).
 //
-// HBM bound: every byte of the window's tokens is read once. Grid = (batch,
-// chunk of the N*D plane); a thread owns 8 consecutive elements (16 bytes, one
-// head since D is a multiple of 16) and streams the window's tokens with 8
-// 16-byte loads in flight, so a warp reads 512 contiguous bytes of one token
-// per instruction. The sum runs over the tokens in order (deterministic).
+// HBM bound: every byte of the window's tokens is read once. One CTA per (group
+// of nh heads, batch). The window starts at a multiple of 16 tokens and pages
+// hold a multiple of 16, so it is cbs / 16 runs of 16 consecutive cache rows,
+// each inside one page: each run is ONE TMA box {D, nh heads, 16 rows} of a 3-D
+// map over the cache [rows, N, D], a few large copies per CTA instead of one
+// per token and chunk (per-copy overhead in the copy engine, not DRAM, limited
+// the version with small copies).
 #include "cmp_internal.cuh"
+#include "cmp_sm100.cuh"
 
 #include <cuda_fp16.h>
 
@@ -21,97 +24,151 @@ namespace cmp {
 namespace {
 
 constexpr int kThreads = 128;
-constexpr int kElems = 8;  // per thread
+constexpr int kRun = 16;                 // cache rows per TMA box
+constexpr int kTargetBytes = 32 << 10;   // window bytes per CTA the head group aims at
 
-__device__ __forceinline__ float to_f32(uint16_t v, bool bf16) {
-  return bf16 ? __bfloat162float(__ushort_as_bfloat16(v)) : __half2float(__ushort_as_half(v));
+template <bool BF16>
+__device__ __forceinline__ float to_f32(uint16_t v) {
+  return BF16 ? __uint_as_float((uint32_t)v << 16) : __half2float(__ushort_as_half(v));
 }
 
-__device__ __forceinline__ uint16_t from_f32(float v, bool bf16) {
-  return bf16 ? __bfloat16_as_ushort(__float2bfloat16_rn(v)) : __half_as_ushort(__float2half_rn(v));
+template <bool BF16>
+__device__ __forceinline__ uint32_t pack(float lo, float hi) {
+  if (BF16) {
+    const __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<const uint32_t*>(&h);
+  }
+  const __half2 h = __floats2half2_rn(lo, hi);
+  return *reinterpret_cast<const uint32_t*>(&h);
 }
 
-__global__ void __launch_bounds__(kThreads) nsa_kernel(NsaParams p) {
-  const int b = blockIdx.x;
-  const int64_t s = p.len[b];
-  if (s < p.cbs || (s - p.cbs) % p.stride != 0) return;  // not a compression step
+// Thread 0 validates the batch's slot and the cache rows of its window, then
+// issues the window's cbs / 16 boxes (heads h0 .. h0 + nh - 1; heads past N read
+// as zeros and are not stored), all completing on one mbarrier; the other
+// threads stage the weights meanwhile. Then each thread sums 4 consecutive
+// elements of one head over the window's tokens in order and stores them.
+template <bool BF16>
+__global__ void __launch_bounds__(kThreads)
+    nsa_kernel(const __grid_constant__ CUtensorMap map, NsaParams p, int nh, int page_shift) {
+  const int b = blockIdx.y;
+  const int h0 = blockIdx.x * nh;
+  const int64_t s = __ldg(p.len + b);
+  if (s < p.cbs || (s - p.cbs) % p.stride != 0) return;  // not a compression step (whole CTA)
+  extern __shared__ __align__(128) unsigned char smem_raw[];
+  // TMA destinations start on 128-byte boundaries (the runs are multiples of 512 B)
+  uint16_t* buf = reinterpret_cast<uint16_t*>(smem_raw + ((128u - (sm100::smem_u32(smem_raw) & 127u)) & 127u));
+  const int per_tok = nh * p.D;
+  float* wsm = reinterpret_cast<float*>(buf + (size_t)p.cbs * per_tok);  // [cbs][nh]
+  __shared__ __align__(8) uint64_t full;
   __shared__ int ok;
-  __shared__ int64_t row0;  // packed: the batch's first row
   if (threadIdx.x == 0) {
-    const int slot = p.slot[b];
+    sm100::prefetch_tmap(&map);
+    const int slot = __ldg(p.slot + b);
     bool good = slot >= 0 && slot < p.result_len;
-    int64_t start = 0;
+    const int64_t first = s - p.cbs;
+    const int runs = p.cbs / kRun;
+    int64_t row[64 / kRun];
     if (p.packed) {
+      int64_t start = 0;
       for (int i = 0; i < b; ++i) {
-        const int64_t li = p.len[i];
+        const int64_t li = __ldg(p.len + i);
         good = good && li >= 0;
         start += li > 0 ? li : 0;
       }
       good = good && start + s <= p.tokens;
+      for (int k = 0; k < runs; ++k) row[k] = start + first + k * kRun;
     } else {
-      // the window spans at most two pages (cbs <= page size)
-      const int64_t first = s - p.cbs, last = s - 1;
-      for (int64_t pg = first / p.pbs; pg <= last / p.pbs; ++pg) {
-        const int32_t blk = pg < p.table_stride ? p.table[(int64_t)b * p.table_stride + pg] : -1;
+      const int32_t* trow = p.table + (int64_t)b * p.table_stride;
+      const int64_t mask = (int64_t(1) << page_shift) - 1;
+      for (int k = 0; k < runs; ++k) {
+        const int64_t pos = first + k * kRun;
+        const int64_t pg = pos >> page_shift;
+        const int32_t blk = pg < p.table_stride ? __ldg(trow + pg) : -1;
         good = good && blk >= 0 && blk < p.tokens;
+        row[k] = ((int64_t)blk << page_shift) + (pos & mask);
       }
     }
     if (!good) atomicOr(p.err, kErrIndex);
     ok = good ? 1 : 0;
-    row0 = start;
+    if (good) {
+      sm100::mbar_init(&full, 1);
+      sm100::fence_barrier_init();
+      sm100::mbar_arrive_expect_tx(&full, (uint32_t)(p.cbs * per_tok * 2));
+      for (int k = 0; k < runs; ++k)
+        sm100::tma_load_3d(buf + (size_t)k * kRun * per_tok, &map, &full, 0, h0, (int)row[k]);
+    }
+  }
+  for (int i = threadIdx.x; i < p.cbs * nh; i += kThreads) {
+    const int j = i / nh, h = h0 + i % nh;
+    wsm[i] = h < p.N ? to_f32<BF16>(__ldg(p.weight + j * p.N + h)) : 0.f;
   }
   __syncthreads();
   if (!ok) return;
-
-  const int64_t plane = (int64_t)p.N * p.D;
-  const int64_t e0 = ((int64_t)blockIdx.y * kThreads + threadIdx.x) * kElems;
-  if (e0 >= plane) return;
-  const int n = (int)(e0 / p.D);
-  const bool bf = p.bf16 != 0;
-  const int64_t first = s - p.cbs;
-  float acc[kElems];
-#pragma unroll
-  for (int k = 0; k < kElems; ++k) acc[k] = 0.f;
-  for (int j0 = 0; j0 < p.cbs; j0 += 8) {  // cbs is a multiple of 16
-    uint4 v[8];
-    float w[8];
-#pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      const int64_t pos = first + j0 + u;
-      int64_t row;
-      if (p.packed) {
-        row = row0 + pos;
-      } else {
-        const int32_t blk = p.table[(int64_t)b * p.table_stride + pos / p.pbs];
-        row = (int64_t)blk * p.pbs + pos % p.pbs;
-      }
-      v[u] = __ldg(reinterpret_cast<const uint4*>(p.input + row * plane + e0));
-      w[u] = to_f32(__ldg(p.weight + (int64_t)(j0 + u) * p.N + n), bf);
-    }
-#pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      const uint32_t q[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
-#pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        acc[2 * k] = fmaf(to_f32((uint16_t)(q[k] & 0xFFFFu), bf), w[u], acc[2 * k]);
-        acc[2 * k + 1] = fmaf(to_f32((uint16_t)(q[k] >> 16), bf), w[u], acc[2 * k + 1]);
-      }
-    }
+  int never = 0;
+  if (!sm100::mbar_wait(&full, 0, &never)) {
+    if (threadIdx.x == 0) atomicOr(p.err, kErrTimeout);
+    return;
   }
-  uint32_t o[4];
-#pragma unroll
-  for (int k = 0; k < 4; ++k)
-    o[k] = (uint32_t)from_f32(acc[2 * k], bf) | ((uint32_t)from_f32(acc[2 * k + 1], bf) << 16);
-  *reinterpret_cast<uint4*>(p.out + (int64_t)p.slot[b] * plane + e0) = make_uint4(o[0], o[1], o[2], o[3]);
+  const int live = (p.N - h0 < nh ? p.N - h0 : nh) * p.D;  // elements of heads < N
+  uint16_t* dst = p.out + (int64_t)__ldg(p.slot + b) * p.N * p.D + (int64_t)h0 * p.D;
+  for (int e = threadIdx.x * 4; e < live; e += kThreads * 4) {
+    const int hh = e / p.D;
+    float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+    for (int j = 0; j < p.cbs; ++j) {
+      const uint2 v = *reinterpret_cast<const uint2*>(buf + (size_t)j * per_tok + e);
+      const float w = wsm[j * nh + hh];
+      a0 = fmaf(to_f32<BF16>((uint16_t)(v.x & 0xFFFFu)), w, a0);
+      a1 = fmaf(to_f32<BF16>((uint16_t)(v.x >> 16)), w, a1);
+      a2 = fmaf(to_f32<BF16>((uint16_t)(v.y & 0xFFFFu)), w, a2);
+      a3 = fmaf(to_f32<BF16>((uint16_t)(v.y >> 16)), w, a3);
+    }
+    uint2 o;
+    o.x = pack<BF16>(a0, a1);
+    o.y = pack<BF16>(a2, a3);
+    *reinterpret_cast<uint2*>(dst + e) = o;
+  }
 }
+
+// The cache as a 3-D tensor (d, head, row) with a box of {D, nh, 16}.
+bool make_cache_map(CUtensorMap* m, const NsaParams& p, int64_t rows, int nh) {
+  sm100::EncodeTiledFn f = sm100::encode_fn();
+  if (!f) return false;
+  const cuuint64_t dims[3] = {(cuuint64_t)p.D, (cuuint64_t)p.N, (cuuint64_t)rows};
+  const cuuint64_t strides[2] = {(cuuint64_t)p.D * 2, (cuuint64_t)p.N * p.D * 2};
+  const cuuint32_t box[3] = {(cuuint32_t)p.D, (cuuint32_t)nh, (cuuint32_t)kRun};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return f(m, p.bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3,
+           const_cast<uint16_t*>(p.input), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+           CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+int g_nsa_conf[2][64] = {{0}, {0}};
 
 }  // namespace
 
 cudaError_t launch_nsa(const NsaParams& p, cudaStream_t s) {
-  const int64_t plane = (int64_t)p.N * p.D;
-  const unsigned chunks = (unsigned)((plane / kElems + kThreads - 1) / kThreads);
-  nsa_kernel<<<dim3((unsigned)p.B, chunks), kThreads, 0, s>>>(p);
-  return cudaGetLastError();
+  const int head_bytes = p.cbs * p.D * 2;  // one head of the window
+  int nh = kTargetBytes / head_bytes;
+  nh = nh < 1 ? 1 : (nh > p.N ? p.N : nh);
+  CUtensorMap map;
+  if (!make_cache_map(&map, p, p.packed ? p.tokens : p.tokens * p.pbs, nh)) return cudaErrorNotSupported;
+  const int page_shift = p.packed ? 0 : (p.pbs == 64 ? 6 : 7);
+  const size_t smem = 128 + (size_t)p.cbs * nh * p.D * 2 + (size_t)p.cbs * nh * 4;  // + alignment slack
+  // the attribute is raised once per device, to the largest size a call can
+  // ask for (window bytes <= kTargetBytes unless one head is larger: cbs <= 64,
+  // D <= 256 gives 32 KB)
+  constexpr size_t kMaxSmem = (size_t)kTargetBytes + kTargetBytes / 2 + 64 * 64 * 4;
+  const dim3 grid((unsigned)((p.N + nh - 1) / nh), (unsigned)p.B);
+  cudaError_t e;
+  if (p.bf16) {
+    e = smem_attr_once(nsa_kernel<true>, kMaxSmem, g_nsa_conf[1]);
+    if (e == cudaSuccess) nsa_kernel<true><<<grid, kThreads, smem, s>>>(map, p, nh, page_shift);
+  } else {
+    e = smem_attr_once(nsa_kernel<false>, kMaxSmem, g_nsa_conf[0]);
+    if (e == cudaSuccess) nsa_kernel<false><<<grid, kThreads, smem, s>>>(map, p, nh, page_shift);
+  }
+  return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 }  // namespace cmp

@@ -146,13 +146,16 @@ def test_nsa_host_checks_reject_before_launch(cmp):
                dict(pbs=32), dict(pbs=256)]:
         assert _nsa(cmp, D(**ok), **kw) == 2, kw
     for k, v in [("N", 0), ("N", 65), ("N", 51), ("D", 8), ("D", 24), ("D", 272), ("result_len", 0),
-                 ("tokens", 0), ("table_stride", 0), ("B", -1)]:
+                 ("tokens", 0), ("table_stride", 0), ("B", -1), ("B", 65536),
+                 ("tokens", (2**31 - 1) // 128 + 1)]:  # paged rows (tokens x 128) past INT32_MAX
         bad = dict(ok)
         bad[k] = v
         assert _nsa(cmp, D(**bad)) == 2, (k, v)
     for name in ["input", "weight", "slot_mapping", "act_seq_len", "block_table", "output_cache"]:
         assert _nsa(cmp, D(**ok), null=name) == 1, name
     assert _nsa(cmp, D(**ok), ptr=0x10004) == 2          # input / output not 16-byte aligned
+    packed_rows = dict(ok, tokens=2**31)                  # packed rows past INT32_MAX
+    assert _nsa(cmp, D(**packed_rows), layout=1) == 2
     # packed layout: no block table needed (still rejected here by the misaligned pointer)
     assert _nsa(cmp, D(**ok), layout=1, null="block_table", ptr=0x10004) == 2
     # B == 0: a no-op, no pointer touched

@@ -123,3 +123,23 @@ def test_bad_table_entry_and_slot_are_reported(lib):
     s0, s1 = i.slot_mapping[0], i.slot_mapping[1]
     assert np.array_equal(got[s0], i.output_cache[s0])
     assert np.abs(to_f64(got[s1], i.dtype) - to_f64(ref.output_cache[s1], i.dtype)).max() < 0.05
+
+
+def test_bench_launch_shape(lib):
+    """The benchmark's launch: 128 batches, N=24, D=192, bf16, paged (page 128),
+    window 32, stride 16, every batch on a compression step (one page per
+    batch here to keep the host pool small; the grid and boxes are the same)."""
+    i = make_nsa_inputs(name="bench", seed=11, B=128, N=24, D=192, compress_block_size=32, compress_stride=16,
+                        page_block_size=128, dtype="bf16", layout="paged", max_seq_len=128,
+                        trigger_fraction=1.0)
+    ref, _ = check(lib, i)
+    assert ref.written.sum() == 128
+
+
+@pytest.mark.parametrize("layout", ["paged", "TND"])
+def test_many_batches(lib, layout):
+    """1000 batches: several waves of CTAs on the 148 SMs."""
+    i = make_nsa_inputs(name="many", seed=12, B=1000, N=8, D=64, compress_block_size=64, compress_stride=16,
+                        page_block_size=64, dtype="fp16", layout=layout, max_seq_len=128, trigger_fraction=0.8)
+    ref, _ = check(lib, i)
+    assert ref.written.sum() >= 700
