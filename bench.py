@@ -557,7 +557,7 @@ def bench_nsa(args, ws, local, peaks, peak_src):
             "us_per_call": us, "timing": "CUDA-graph replay of 50 x (L2 flush + call) minus 50 flushes, / 50",
             "roofline": {"bound": "hbm", "achieved": ach, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                          "frac": ach / peaks["hbm_gbs"], "algorithmic_bytes_per_call": nbytes,
-                         "peak_source": peak_src}}
+                         "traffic": traffic_for("cmp_nsa.cu", "nsa_compress"), "peak_source": peak_src}}
 
 
 def run_ours(args):
