@@ -585,7 +585,7 @@ def run_ours(args):
         torch.cuda.empty_cache()
     cpu = None
     if rank == 0 and ws == 1 and args.only == "all" and not args.no_cpu_baseline:
-        cpu = cpu_baseline(args.cpu_tokens)
+        cpu = cpu_baseline(args.cpu_tokens or cpu_sample_tokens(args.cpu_seconds))
 
     if rank == 0:
         line = {"metric": METRIC, "value": pre["value"] if pre else None, "unit": "tokens/s",
@@ -632,6 +632,15 @@ def cpu_baseline(tokens: int):
                       f"prefill workload, float64 numpy oracle, {dt:.2f} s"}
 
 
+def cpu_sample_tokens(seconds: float) -> int:
+    """Tokens of the prefill workload the oracle processes in about ``seconds`` on
+    this host (a 2048-token probe sets the rate), whole windows, at most the
+    workload."""
+    rate = cpu_baseline(2048)["value"]
+    r = PREFILL["ratio"]
+    return int(max(4096, min(PREFILL["T"], rate * seconds)) // r * r)
+
+
 def run_reference(args):
     """The CPU oracle as the reference arm: each step is the oracle on a bounded
     sample of the prefill workload, sized so warm-up plus all steps take about
@@ -673,7 +682,9 @@ def main():
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
-    ap.add_argument("--cpu-tokens", type=int, default=8192)
+    ap.add_argument("--cpu-tokens", type=int, default=None,
+                    help="tokens of the CPU-baseline sample (default: about --cpu-seconds of oracle work)")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--only", choices=("all", "prefill", "decode", "nsa"), default="all",
                     help="run only one part (for profiler captures)")
