@@ -268,7 +268,8 @@ enum {
   CMP_KERNEL_DECODE_CP = 8,    /* decode (T <= 64) in one cooperative kernel of 4-CTA clusters
                                   that each own 16 channels */
   CMP_KERNEL_NSA = 9,          /* NsaCompressWithCache */
-  CMP_KERNEL_COUNT = 10
+  CMP_KERNEL_NSA_SCAN = 10,    /* NsaCompressWithCache, packed layout: each batch's first row */
+  CMP_KERNEL_COUNT = 11
 };
 
 /* Name of a kernel id (NULL if out of range). */

@@ -20,7 +20,7 @@ CMP_OK = 0
 STATUS = {0: "CMP_OK", 1: "CMP_ERR_NULLPTR", 2: "CMP_ERR_INVALID", 3: "CMP_ERR_UNSUPPORTED",
           4: "CMP_ERR_CUDA", 5: "CMP_ERR_DEVICE_INDEX", 6: "CMP_ERR_TIMEOUT"}
 KERNELS = ("sched", "proj_tcgen05", "proj_mma_sync", "proj_decode", "pool_epilogue",
-           "fused_tcgen05", "finish", "decode_fused", "decode_cp", "nsa_compress")
+           "fused_tcgen05", "finish", "decode_fused", "decode_cp", "nsa_compress", "nsa_scan")
 
 
 class CmpError(RuntimeError):

@@ -23,6 +23,7 @@ bool decode_cp_supported(const Params& p);
 size_t decode_cp_workspace(const Params& p);
 cudaError_t launch_decode_cp(const Params& p, float* ss, void* counter, cudaStream_t s);
 cudaError_t launch_nsa(const NsaParams& p, cudaStream_t s);
+cudaError_t launch_nsa_scan(const NsaParams& p, cudaStream_t s);
 }  // namespace cmp
 
 namespace {
@@ -440,9 +441,11 @@ int cmp_nsa_compress(const void* input, const void* weight, const int32_t* slot_
     return CMP_ERR_INVALID;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   unsigned char* ws = nullptr;
-  const int rc = get_workspace(s, zeroed_bytes(), &ws);
+  // packed: the batches' first rows follow the zeroed header
+  const int rc = get_workspace(s, zeroed_bytes() + (paged ? 0 : (size_t)d.B * 8), &ws);
   if (rc != CMP_OK) return rc;
   cmp::NsaParams p{};
+  p.starts = paged ? nullptr : reinterpret_cast<int64_t*>(ws + zeroed_bytes());
   p.input = static_cast<const uint16_t*>(input);
   p.weight = static_cast<const uint16_t*>(weight);
   p.slot = slot_mapping;
@@ -461,6 +464,8 @@ int cmp_nsa_compress(const void* input, const void* weight, const int32_t* slot_
   p.tokens = d.tokens;
   p.table_stride = paged ? d.table_stride : 1;
   p.result_len = d.result_len;
+  if (!paged && launch(CMP_KERNEL_NSA_SCAN, s, [&] { return cmp::launch_nsa_scan(p, s); }) != cudaSuccess)
+    return CMP_ERR_CUDA;
   if (launch(CMP_KERNEL_NSA, s, [&] { return cmp::launch_nsa(p, s); }) != cudaSuccess) return CMP_ERR_CUDA;
   return CMP_OK;
 }
@@ -513,7 +518,7 @@ const char* cmp_kernel_name(int kernel) {
   static const char* names[CMP_KERNEL_COUNT] = {"sched",         "proj_tcgen05",  "proj_mma_sync",
                                                 "proj_decode",   "pool_epilogue", "fused_tcgen05",
                                                 "finish",        "decode_fused",  "decode_cp",
-                                                "nsa_compress"};
+                                                "nsa_compress",  "nsa_scan"};
   return (kernel >= 0 && kernel < CMP_KERNEL_COUNT) ? names[kernel] : nullptr;
 }
 

@@ -504,18 +504,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (threadIdx.x == 0 && sm.abort) atomicOr(p.err, kErrTimeout);
 }
 
-bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows) {
-  EncodeTiledFn f = encode_fn();
-  if (!f) return false;
-  const cuuint64_t dims[2] = {cols, rows};
-  const cuuint64_t strides[1] = {cols * 2};
-  const cuuint32_t box[2] = {(cuuint32_t)BK, box_rows};
-  const cuuint32_t estr[2] = {1, 1};
-  return f(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
-           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 // CTAs of one variant that can be resident at once on the current device (cached).
 template <int MAXT>
 int max_resident() {
@@ -574,8 +562,8 @@ size_t decode_fused_workspace(const Params& p) {
 cudaError_t launch_decode_fused(const Params& p, float* part, void* bar, cudaStream_t s) {
   const int NT = (p.T + 15) / 16 * 16;
   CUtensorMap mx, mkv, mg;
-  if (!make_map(&mx, p.x, p.T, p.H, (uint32_t)NT) || !make_map(&mkv, p.wkv, p.C, p.H, BM) ||
-      !make_map(&mg, p.wgate, p.C, p.H, BM))
+  if (!make_tile_map(&mx, p.x, p.T, p.H, (uint32_t)NT) || !make_tile_map(&mkv, p.wkv, p.C, p.H, BM) ||
+      !make_tile_map(&mg, p.wgate, p.C, p.H, BM))
     return cudaErrorInvalidValue;
   DecodeArgs a;
   a.part = part;

@@ -141,6 +141,7 @@ struct NsaParams {
   const int64_t* len;      // [B] per-batch lengths
   const int32_t* table;    // [B, table_stride] (paged)
   uint16_t* out;           // [result_len, N, D]
+  int64_t* starts;         // [B] packed: first row of each batch (-1: a negative length before it)
   unsigned* err;           // device error word
   int B, N, D, cbs, stride, pbs, packed, bf16;
   int64_t tokens, table_stride, result_len;

@@ -69,13 +69,9 @@ __global__ void __launch_bounds__(kThreads)
     const int runs = p.cbs / kRun;
     int64_t row[64 / kRun];
     if (p.packed) {
-      int64_t start = 0;
-      for (int i = 0; i < b; ++i) {
-        const int64_t li = __ldg(p.len + i);
-        good = good && li >= 0;
-        start += li > 0 ? li : 0;
-      }
-      good = good && start + s <= p.tokens;
+      pdl_wait();  // the row starts come from nsa_scan_kernel, launched just before
+      const int64_t start = p.starts[b];
+      good = good && start >= 0 && start + s <= p.tokens;
       for (int k = 0; k < runs; ++k) row[k] = start + first + k * kRun;
     } else {
       const int32_t* trow = p.table + (int64_t)b * p.table_stride;
@@ -129,6 +125,74 @@ __global__ void __launch_bounds__(kThreads)
   }
 }
 
+// Packed layout: the first row of every batch, starts[b] = sum of the lengths of
+// batches before b (-1 if one of them is negative), by one CTA: each thread sums
+// a contiguous chunk of up to 64 lengths, the chunk totals are scanned across
+// the block, and each thread then writes its chunk's starts.
+constexpr int kScanThreads = 1024;
+
+__global__ void __launch_bounds__(kScanThreads) nsa_scan_kernel(const int64_t* len, int B, int64_t* starts) {
+  pdl_trigger();  // the main kernel may be scheduled now; it waits for this grid to finish
+  __shared__ int64_t w_sum[kScanThreads / 32];
+  __shared__ int w_neg[kScanThreads / 32];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int per = (B + kScanThreads - 1) / kScanThreads;
+  const int i0 = threadIdx.x * per, i1 = i0 + per < B ? i0 + per : B;
+  int64_t sum = 0;
+  int neg = 0;
+  for (int i = i0; i < i1; ++i) {
+    const int64_t li = __ldg(len + i);
+    sum += li > 0 ? li : 0;
+    neg |= li < 0;
+  }
+  int64_t inc = sum;  // inclusive scan over the warp
+  int ineg = neg;
+  for (int o = 1; o < 32; o <<= 1) {
+    const int64_t t = __shfl_up_sync(0xffffffffu, inc, o);
+    const int n = __shfl_up_sync(0xffffffffu, ineg, o);
+    if (lane >= o) {
+      inc += t;
+      ineg |= n;
+    }
+  }
+  if (lane == 31) {
+    w_sum[warp] = inc;
+    w_neg[warp] = ineg;
+  }
+  __syncthreads();
+  if (warp == 0) {  // inclusive scan of the warp totals
+    int64_t v = w_sum[lane];
+    int n = w_neg[lane];
+    for (int o = 1; o < 32; o <<= 1) {
+      const int64_t t = __shfl_up_sync(0xffffffffu, v, o);
+      const int m = __shfl_up_sync(0xffffffffu, n, o);
+      if (lane >= o) {
+        v += t;
+        n |= m;
+      }
+    }
+    w_sum[lane] = v;
+    w_neg[lane] = n;
+  }
+  __syncthreads();
+  int64_t run = __shfl_up_sync(0xffffffffu, inc, 1);  // exclusive within the warp
+  int nrun = __shfl_up_sync(0xffffffffu, ineg, 1);
+  if (lane == 0) {
+    run = 0;
+    nrun = 0;
+  }
+  if (warp > 0) {
+    run += w_sum[warp - 1];
+    nrun |= w_neg[warp - 1];
+  }
+  for (int i = i0; i < i1; ++i) {
+    starts[i] = nrun ? -1 : run;
+    const int64_t li = __ldg(len + i);
+    run += li > 0 ? li : 0;
+    nrun |= li < 0;
+  }
+}
+
 // The cache as a 3-D tensor (d, head, row) with a box of {D, nh, 16}.
 bool make_cache_map(CUtensorMap* m, const NsaParams& p, int64_t rows, int nh) {
   sm100::EncodeTiledFn f = sm100::encode_fn();
@@ -160,15 +224,18 @@ cudaError_t launch_nsa(const NsaParams& p, cudaStream_t s) {
   // D <= 256 gives 32 KB)
   constexpr size_t kMaxSmem = (size_t)kTargetBytes + kTargetBytes / 2 + 64 * 64 * 4;
   const dim3 grid((unsigned)((p.N + nh - 1) / nh), (unsigned)p.B);
-  cudaError_t e;
-  if (p.bf16) {
-    e = smem_attr_once(nsa_kernel<true>, kMaxSmem, g_nsa_conf[1]);
-    if (e == cudaSuccess) nsa_kernel<true><<<grid, kThreads, smem, s>>>(map, p, nh, page_shift);
-  } else {
-    e = smem_attr_once(nsa_kernel<false>, kMaxSmem, g_nsa_conf[0]);
-    if (e == cudaSuccess) nsa_kernel<false><<<grid, kThreads, smem, s>>>(map, p, nh, page_shift);
-  }
-  return e != cudaSuccess ? e : cudaGetLastError();
+  auto* kernel = p.bf16 ? nsa_kernel<true> : nsa_kernel<false>;
+  cudaError_t e = smem_attr_once(kernel, kMaxSmem, g_nsa_conf[p.bf16 ? 1 : 0]);
+  if (e != cudaSuccess) return e;
+  if (p.packed)  // a programmatic dependent of nsa_scan_kernel
+    return launch_chained(kernel, grid, dim3(kThreads), smem, s, 1, map, p, nh, page_shift);
+  kernel<<<grid, kThreads, smem, s>>>(map, p, nh, page_shift);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_nsa_scan(const NsaParams& p, cudaStream_t s) {
+  nsa_scan_kernel<<<1, kScanThreads, 0, s>>>(p.len, p.B, p.starts);
+  return cudaGetLastError();
 }
 
 }  // namespace cmp

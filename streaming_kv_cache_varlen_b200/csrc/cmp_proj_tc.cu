@@ -245,19 +245,6 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 // ---- host side ------------------------------------------------------------------
 
-// 2D bf16 row-major [rows, cols] with a (box_rows x 64) box, 128-byte swizzle.
-bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows) {
-  EncodeTiledFn f = encode_fn();
-  if (!f) return false;
-  const cuuint64_t dims[2] = {cols, rows};
-  const cuuint64_t strides[1] = {cols * 2};
-  const cuuint32_t box[2] = {(cuuint32_t)BK, box_rows};
-  const cuuint32_t estr[2] = {1, 1};
-  return f(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
-           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 int sm_count() {
   int dev = 0, n = 148;
   cudaGetDevice(&dev);
@@ -273,8 +260,8 @@ bool proj_tc_supported(const Params& p) {
 
 cudaError_t launch_proj_tc(const Params& p, cudaStream_t s) {
   CUtensorMap mx, mkv, mg;
-  if (!make_map(&mx, p.x, p.T, p.H, BN) || !make_map(&mkv, p.wkv, p.C, p.H, BM) ||
-      !make_map(&mg, p.wgate, p.C, p.H, BM))
+  if (!make_tile_map(&mx, p.x, p.T, p.H, BN) || !make_tile_map(&mkv, p.wkv, p.C, p.H, BM) ||
+      !make_tile_map(&mg, p.wgate, p.C, p.H, BM))
     return cudaErrorInvalidValue;
   const size_t smem = sizeof(Smem) + 1024;
   static int configured[64] = {0};

@@ -47,16 +47,20 @@ def check(cmp, i):
     w = ref.written
     # slots not written: bit for bit the cache before the call
     assert np.array_equal(got[~w], i.output_cache[~w])
-    # written slots: the exact sum rounded once, within one unit of the dtype
-    # (the library sums in fp32, so a sum next to a rounding boundary may round
-    # to the other neighbour)
-    g = to_f64(got[w], i.dtype)
-    e = to_f64(ref.output_cache[w], i.dtype)
-    mant = 10 if i.dtype == "fp16" else 7
+    assert_within_one_unit(got[w], ref.output_cache[w], i.dtype)
+    return ref, got
+
+
+def assert_within_one_unit(got_bits, ref_bits, dtype):
+    """Written slots: the exact sum rounded once, within one unit of the dtype
+    (the library sums in fp32, so a sum next to a rounding boundary may round to
+    the other neighbour)."""
+    g = to_f64(got_bits, dtype)
+    e = to_f64(ref_bits, dtype)
+    mant = 10 if dtype == "fp16" else 7
     mag = np.maximum(np.abs(e), np.abs(g))
     ulp = np.exp2(np.floor(np.log2(np.maximum(mag, 1e-30))) - mant)
     assert (np.abs(g - e) <= ulp + 1e-5).all()
-    return ref, got
 
 
 @pytest.mark.parametrize("dtype", ["bf16", "fp16"])
@@ -143,3 +147,33 @@ def test_many_batches(lib, layout):
                         page_block_size=64, dtype="fp16", layout=layout, max_seq_len=128, trigger_fraction=0.8)
     ref, _ = check(lib, i)
     assert ref.written.sum() >= 700
+
+
+def test_packed_rows_of_many_batches(lib):
+    """20000 packed batches: every batch's first row comes from the scan kernel
+    (chunks of 20 lengths per thread, scanned across the block)."""
+    i = make_nsa_inputs(name="scan", seed=13, B=20000, N=1, D=16, compress_block_size=16, compress_stride=16,
+                        dtype="bf16", layout="TND", max_seq_len=64, trigger_fraction=0.5)
+    ref, _ = check(lib, i)
+    assert ref.written.sum() >= 8000
+
+
+def test_packed_negative_length_is_reported(lib):
+    """A negative length makes the rows of every later batch unknown: those
+    batches are skipped and reported; earlier ones are still written."""
+    import dataclasses
+    i = make_nsa_inputs(name="neg", seed=14, B=4, N=2, D=32, compress_block_size=32, compress_stride=16,
+                        dtype="fp16", layout="TND", lengths=[48, 40, 32, 64], max_seq_len=64)
+    lens = i.act_seq_len.copy()
+    lens[1] = -5
+    bad = dataclasses.replace(i, act_seq_len=lens)
+    got, err = gpu_call(lib, bad)
+    assert err == 5                            # CMP_ERR_DEVICE_INDEX
+    ref = nsa_compress(i.input, i.weight, i.slot_mapping, i.act_seq_len, i.block_table, i.output_cache,
+                       dtype=i.dtype, compress_block_size=32, compress_stride=16, layout="TND")
+    s0 = i.slot_mapping[0]
+    assert ref.written[s0]
+    assert_within_one_unit(got[s0], ref.output_cache[s0], i.dtype)
+    for b in (2, 3):
+        s = i.slot_mapping[b]
+        assert np.array_equal(got[s], i.output_cache[s])
