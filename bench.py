@@ -14,7 +14,12 @@ Also reported on the same line:
   * decode: the C4A 32-request decode step (one token each), microseconds per
     call, with L2 flushed before every timed call;
   * roofline: the projection kernel's tensor throughput against the measured
-    bf16 peak, and the decode call's HBM throughput against measured bandwidth;
+    bf16 peak (with the pooling epilogue's HBM throughput beside it), and the
+    decode call's HBM throughput against measured bandwidth;
+  * nsa: the NsaCompressWithCache decode step (128 batches), microseconds per
+    call with L2 flushed before every timed call, against HBM bandwidth;
+  * configs: the other workloads (c4li_tiny, c4a_varlen, c4li_chunked),
+    microseconds per step and projection TFLOP/s;
   * cpu_baseline: the CPU oracle on a bounded sample of the same workload.
 
 Multi-GPU (torchrun): every rank runs its own replica on its own GPU (requests
@@ -231,17 +236,23 @@ def prefill_inputs(device, seed: int):
                 ratio=r, rope_head_dim=64, rotate=False)
 
 
-def decode_inputs(device):
+def with_library_rope(inp):
+    """sin/cos rows for the output rows the library's layout gives (positions w*ratio)."""
     import numpy as np
-    import torch
 
     import streaming_kv_cache_varlen_b200 as cmp
-    from workloads import make_config, rope_tables
+    from workloads import rope_tables
 
-    inp = make_config("c4a_decode")
     rs, rw = cmp.out_row_layout(inp.cu_seqlens, inp.start_pos, inp.ratio)
     cos, sin = rope_tables(np.where(rw >= 0, rw * inp.ratio, 0), 64)
-    inp = inp.__class__(**{**inp.__dict__, "cos": cos, "sin": sin})
+    return inp.__class__(**{**inp.__dict__, "cos": cos, "sin": sin})
+
+
+def device_args(inp, device, kv_state=None, score_state=None):
+    """The compressor's arguments for ``inp`` as device tensors (states optional:
+    pass device buffers to carry state across calls)."""
+    import numpy as np
+    import torch
 
     def bfd(a):
         return None if a is None else torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).to(device).view(torch.bfloat16)
@@ -249,12 +260,87 @@ def decode_inputs(device):
     def d(a):
         return torch.from_numpy(np.ascontiguousarray(a)).to(device)
 
-    args = dict(x=bfd(inp.x), kv_state=d(inp.kv_state), score_state=d(inp.score_state),
+    return dict(x=bfd(inp.x), kv_state=d(inp.kv_state) if kv_state is None else kv_state,
+                score_state=d(inp.score_state) if score_state is None else score_state,
                 kv_block_table=d(inp.kv_block_table), state_block_table=d(inp.state_block_table),
                 sin=bfd(inp.sin), cos=bfd(inp.cos), wkv=bfd(inp.wkv), wgate=bfd(inp.wgate),
-                ape=d(inp.ape), norm_weight=bfd(inp.norm_weight), hadamard=None,
+                ape=d(inp.ape), norm_weight=bfd(inp.norm_weight), hadamard=bfd(inp.hadamard),
                 start_pos=d(inp.start_pos), cu_seqlens=d(inp.cu_seqlens), ratio=inp.ratio,
-                rope_head_dim=64, rotate=False)
+                rope_head_dim=64, rotate=inp.hadamard is not None)
+
+
+def bench_configs(args, ws, local, peaks, peak_src):
+    """The other workloads, reported beside the headline: c4li_tiny and
+    c4a_varlen (one call each) and c4li_chunked (its 4 calls, state carried from
+    call to call). Device time per step: a CUDA graph of 20 back-to-back steps
+    after 3 warm-ups, the best of 3 replays / 20 (a repeated step recomputes the
+    same values: a call reads only positions before its start and writes only
+    its tail), no L2 flush; achieved = the projection's 2*T*H*2C flop over
+    that time."""
+    import torch
+
+    import streaming_kv_cache_varlen_b200 as cmp
+    from workloads import make_chunked, make_config
+
+    device = torch.device("cuda", local)
+    res = {}
+    for name in ("c4li_tiny", "c4a_varlen", "c4li_chunked"):
+        if name == "c4li_chunked":
+            ch = make_chunked()
+            calls = [with_library_rope(c) for c in ch.calls]
+            first = device_args(calls[0], device)
+            steps_args = [first] + [device_args(c, device, first["kv_state"], first["score_state"])
+                                    for c in calls[1:]]
+        else:
+            calls = [with_library_rope(make_config(name))]
+            steps_args = [device_args(calls[0], device)]
+        outs = [torch.empty((cmp.out_rows(c.B, c.T, c.ratio), c.D), dtype=torch.bfloat16, device=device)
+                for c in calls]
+        flops = sum(2.0 * c.T * c.H * 2 * c.C for c in calls)
+
+        def step():
+            for a, o in zip(steps_args, outs):
+                cmp.compressor(**a, out=o)
+
+        side = torch.cuda.Stream(device)
+        side.wait_stream(torch.cuda.current_stream(device))  # inputs were made on the current stream
+        with torch.cuda.stream(side):
+            for _ in range(3):
+                step()
+        torch.cuda.synchronize()
+        assert cmp.get_error(side) == 0
+        n = 20
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=side):
+            for _ in range(n):
+                step()
+        torch.cuda.synchronize()
+        best = None
+        barrier(ws)
+        for _ in range(3):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            with torch.cuda.stream(side):
+                e0.record(side)
+                g.replay()
+                e1.record(side)
+            torch.cuda.synchronize()
+            best = e0.elapsed_time(e1) if best is None else min(best, e0.elapsed_time(e1))
+        us = max_over_ranks(best, ws) * 1e3 / n
+        assert cmp.get_error(side) == 0
+        del g
+        tf = flops / (us / 1e6) / 1e12
+        res[name] = {"calls_per_step": len(calls), "tokens_per_step": int(sum(c.T for c in calls)),
+                     "us_per_step": us, "tflops": tf, "frac_of_bf16_burst": tf / peaks["bf16_tflops"]}
+        del steps_args, outs
+        torch.cuda.empty_cache()
+    return res
+
+
+def decode_inputs(device):
+    from workloads import make_config
+
+    inp = with_library_rope(make_config("c4a_decode"))
+    args = device_args(inp, device)
     # algorithmic bytes of one decode call: both weight matrices, x, the earlier
     # state rows the completed windows pool (coff*ratio - 1 half rows of D floats,
     # kv and score), the state rows written (every token, kv and score), the ape
@@ -351,6 +437,18 @@ def bench_prefill(args, ws, local, stream, peaks, peak_src):
                 "frac_of_burst": achieved / peaks["bf16_tflops"] if achieved else None,
                 "algorithmic_flops_per_launch": flops,
                 "kernel_ms": {k: (v[0] / v[1] if v[1] else None) for k, v in prof.items()}}
+    # the pooling epilogue that follows the fused projection (merge, RMSNorm,
+    # RoPE, bf16 store): HBM, its algorithmic bytes over its launch time
+    f_ms, f_n = prof["finish"]
+    if f_n:
+        n_out, coff, D = out.shape[0], (2 if PREFILL["ratio"] == 4 else 1), PREFILL["D"]
+        fb = (n_out * coff * D * 4 * (2 if coff == 2 else 1)  # pooled halves (+ their lse)
+              + n_out * 64 * 2 * 2 + D * 2                   # sin, cos rows, norm_weight
+              + n_out * D * 2)                               # bf16 rows out
+        f_gbs = fb / (f_ms / f_n / 1e3) / 1e9
+        roofline["epilogue"] = {"kernel": "finish", "bound": "hbm", "us": f_ms / f_n * 1e3,
+                                "algorithmic_bytes": fb, "achieved": f_gbs, "unit": "GB/s",
+                                "frac": f_gbs / peaks["hbm_gbs"]}
     return dict(value=value, ms_step=ms / args.steps, launches=launches, roofline=roofline,
                 clocks=clocks, inputs=pf, out=out)
 
@@ -583,6 +681,9 @@ def run_ours(args):
     if args.only in ("all", "nsa"):
         nsa = bench_nsa(args, ws, local, peaks, peak_src)
         torch.cuda.empty_cache()
+    configs = None
+    if args.only in ("all", "configs"):
+        configs = bench_configs(args, ws, local, peaks, peak_src)
     cpu = None
     if rank == 0 and ws == 1 and args.only == "all" and not args.no_cpu_baseline:
         cpu = cpu_baseline(args.cpu_tokens or cpu_sample_tokens(args.cpu_seconds))
@@ -599,7 +700,7 @@ def run_ours(args):
                            "parallelism": f"dp{ws} (independent replicas)",
                            "l2": "inputs larger than L2 (x is 1 GiB per step)"},
                 "e2e": e2e, "gpu_launches": pre["launches"] if pre else None,
-                "roofline": pre["roofline"] if pre else None, "decode": decode, "nsa": nsa,
+                "roofline": pre["roofline"] if pre else None, "decode": decode, "nsa": nsa, "configs": configs,
                 "clocks": pre["clocks"] if pre else None, "cpu_baseline": cpu}
         print(json.dumps(line), flush=True)
     if ws > 1:
@@ -686,7 +787,7 @@ def main():
                     help="tokens of the CPU-baseline sample (default: about --cpu-seconds of oracle work)")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--only", choices=("all", "prefill", "decode", "nsa"), default="all",
+    ap.add_argument("--only", choices=("all", "prefill", "decode", "nsa", "configs"), default="all",
                     help="run only one part (for profiler captures)")
     ap.add_argument("--prefill-tokens", type=int, default=PREFILL["T"],
                     help="tokens of the prefill sequence (smaller cases for profiler captures)")

@@ -76,9 +76,12 @@ WsLayout ws_layout(int64_t B, int64_t T, int64_t C, int64_t n_out, bool fused, s
 int choose_path(const Params& p, int forced) {
   int which = forced;
   if (which == 0) {
+    // small T: the channel-group kernel; else weight streaming, which measured
+    // as fast or faster than the K-split kernel on the decode shapes (much
+    // faster when each K slice would be one or two 64-column steps)
     if (cmp::decode_cp_supported(p)) which = 6;
-    else if (cmp::decode_fused_supported(p)) which = 5;
     else if (cmp::proj_decode_supported(p)) which = 3;
+    else if (cmp::decode_fused_supported(p)) which = 5;
     else if (cmp::fused_supported(p) && p.T >= 1024 && (int64_t)p.T >= 256LL * p.B) which = 4;
     else if (cmp::proj_tc_supported(p)) which = 2;
     else which = 1;
