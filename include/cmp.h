@@ -291,8 +291,8 @@ CMP_API int cmp_profile_stop(double* ms, int64_t* launches);
  * channel-group decode kernel, or without it (rotate, or a device that cannot
  * hold its clusters) the weight-streaming projection + pooling kernels, else
  * the K-split one-kernel decode; the fused tcgen05 pooling kernel for long
- * sequences, T >= 1024 and T >= 256*B; else the tcgen05 projection + pooling
- * kernel), 1 = force the mma.sync projection, 2 = the tcgen05 projection,
+ * sequences, T >= 1024 and T >= 256*B, when its (T/256)*(C/128) work items
+ * fill the SMs twice; else the tcgen05 projection + pooling kernel), 1 = force the mma.sync projection, 2 = the tcgen05 projection,
  * 3 = weight streaming, 4 = the fused path, 5 = the K-split one-kernel decode,
  * 6 = the channel-group decode. A forced path a call cannot take falls back
  * to 1.

@@ -73,6 +73,12 @@ WsLayout ws_layout(int64_t B, int64_t T, int64_t C, int64_t n_out, bool fused, s
 // 3 small-T weight streaming (+ pooling kernel), 4 fused tcgen05 pooling
 // (+ finish kernel), 5 decode in one cooperative kernel (K-split grid),
 // 6 decode in one cooperative kernel of channel-group clusters.
+int sm_count_cached();
+
+// The fused prefill's work items (256-position tiles x 128-channel blocks),
+// estimated from the token count (the lengths are on the device).
+int64_t fused_items_estimate(const Params& p) { return ((int64_t)p.T / 256) * (p.C / 128); }
+
 int choose_path(const Params& p, int forced) {
   int which = forced;
   if (which == 0) {
@@ -82,7 +88,12 @@ int choose_path(const Params& p, int forced) {
     if (cmp::decode_cp_supported(p)) which = 6;
     else if (cmp::proj_decode_supported(p)) which = 3;
     else if (cmp::decode_fused_supported(p)) which = 5;
-    else if (cmp::fused_supported(p) && p.T >= 1024 && (int64_t)p.T >= 256LL * p.B) which = 4;
+    // the fused kernel when its items fill the SMs at least twice (narrow state
+    // rows over ~10K tokens leave it half the GPU: the separate projection, with
+    // twice the items, measured 17 % faster there)
+    else if (cmp::fused_supported(p) && p.T >= 1024 && (int64_t)p.T >= 256LL * p.B &&
+             (fused_items_estimate(p) >= 2LL * sm_count_cached() || !cmp::proj_tc_supported(p)))
+      which = 4;
     else if (cmp::proj_tc_supported(p)) which = 2;
     else which = 1;
   }
