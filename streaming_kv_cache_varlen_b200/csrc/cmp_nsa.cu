@@ -52,6 +52,15 @@ __global__ void __launch_bounds__(kThreads)
     nsa_kernel(const __grid_constant__ CUtensorMap map, NsaParams p, int nh, int page_shift) {
   const int b = blockIdx.y;
   const int h0 = blockIdx.x * nh;
+  const int lane = threadIdx.x & 31;
+  // paged, table rows of at most 32 pages: warp 0 loads the batch's whole row
+  // together with its length and slot, so the entries are at hand when the
+  // window is known (one round trip instead of two)
+  const bool row_in_warp = !p.packed && p.table_stride <= 32;
+  const int32_t* trow = p.table + (int64_t)b * p.table_stride;
+  int32_t tpre = -1;
+  if (threadIdx.x < 32 && row_in_warp && lane < p.table_stride) tpre = __ldg(trow + lane);
+  const int slot = threadIdx.x == 0 ? __ldg(p.slot + b) : 0;
   const int64_t s = __ldg(p.len + b);
   if (s < p.cbs || (s - p.cbs) % p.stride != 0) return;  // not a compression step (whole CTA)
   extern __shared__ __align__(128) unsigned char smem_raw[];
@@ -61,37 +70,45 @@ __global__ void __launch_bounds__(kThreads)
   float* wsm = reinterpret_cast<float*>(buf + (size_t)p.cbs * per_tok);  // [cbs][nh]
   __shared__ __align__(8) uint64_t full;
   __shared__ int ok;
-  if (threadIdx.x == 0) {
-    sm100::prefetch_tmap(&map);
-    const int slot = __ldg(p.slot + b);
-    bool good = slot >= 0 && slot < p.result_len;
+  if (threadIdx.x < 32) {  // warp 0: validation; lane 0 issues the copies
     const int64_t first = s - p.cbs;
     const int runs = p.cbs / kRun;
     int64_t row[64 / kRun];
+    bool good = slot >= 0 && slot < p.result_len;
     if (p.packed) {
-      pdl_wait();  // the row starts come from nsa_scan_kernel, launched just before
-      const int64_t start = p.starts[b];
-      good = good && start >= 0 && start + s <= p.tokens;
-      for (int k = 0; k < runs; ++k) row[k] = start + first + k * kRun;
+      if (lane == 0) {
+        pdl_wait();  // the row starts come from nsa_scan_kernel, launched just before
+        const int64_t start = p.starts[b];
+        good = good && start >= 0 && start + s <= p.tokens;
+        for (int k = 0; k < runs; ++k) row[k] = start + first + k * kRun;
+      }
     } else {
-      const int32_t* trow = p.table + (int64_t)b * p.table_stride;
       const int64_t mask = (int64_t(1) << page_shift) - 1;
       for (int k = 0; k < runs; ++k) {
         const int64_t pos = first + k * kRun;
         const int64_t pg = pos >> page_shift;
-        const int32_t blk = pg < p.table_stride ? __ldg(trow + pg) : -1;
+        int32_t blk;
+        if (row_in_warp) {  // uniform across the warp: every lane shuffles
+          const int32_t v = __shfl_sync(0xffffffffu, tpre, (int)(pg & 31));
+          blk = pg < p.table_stride ? v : -1;
+        } else {
+          blk = lane == 0 && pg < p.table_stride ? __ldg(trow + pg) : -1;
+        }
         good = good && blk >= 0 && blk < p.tokens;
         row[k] = ((int64_t)blk << page_shift) + (pos & mask);
       }
     }
-    if (!good) atomicOr(p.err, kErrIndex);
-    ok = good ? 1 : 0;
-    if (good) {
-      sm100::mbar_init(&full, 1);
-      sm100::fence_barrier_init();
-      sm100::mbar_arrive_expect_tx(&full, (uint32_t)(p.cbs * per_tok * 2));
-      for (int k = 0; k < runs; ++k)
-        sm100::tma_load_3d(buf + (size_t)k * kRun * per_tok, &map, &full, 0, h0, (int)row[k]);
+    if (lane == 0) {
+      if (!good) atomicOr(p.err, kErrIndex);
+      ok = good ? 1 : 0;
+      if (good) {
+        sm100::prefetch_tmap(&map);
+        sm100::mbar_init(&full, 1);
+        sm100::fence_barrier_init();
+        sm100::mbar_arrive_expect_tx(&full, (uint32_t)(p.cbs * per_tok * 2));
+        for (int k = 0; k < runs; ++k)
+          sm100::tma_load_3d(buf + (size_t)k * kRun * per_tok, &map, &full, 0, h0, (int)row[k]);
+      }
     }
   }
   for (int i = threadIdx.x; i < p.cbs * nh; i += kThreads) {

@@ -177,3 +177,15 @@ def test_packed_negative_length_is_reported(lib):
     for b in (2, 3):
         s = i.slot_mapping[b]
         assert np.array_equal(got[s], i.output_cache[s])
+
+
+@pytest.mark.parametrize("pbs", [64, 128])
+def test_long_table_rows(lib, pbs):
+    """Table rows wider than 32 pages (the entries are then read one by one
+    instead of from the warp's copy of the row), windows deep in the row."""
+    i = make_nsa_inputs(name="longrow", seed=15 + pbs, B=6, N=2, D=16, compress_block_size=64,
+                        compress_stride=32, page_block_size=pbs, dtype="bf16", layout="paged",
+                        max_seq_len=64 * pbs, trigger_fraction=1.0)
+    assert i.block_table.shape[1] == 64
+    ref, _ = check(lib, i)
+    assert ref.written.sum() == 6
