@@ -188,7 +188,7 @@ __device__ __forceinline__ uint32_t peer_addr(const void* local, uint32_t peer) 
 }
 
 // Bulk copy of `bytes` from this CTA's shared memory into a peer's, completing
-// on the peer's mbarrier (both addresses from peer_addr). No multicast.
+// on the peer's mbarrier (both addresses from peer_addr); one destination CTA per copy.
 __device__ __forceinline__ void bulk_copy_to_peer(uint32_t dst, const void* src, uint32_t bytes, uint32_t mbar) {
   asm volatile(
       "cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
@@ -249,7 +249,7 @@ __device__ __forceinline__ int table_entry(const Params& p, const int32_t* __res
 // Warps 2-3: validation, output-row offsets, per-token facts, the window of
 // every output row, and, for this CTA's channels (columns half * D + ch0 .. +3),
 // the state rows of those windows, ape, norm_weight and the RoPE table entries.
-// Loads are grouped in three rounds: inputs, block-table entries, state rows.
+// Loads are grouped in three waves: inputs, block-table entries, state rows.
 template <int MAXT>
 __device__ void call_metadata(const Params& p, Smem<MAXT>& sm, int NT, int ch0) {
   const int et = threadIdx.x - 64;  // 0..63
@@ -258,7 +258,7 @@ __device__ void call_metadata(const Params& p, Smem<MAXT>& sm, int NT, int ch0) 
   const int r0 = p.D - p.rope, hr = p.rope / 2;
   const bool roped = ch0 >= r0;
 
-  // ---- round 1: everything that depends on nothing ----
+  // ---- first wave of loads: everything that depends on nothing ----
   int cuv[5], spv[4];
 #pragma unroll
   for (int u = 0; u < 5; ++u) {
@@ -436,7 +436,7 @@ __device__ void call_metadata(const Params& p, Smem<MAXT>& sm, int NT, int ch0) 
   }
   asm volatile("bar.sync 2, 64;" ::: "memory");
 
-  // ---- round 2: block-table entries (tails, then hist rows i = et + 64u) ----
+  // ---- second wave of loads: block-table entries (tails, then hist rows i = et + 64u) ----
   const int total = sm.hstart[p.n_out];
   int hb[4], hq[4], hj[4];
 #pragma unroll
@@ -473,7 +473,7 @@ __device__ void call_metadata(const Params& p, Smem<MAXT>& sm, int NT, int ch0) 
     sm.tok[et] = ti;
   }
 
-  // ---- round 3: the state rows (a row that does not exist: kv 0, score -inf) ----
+  // ---- third wave of loads: the state rows (a row that does not exist: kv 0, score -inf) ----
   float4 v[4][2];
 #pragma unroll
   for (int u = 0; u < 4; ++u) {
