@@ -561,7 +561,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_arrive_expect_tx(&sm.recv_full, (uint32_t)(KQ * kinds * p.T * OWN * 4));
     prefetch_tmap(&map_w);
     prefetch_tmap(&map_x);
-    sm.bar_target = grid_target(a.counter);
   }
   if (warp == 1) tmem_alloc(&sm.tmem_base, tmem_cols);
   cluster_arrive_relaxed();  // cluster barrier 0: this CTA runs (its barriers are initialized)
@@ -610,6 +609,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     if (ok) mma_commit(&sm.acc_full);
   } else if (warp >= 2) {
+    // the grid barrier's target, read here rather than before the stream starts
+    // (a cold global load); any time before this CTA's own arrival is correct:
+    // the count cannot reach the next multiple while this CTA's share is missing
+    if (threadIdx.x == 64) sm.bar_target = grid_target(a.counter);
     call_metadata<MAXT>(p, sm, NT, ch0);
   }
 
