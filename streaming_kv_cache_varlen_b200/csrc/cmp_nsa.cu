@@ -42,11 +42,13 @@ __device__ __forceinline__ uint32_t pack(float lo, float hi) {
   return *reinterpret_cast<const uint32_t*>(&h);
 }
 
-// Thread 0 validates the batch's slot and the cache rows of its window, then
-// issues the window's cbs / 16 boxes (heads h0 .. h0 + nh - 1; heads past N read
-// as zeros and are not stored), all completing on one mbarrier; the other
+// Warp 0 validates the batch's slot and the cache rows of its window, then lane
+// 0 issues the window's cbs / 16 boxes (heads h0 .. h0 + nh - 1; heads past N
+// read as zeros and are not stored), all completing on one mbarrier; the other
 // threads stage the weights meanwhile. Then each thread sums 4 consecutive
 // elements of one head over the window's tokens in order and stores them.
+// Packed layout (a programmatic dependent of nsa_scan_kernel): only lane 0 waits
+// for the scan, and every thread's stores come after it through __syncthreads.
 template <bool BF16>
 __global__ void __launch_bounds__(kThreads)
     nsa_kernel(const __grid_constant__ CUtensorMap map, NsaParams p, int nh, int page_shift) {
