@@ -337,7 +337,7 @@ def _check_args(a):
 def compressor(x, kv_state, score_state, kv_block_table, state_block_table, sin, cos,
                wkv, wgate, ape, norm_weight, hadamard, start_pos, cu_seqlens,
                ratio, rope_head_dim, rotate, *, windows_only: Optional[Sequence[int]] = None,
-               write_state: bool = True, chunk: int = 512) -> Result:
+               write_state: bool = True, chunk: int = 512, round_after_norm: bool = False) -> Result:
     """One call of the Compressor, with the argument order of the pages' prototype
     ("函数原型": x, kv_state, score_state, kv_block_table, state_block_table, sin, cos,
     wkv, wgate, ape, weight, hadamard, start_pos, ratio, rope_head_dim, rotate),
@@ -348,6 +348,12 @@ def compressor(x, kv_state, score_state, kv_block_table, state_block_table, sin,
     listed output rows (for spot checks of very large calls); other rows then
     come back as NaN in the float arrays and 0 in ``out``. ``write_state=False``
     skips the state update.
+
+    ``round_after_norm`` rounds the RMSNorm result to bf16 before RoPE and the
+    rotation: the PyPTO walk-through's rms_norm helper works in fp32 and casts its
+    result back to the input dtype (算子级辅助函数). The default keeps float64 up to
+    the one final rounding. The output tolerance is meant to hold for either
+    reading.
     """
     a = _as_dict(x=np.asarray(x), kv_state=np.asarray(kv_state, dtype=np.float32),
                  score_state=np.asarray(score_state, dtype=np.float32),
@@ -393,6 +399,8 @@ def compressor(x, kv_state, score_state, kv_block_table, state_block_table, sin,
     out_f = normed.copy()
     if sel.any():
         z = rms_norm(pooled[sel], norm_weight)
+        if round_after_norm:
+            z = bf16_to_f64(f64_to_bf16_bits(z))
         normed[sel] = z
         z = rope_interleaved(z, np.asarray(cos)[sel], np.asarray(sin)[sel], int(rope_head_dim))
         if rotate:

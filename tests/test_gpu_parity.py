@@ -314,3 +314,20 @@ def test_bad_cu_seqlens_rejected_on_device(lib):
     out = lib.compressor(**args)
     assert lib.get_error() == 5
     assert (bits(out) == 0).all() and torch.equal(args["kv_state"], kv0)
+
+
+@pytest.mark.parametrize("case", ["c4li_tiny", "c4a_short"])
+def test_output_within_tolerance_of_both_rounding_readings(lib, case):
+    """The library keeps fp32 to the final bf16 store; the output must be within
+    the stated tolerance of the oracle both without and with a bf16 rounding
+    after RMSNorm (the PyPTO helper's cast back to the input dtype)."""
+    if case == "c4li_tiny":
+        inp = make_config("c4li_tiny")
+    else:
+        inp = make_inputs(name="c4a_short", seed=21, lengths=[67, 130], start_pos=[0, 5], H=512, D=512,
+                          coff=2, ratio=4, block_size=16, rotate=False)
+    inp = with_rope(inp)
+    out, _, _, err = run(lib, inp)
+    assert err == 0
+    assert_out_close(out, run_inputs(inp))
+    assert_out_close(out, run_inputs(inp, round_after_norm=True))
