@@ -299,6 +299,15 @@ CMP_API int cmp_profile_stop(double* ms, int64_t* launches);
  * Returns the previous value, or -1 if out of range. */
 CMP_API int cmp_set_proj_kernel(int which);
 
+/* Testing knob for failure detection: the next `launches` launches of the
+ * channel-group decode kernel (CMP_KERNEL_DECODE_CP) wait at their grid barrier
+ * for a count no arrival reaches. Each CTA's bounded wait gives up after about
+ * one second, the rows of the call come out as zeros, the CTAs free their tensor
+ * memory and return, and cmp_get_error then reports CMP_ERR_TIMEOUT and resets
+ * the barrier words, so the next call runs normally. Nothing faults or hangs.
+ * Returns the previous count, or -1 if launches < 0. */
+CMP_API int cmp_debug_unreachable_barrier(int launches);
+
 #ifdef __cplusplus
 }
 #endif

@@ -63,6 +63,7 @@ def _load() -> ctypes.CDLL:
         "cmp_profile_start": (ctypes.c_int, []),
         "cmp_profile_stop": (ctypes.c_int, [P, P]),
         "cmp_set_proj_kernel": (ctypes.c_int, [ctypes.c_int]),
+        "cmp_debug_unreachable_barrier": (ctypes.c_int, [ctypes.c_int]),
         "cmp_nsa_compress": (ctypes.c_int, [P, P, P, P, P, I32, I32, I64, I64, I64, P, P,
                                             ctypes.POINTER(cmp_nsa_dims)]),
     }
@@ -276,6 +277,13 @@ def profile_stop() -> Dict[str, Tuple[float, int]]:
     if st != CMP_OK:
         raise CmpError(st, "cmp_profile_stop")
     return {KERNELS[i]: (float(ms[i]), int(n[i])) for i in range(len(KERNELS))}
+
+
+def debug_unreachable_barrier(launches: int) -> int:
+    """Testing knob: the next ``launches`` channel-group decode launches time out
+    at their grid barrier (about 1 s each; get_error then reports
+    CMP_ERR_TIMEOUT). Returns the previous count."""
+    return int(lib.cmp_debug_unreachable_barrier(launches))
 
 
 def set_proj_kernel(which: int) -> int:

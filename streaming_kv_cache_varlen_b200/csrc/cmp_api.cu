@@ -21,7 +21,7 @@ size_t decode_fused_workspace(const Params& p);
 cudaError_t launch_decode_fused(const Params& p, float* part, void* bar, cudaStream_t s);
 bool decode_cp_supported(const Params& p);
 size_t decode_cp_workspace(const Params& p);
-cudaError_t launch_decode_cp(const Params& p, float* ss, void* counter, cudaStream_t s);
+cudaError_t launch_decode_cp(const Params& p, float* ss, void* counter, cudaStream_t s, bool unreachable);
 cudaError_t launch_nsa(const NsaParams& p, cudaStream_t s);
 cudaError_t launch_nsa_scan(const NsaParams& p, cudaStream_t s);
 }  // namespace cmp
@@ -126,6 +126,7 @@ std::map<std::pair<int, cudaStream_t>, Workspace> g_ws;
 std::map<std::pair<int, cudaStream_t>, unsigned> g_pending_err;  // kept across a regrow
 std::atomic<int64_t> g_launches{0};
 std::atomic<int> g_proj_kernel{0};
+std::atomic<int> g_unreachable_barrier{0};  // launches left whose grid barrier cannot be reached
 
 // ---- profiling ---------------------------------------------------------------
 
@@ -258,8 +259,11 @@ int run_path(Params& p, int which, cudaStream_t s) {
   if (which == 6) {  // decode: one cooperative kernel of clusters, no scheduler launch
     float* ss = reinterpret_cast<float*>(ws + L.part);
     void* counter = ws + L.err + kCounterOffset;
-    const cudaError_t e =
-        launch(CMP_KERNEL_DECODE_CP, s, [&] { return cmp::launch_decode_cp(p, ss, counter, s); });
+    bool unreachable = false;  // the timeout test's knob, consumed one launch at a time
+    for (int v = g_unreachable_barrier.load(); v > 0 && !unreachable;)
+      unreachable = g_unreachable_barrier.compare_exchange_weak(v, v - 1);
+    const cudaError_t e = launch(CMP_KERNEL_DECODE_CP, s,
+                                 [&] { return cmp::launch_decode_cp(p, ss, counter, s, unreachable); });
     if (e == cudaErrorNotSupported) return kRetryOtherPath;
     return e == cudaSuccess ? CMP_OK : CMP_ERR_CUDA;
   }
@@ -482,6 +486,11 @@ int cmp_nsa_compress(const void* input, const void* weight, const int32_t* slot_
     return CMP_ERR_CUDA;
   if (launch(CMP_KERNEL_NSA, s, [&] { return cmp::launch_nsa(p, s); }) != cudaSuccess) return CMP_ERR_CUDA;
   return CMP_OK;
+}
+
+int cmp_debug_unreachable_barrier(int launches) {
+  if (launches < 0) return -1;
+  return g_unreachable_barrier.exchange(launches);
 }
 
 int cmp_get_error(void* stream) {

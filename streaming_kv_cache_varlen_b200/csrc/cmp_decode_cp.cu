@@ -226,6 +226,7 @@ struct CpArgs {
   float* ss;          // [kReplicas][n_out][D/4] each CTA's sum of squares of its channels, per output row
   unsigned* counter;  // grid-barrier counter (zeroed at creation)
   int kv_first;     // the 4-D weight map holds wkv before wgate (else the other way round)
+  uint32_t bar_extra;  // added to the barrier target: kQuantum makes it unreachable (timeout test)
 };
 
 // Window row j of window w: its absolute position (rows are in rising order).
@@ -615,7 +616,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // the grid barrier's target, read here rather than before the stream starts
     // (a cold global load); any time before this CTA's own arrival is correct:
     // the count cannot reach the next multiple while this CTA's share is missing
-    if (threadIdx.x == 64) sm.bar_target = grid_target(a.counter);
+    if (threadIdx.x == 64) sm.bar_target = grid_target(a.counter) + a.bar_extra;
     call_metadata<MAXT>(p, sm, NT, ch0);
   }
 
@@ -914,7 +915,7 @@ size_t decode_cp_workspace(const Params& p) {
 // Launch. If the device refuses the launch form itself (a cooperative launch of
 // clusters), the path is disabled on this device and cudaErrorNotSupported is
 // returned before anything ran, so that the caller can take another path.
-cudaError_t launch_decode_cp(const Params& p, float* ss, void* counter, cudaStream_t s) {
+cudaError_t launch_decode_cp(const Params& p, float* ss, void* counter, cudaStream_t s, bool unreachable) {
   const int NT = (p.T + 15) / 16 * 16;
   CUtensorMap mx, mw;
   CpArgs a;
@@ -922,6 +923,7 @@ cudaError_t launch_decode_cp(const Params& p, float* ss, void* counter, cudaStre
     return cudaErrorInvalidValue;
   a.ss = ss;
   a.counter = static_cast<unsigned*>(counter);
+  a.bar_extra = unreachable ? kQuantum : 0u;
   const int grid = (p.D / GCH) * KQ;
   cudaLaunchAttribute attr[2];
   cudaError_t e;

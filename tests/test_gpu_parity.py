@@ -331,3 +331,28 @@ def test_output_within_tolerance_of_both_rounding_readings(lib, case):
     assert err == 0
     assert_out_close(out, run_inputs(inp))
     assert_out_close(out, run_inputs(inp, round_after_norm=True))
+
+
+def test_barrier_timeout_is_reported_and_the_next_call_recovers(lib):
+    """Failure detection without a GPU fault: a testing knob makes one launch of
+    the channel-group decode kernel wait at its grid barrier for a count no
+    arrival reaches. Every CTA's bounded wait gives up after about a second, the
+    call reports CMP_ERR_TIMEOUT, get_error resets the barrier words, and the
+    next call runs normally and matches the oracle."""
+    import time
+    inp = with_rope(make_config("c4a_decode"))
+    prev = lib.set_proj_kernel(6)
+    try:
+        assert lib.debug_unreachable_barrier(1) == 0
+        n0 = lib.launch_count()
+        t0 = time.monotonic()
+        _, _, _, err = run(lib, inp)
+        assert err == 6                                  # CMP_ERR_TIMEOUT
+        assert time.monotonic() - t0 < 30
+        assert lib.launch_count() - n0 == 1              # the channel-group kernel, once
+        assert lib.debug_unreachable_barrier(0) == 0     # the knob was consumed
+        check(lib, inp)                                  # the context and the barrier recovered
+        check(lib, inp)
+    finally:
+        lib.debug_unreachable_barrier(0)
+        lib.set_proj_kernel(prev)
