@@ -189,3 +189,21 @@ def test_long_table_rows(lib, pbs):
     assert i.block_table.shape[1] == 64
     ref, _ = check(lib, i)
     assert ref.written.sum() == 6
+
+
+def test_largest_heads_and_window(lib):
+    """N = 64 heads of D = 256 with a 64-token window: 32 KB per head, one head
+    per CTA, the largest shared-memory window a call can ask for."""
+    i = make_nsa_inputs(name="maxhead", seed=16, B=4, N=64, D=256, compress_block_size=64, compress_stride=64,
+                        page_block_size=128, dtype="fp16", layout="paged", max_seq_len=256, trigger_fraction=1.0)
+    ref, _ = check(lib, i)
+    assert ref.written.sum() == 4
+
+
+@pytest.mark.parametrize("layout", ["paged", "TND"])
+def test_most_batches(lib, layout):
+    """B = 65535, the largest batch count (one grid row per batch)."""
+    i = make_nsa_inputs(name="maxb", seed=17, B=65535, N=1, D=16, compress_block_size=16, compress_stride=16,
+                        page_block_size=64, dtype="bf16", layout=layout, max_seq_len=64, trigger_fraction=0.5)
+    ref, _ = check(lib, i)
+    assert ref.written.sum() >= 30000
