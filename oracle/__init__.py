@@ -17,7 +17,12 @@ the pins are brute force on tiny inputs, closed forms (equal scores give the
 window mean, one dominant score selects its row, masked first window, RMSNorm
 unit rms, RoPE identity and pair norms, Hadamard orthogonality) and the
 streaming invariants (token by token, chunked and reordered calls equal one
-call). See tests/test_oracle_pins.py. ``oracle.nsa`` is pinned by the example
+call). See tests/test_oracle_pins.py. One exception, parity unpinned: where
+several sequences share a call, the placement of their output rows
+(``compressor.layout``) is a reading; no page prints one. The pins fix only what
+the pages fix there: the row count min(T, T//ratio + B), zero rows without a
+window, one row per request in request order for decode, and window order for
+one sequence. ``oracle.nsa`` is pinned by the example
 of its page (a closed form on its all-ones inputs), brute force, the trigger
 rule and closed forms (tests/test_oracle_nsa.py).
 """

@@ -27,8 +27,9 @@ of the current one; ape row = position mod ratio; state slot of position p =
 (table[b][p // block_size], p % block_size); the state rows written are the
 tail rows a later call can still read; output row of the k-th window that
 sequence b completes = sum of earlier sequences' capacities min(L, L//ratio+1)
-plus k; interleaved RoPE pairs (2j, 2j+1) of the last rope_head_dim channels,
-using table columns j and rope_head_dim/2 + j.
+plus k (parity unpinned: no page prints a multi-sequence row placement); interleaved
+RoPE pairs (2j, 2j+1) of the last rope_head_dim channels, using table columns j and
+rope_head_dim/2 + j.
 """
 
 from __future__ import annotations
