@@ -18,7 +18,7 @@ from __future__ import annotations
 
 import math
 import struct
-from typing import Dict, List, Optional, Sequence, Tuple
+from typing import Dict, List, Sequence, Tuple
 
 
 def _bf16(u: int) -> float:

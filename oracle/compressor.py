@@ -35,7 +35,6 @@ rope_head_dim/2 + j.
 from __future__ import annotations
 
 import dataclasses
-import math
 from typing import List, Optional, Sequence, Tuple
 
 import numpy as np

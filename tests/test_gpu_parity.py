@@ -13,7 +13,7 @@ import numpy as np
 import pytest
 
 from oracle import run_inputs, window_row_positions
-from workloads import make_chunked, make_config, make_inputs, bf16_bits, sylvester
+from workloads import make_chunked, make_config, make_inputs, bf16_bits
 from tests.gpu_helpers import (assert_out_close, assert_state_close, bits, dev, run, to_device)
 
 pytestmark = pytest.mark.gpu

@@ -17,7 +17,7 @@ import oracle
 from oracle import brute
 from oracle.compressor import (bf16_to_f64, compressor, f64_to_bf16_bits, layout, out_rows,
                                run_inputs, window_row_positions)
-from workloads import bf16_bits, hadamard_bits, make_inputs, rope_tables, sylvester
+from workloads import bf16_bits, hadamard_bits, make_inputs, sylvester
 
 GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
 
