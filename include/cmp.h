@@ -237,8 +237,12 @@ enum { CMP_NSA_PAGED = 0, CMP_NSA_PACKED = 1 };
  * int32 [B], distinct values in [0, result_len). act_seq_len: device int64 [B].
  * block_table: device int32 [B, table_stride] (paged; NULL allowed when packed).
  * output_cache: device [result_len, N, D], same dtype, updated in place;
- * 16-byte aligned. All memory is the caller's; the call is asynchronous on
- * `stream` (a cudaStream_t, NULL = default stream).
+ * 16-byte aligned. The call is asynchronous on `stream` (a cudaStream_t, NULL =
+ * default stream). It keeps its error word, and for the packed layout the B
+ * batches' first rows (8 * B bytes), in the library's workspace for this device
+ * and stream. Growing that workspace synchronises the device, so make the
+ * largest call once before capturing calls into a CUDA graph, as for
+ * cmp_compressor. All other memory is the caller's.
  * compress_block_size: a multiple of 16 in [16, 64], >= compress_stride;
  * compress_stride: 16, 32, 48 or 64; page_block_size: 64 or 128 (paged).
  * Returns CMP_OK, CMP_ERR_NULLPTR (a required pointer or dims is NULL),
