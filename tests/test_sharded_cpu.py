@@ -10,6 +10,8 @@ import socket
 import numpy as np
 import pytest
 import torch
+from hypothesis import given, settings
+from hypothesis import strategies as st
 import torch.multiprocessing as mp
 
 from streaming_kv_cache_varlen_b200 import sharded
@@ -99,7 +101,20 @@ def test_plan_partitions_windows(ratio):
                                                   (4, 8, 4, False), (128, 1100, 3, False),
                                                   (2, 333, 2, False), (4, 7, 3, False)])
 def test_emulated_ranks_equal_one_shot(ratio, T, world, rotate):
-    inp = one_sequence(T, ratio, seed=ratio + T, rotate=rotate)
+    emulate_and_check(ratio, T, world, rotate, seed=ratio + T)
+
+
+@settings(max_examples=25, deadline=None, derandomize=True)
+@given(ratio=st.sampled_from([1, 2, 4, 8, 16, 128]), T=st.integers(1, 300), world=st.integers(1, 6),
+       rotate=st.booleans(), bs=st.sampled_from([16, 32, 64]), seed=st.integers(0, 1000))
+def test_emulated_ranks_equal_one_shot_random(ratio, T, world, rotate, bs, seed):
+    """Random lengths, ratios, rank counts and block sizes: the assembled rows
+    and the state tail equal the one-shot oracle bit for bit."""
+    emulate_and_check(ratio, T, world, rotate, seed=seed, bs=bs)
+
+
+def emulate_and_check(ratio, T, world, rotate, seed, bs=32):
+    inp = one_sequence(T, ratio, seed=seed, rotate=rotate, bs=bs)
     ref = one_shot(inp)
     args = common_args(inp)
     shards = sharded.plan(T, ratio, world)
