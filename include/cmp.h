@@ -146,7 +146,8 @@ CMP_API int cmp_out_row_layout(const int32_t* cu_seqlens, const int32_t* start_p
  * if a later call needs more); see cmp_workspace_size / cmp_release_workspaces.
  * Results are bitwise reproducible run to run (no floating-point atomics).
  * Requirements the library does not check: the pool rows used by different
- * sequences are disjoint, and the tables map the blocks a call needs.
+ * sequences are disjoint, and the tables map the blocks a call needs (the Python
+ * binding's debug_check_tables checks both on the host, for tests and debugging).
  *
  * Returns CMP_OK, CMP_ERR_NULLPTR, CMP_ERR_INVALID, CMP_ERR_UNSUPPORTED or
  * CMP_ERR_CUDA, all decided on the host before anything is launched, except

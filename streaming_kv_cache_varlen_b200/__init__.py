@@ -241,6 +241,54 @@ def nsa_compress(input, weight, slot_mapping, act_seq_len, output_cache, *, comp
     return output_cache
 
 
+def debug_check_tables(kv_block_table, state_block_table, cu_seqlens, start_pos, ratio: int,
+                       block_size: int, block_num: int):
+    """Host-side check of a call's documented preconditions, for tests and
+    debugging (the library never runs it): every table entry the call reads or
+    writes lies in [0, block_num), and no pool row is used by two sequences.
+    Sequence b at positions [s, e) reads the rows before s of the windows it
+    completes, from ((s // ratio) - coff + 1) * ratio on, only if it completes
+    one; it writes its tail rows, from ((e // ratio) - coff + 1) * ratio on. Arguments are host arrays (numpy or CPU
+    tensors). Returns a list of problems, empty when there are none."""
+    import numpy as np
+
+    def host(a):
+        return None if a is None else np.asarray(a.cpu() if hasattr(a, "cpu") else a)
+
+    kv, sc, cu = host(kv_block_table), host(state_block_table), host(cu_seqlens).astype(np.int64)
+    B = cu.shape[0] - 1
+    sp = np.zeros(B, dtype=np.int64) if start_pos is None else host(start_pos).astype(np.int64)
+    coff = 2 if ratio == 4 else 1
+    problems, owner = [], ({}, {})
+    for b in range(B):
+        s, e = int(sp[b]), int(sp[b]) + int(cu[b + 1] - cu[b])
+        if e == s:
+            continue
+        blocks = set()
+        w0 = s // ratio  # the first window the call can complete
+        if (w0 + 1) * ratio <= e:  # it does: its rows before s come from the state
+            read_lo = max(0, (w0 - coff + 1) * ratio)
+            if read_lo < s:
+                blocks.update(range(read_lo // block_size, (s - 1) // block_size + 1))
+        write_lo = max(s, (e // ratio - coff + 1) * ratio)  # the tail rows
+        if write_lo < e:
+            blocks.update(range(write_lo // block_size, (e - 1) // block_size + 1))
+        for which, table in enumerate((kv, sc)):
+            for blk in sorted(blocks):
+                if blk >= table.shape[1]:
+                    problems.append(f"sequence {b}: block {blk} is past the table's {table.shape[1]} columns")
+                    continue
+                row = int(table[b, blk])
+                if not 0 <= row < block_num:
+                    problems.append(f"sequence {b}: table entry [{b}][{blk}] = {row} is outside [0, {block_num})")
+                    continue
+                other = owner[which].setdefault(row, b)
+                if other != b:
+                    name = "kv" if which == 0 else "score"
+                    problems.append(f"{name} pool row {row} is used by sequences {other} and {b}")
+    return problems
+
+
 def get_error(stream=None) -> int:
     """Synchronise the stream and return (and clear) the device error status."""
     import torch
