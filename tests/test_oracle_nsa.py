@@ -7,6 +7,8 @@ import os
 
 import numpy as np
 import pytest
+from hypothesis import given, settings
+from hypothesis import strategies as st
 
 from oracle.nsa import half_to_f64, nsa_compress, nsa_compress_brute, to_f64, triggers
 from workloads import make_nsa_inputs
@@ -119,3 +121,27 @@ def test_paged_and_packed_layouts_agree():
                          i.output_cache, dtype=i.dtype, compress_block_size=32, compress_stride=32,
                          layout="TND")
     assert np.array_equal(r_paged.output_cache, r_tnd.output_cache)
+
+
+@settings(max_examples=20, deadline=None, derandomize=True)
+@given(dtype=st.sampled_from(["fp16", "bf16"]), layout=st.sampled_from(["paged", "TND"]),
+       cbs=st.sampled_from([16, 32, 48, 64]), stride=st.sampled_from([16, 32, 48, 64]),
+       pbs=st.sampled_from([64, 128]), B=st.integers(1, 4), N=st.integers(1, 3),
+       seed=st.integers(0, 10_000), frac=st.floats(0.0, 1.0))
+def test_brute_force_random(dtype, layout, cbs, stride, pbs, B, N, seed, frac):
+    """The definition and its pure-Python restatement agree exactly on random
+    small calls, including ones where no batch is on a compression step."""
+    if stride > cbs:
+        stride = cbs
+    i = make_nsa_inputs(name="rand", seed=seed, B=B, N=N, D=4, compress_block_size=cbs,
+                        compress_stride=stride, page_block_size=pbs, dtype=dtype, layout=layout,
+                        max_seq_len=192, trigger_fraction=frac)
+    r = call(i)
+    ref = nsa_compress_brute(i.input, i.weight, i.slot_mapping, i.act_seq_len, i.block_table,
+                             i.output_cache, dtype=dtype, compress_block_size=cbs,
+                             compress_stride=stride, page_block_size=pbs, layout=layout)
+    assert set(ref) == {(s, n, d) for s in np.nonzero(r.written)[0] for n in range(N) for d in range(4)}
+    for (s, n, d), v in ref.items():
+        assert r.sums[s, n, d] == v
+    # slots not written keep the cache's bits
+    assert np.array_equal(r.output_cache[~r.written], i.output_cache[~r.written])
