@@ -12,6 +12,8 @@ import os
 
 import numpy as np
 import pytest
+from hypothesis import assume, given, settings
+from hypothesis import strategies as st
 
 import oracle
 from oracle import brute
@@ -97,7 +99,23 @@ BRUTE_CASES = [
 
 @pytest.mark.parametrize("case", BRUTE_CASES)
 def test_oracle_matches_brute_force(case):
-    inp = tiny(**case)
+    _check_against_brute(tiny(**case))
+
+
+@settings(max_examples=20, deadline=None, derandomize=True)
+@given(lengths=st.lists(st.integers(0, 14), min_size=1, max_size=3), data=st.data(),
+       ratio=st.sampled_from([1, 2, 4, 8]), rotate=st.booleans(), bs=st.sampled_from([2, 4, 8]),
+       seed=st.integers(0, 1000))
+def test_oracle_matches_brute_force_random(lengths, data, ratio, rotate, bs, seed):
+    """Random tiny varlen calls (empty sequences, mid-window starts, every
+    ratio up to 8, with and without rotation): the numpy definition and the
+    pure-Python closed form agree."""
+    assume(sum(lengths) > 0)
+    start_pos = data.draw(st.lists(st.integers(0, 40), min_size=len(lengths), max_size=len(lengths)))
+    _check_against_brute(tiny(lengths, start_pos, ratio=ratio, rotate=rotate, bs=bs, seed=seed))
+
+
+def _check_against_brute(inp):
     res = run_inputs(inp)
     lay, (wins, kv_new, sc_new) = _brute(inp)
     assert len(wins) == len(lay.rows)
