@@ -69,6 +69,8 @@ class NsaResult:
     output_cache: np.ndarray   # uint16 bits, the whole cache after the call
     written: np.ndarray        # bool [result_len]: slots this call wrote
     sums: np.ndarray           # float64 [result_len, N, D] exact sums (NaN where not written)
+    abs_sums: np.ndarray       # float64 [result_len, N, D] exact sums of |product| (NaN where not
+                               # written): the scale of any finite-precision summation's error
 
 
 def nsa_compress(input_bits, weight_bits, slot_mapping, act_seq_len, block_table, output_cache_bits, *,
@@ -94,12 +96,14 @@ def nsa_compress(input_bits, weight_bits, slot_mapping, act_seq_len, block_table
     start = np.concatenate([[0], np.cumsum(lens)])  # TND row of each batch's first token
     written = np.zeros(result_len, dtype=bool)
     sums = np.full((result_len, N, D), np.nan)
+    abs_sums = np.full((result_len, N, D), np.nan)
     for b in range(B):
         s = int(lens[b])
         if not triggers(s, cbs, stride):
             continue
         idx = (s - cbs) // stride
         acc = np.zeros((N, D))
+        mag = np.zeros((N, D))
         for j in range(cbs):
             p = idx * stride + j
             if layout == "paged":
@@ -107,12 +111,15 @@ def nsa_compress(input_bits, weight_bits, slot_mapping, act_seq_len, block_table
                 tok = inp[blk, p % page_block_size]
             else:
                 tok = inp[int(start[b]) + p]
-            acc += to_f64(tok, dtype) * w[j][:, None]
+            prod = to_f64(tok, dtype) * w[j][:, None]
+            acc += prod
+            mag += np.abs(prod)
         slot = int(slots[b])
         out[slot] = to_bits(acc, dtype)
         sums[slot] = acc
+        abs_sums[slot] = mag
         written[slot] = True
-    return NsaResult(output_cache=out, written=written, sums=sums)
+    return NsaResult(output_cache=out, written=written, sums=sums, abs_sums=abs_sums)
 
 
 def nsa_compress_brute(input_bits, weight_bits, slot_mapping, act_seq_len, block_table,

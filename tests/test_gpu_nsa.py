@@ -47,20 +47,29 @@ def check(cmp, i):
     w = ref.written
     # slots not written: bit for bit the cache before the call
     assert np.array_equal(got[~w], i.output_cache[~w])
-    assert_within_one_unit(got[w], ref.output_cache[w], i.dtype)
+    assert_within_fp32_bound(got[w], ref.output_cache[w], ref.abs_sums[w], i.compress_block_size,
+                             i.dtype)
     return ref, got
 
 
-def assert_within_one_unit(got_bits, ref_bits, dtype):
-    """Written slots: the exact sum rounded once, within one unit of the dtype
-    (the library sums in fp32, so a sum next to a rounding boundary may round to
-    the other neighbour)."""
+def assert_within_fp32_bound(got_bits, ref_bits, abs_sums, cbs, dtype):
+    """Written slots against the exact sum rounded once to the dtype.
+
+    The page fixes fp32 products and an fp32 sum with one round-to-nearest-even
+    cast (计算公式 and the kernel description), not the order of the sum. A
+    product of two 16-bit values is exact in fp32, and a recursive fp32 sum of
+    n terms is within gamma_{n-1} * sum |term| of the exact one (gamma_k =
+    k u / (1 - k u), u = 2^-24). Each side's final cast adds at most half a unit
+    of the dtype, so |gpu - oracle| <= one unit + gamma_{n-1} * sum |term|."""
     g = to_f64(got_bits, dtype)
     e = to_f64(ref_bits, dtype)
-    mant = 10 if dtype == "fp16" else 7
+    mant, min_spacing = (10, 2.0 ** -24) if dtype == "fp16" else (7, 2.0 ** -133)
     mag = np.maximum(np.abs(e), np.abs(g))
-    ulp = np.exp2(np.floor(np.log2(np.maximum(mag, 1e-30))) - mant)
-    assert (np.abs(g - e) <= ulp + 1e-5).all()
+    ulp = np.maximum(np.exp2(np.floor(np.log2(np.maximum(mag, 1e-300))) - mant), min_spacing)
+    u = 2.0 ** -24
+    k = cbs - 1
+    gamma = k * u / (1 - k * u)
+    assert (np.abs(g - e) <= ulp + gamma * abs_sums).all()
 
 
 @pytest.mark.parametrize("dtype", ["bf16", "fp16"])
@@ -173,7 +182,7 @@ def test_packed_negative_length_is_reported(lib):
                        dtype=i.dtype, compress_block_size=32, compress_stride=16, layout="TND")
     s0 = i.slot_mapping[0]
     assert ref.written[s0]
-    assert_within_one_unit(got[s0], ref.output_cache[s0], i.dtype)
+    assert_within_fp32_bound(got[s0], ref.output_cache[s0], ref.abs_sums[s0], 32, i.dtype)
     for b in (2, 3):
         s = i.slot_mapping[b]
         assert np.array_equal(got[s], i.output_cache[s])

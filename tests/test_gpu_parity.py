@@ -59,7 +59,7 @@ def test_c4a_decode(lib, proj_kernel):
 
 
 @pytest.mark.slow
-def test_c128a_128k_prefill_sampled(lib):
+def test_c128a_128k_prefill(lib):
     inp = with_rope(make_config("c128a_128k"))
     args = to_device(inp)
     kv0 = args["kv_state"].clone()
@@ -68,9 +68,9 @@ def test_c128a_128k_prefill_sampled(lib):
     assert lib.get_error() == 0
     o = bits(out)
     assert o.shape == (1025, 512)
-    rows = [0, 1, 2, 127, 128, 511, 777, 1022, 1023, 1024]
-    res = run_inputs(inp, windows_only=rows)
-    assert_out_close(o, res, rows)
+    # every one of the 1025 rows against the oracle (a few seconds of CPU work)
+    res = run_inputs(inp)
+    assert_out_close(o, res)
     assert np.all(o[1024] == 0)
     # e = 131072 is window aligned: no tail, so no state byte may change
     import torch

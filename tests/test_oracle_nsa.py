@@ -59,6 +59,29 @@ def test_brute_force_tiny(dtype, layout, cbs, stride, pbs):
     assert r.written.sum() >= 1
 
 
+def test_abs_sums_bound_the_sums():
+    """The sums of |product| the GPU tolerance scales with: >= |sum| everywhere,
+    equal to the sum when every value is positive, and equal to the brute-force
+    sum of |input| * |weight| over the window."""
+    import dataclasses
+    i = make_nsa_inputs(name="abs", seed=31, B=6, N=3, D=4, compress_block_size=32,
+                        compress_stride=16, page_block_size=64, max_seq_len=200, trigger_fraction=1.0)
+    r = call(i)
+    w = r.written
+    assert w.sum() >= 1
+    assert (r.abs_sums[w] >= np.abs(r.sums[w])).all()
+    # |values|: clear the sign bits, then the sum is its own magnitude
+    pos = dataclasses.replace(i, input=i.input & np.uint16(0x7FFF), weight=i.weight & np.uint16(0x7FFF))
+    rp = call(pos)
+    assert np.array_equal(rp.abs_sums[w], rp.sums[w])
+    assert np.array_equal(rp.abs_sums[w], r.abs_sums[w])
+    ref = nsa_compress_brute(pos.input, pos.weight, pos.slot_mapping, pos.act_seq_len, pos.block_table,
+                             pos.output_cache, dtype="bf16", compress_block_size=32, compress_stride=16,
+                             page_block_size=64, layout="paged")
+    for (s, n, d), v in ref.items():
+        assert r.abs_sums[s, n, d] == v
+
+
 def test_trigger_rule_and_untouched_slots():
     cbs, stride = 32, 16
     lens = [0, 31, 32, 33, 47, 48, 64, 95, 96, 100]

@@ -15,8 +15,8 @@ SRC = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), 
 
 MUTATIONS = {
     "window one token early": ("p = idx * stride + j\n", "p = idx * stride + j - 1\n"),
-    "heads of the weight reversed": ("acc += to_f64(tok, dtype) * w[j][:, None]",
-                                     "acc += to_f64(tok, dtype) * w[j][::-1][:, None]"),
+    "heads of the weight reversed": ("prod = to_f64(tok, dtype) * w[j][:, None]",
+                                     "prod = to_f64(tok, dtype) * w[j][::-1][:, None]"),
     "trigger ignores the stride": (
         "return s >= compress_block_size and (s - compress_block_size) % stride == 0",
         "return s >= compress_block_size"),
