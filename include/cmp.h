@@ -180,9 +180,14 @@ CMP_API int cmp_compressor(const cmp_bf16* x, float* kv_state, float* score_stat
  * array's device address once (cudaGetSymbolAddress); make that first call
  * before any stream capture. All calls on a device share the array, so calls
  * that overlap on the GPU race and must be ordered by the caller (one stream,
- * or events). The array keeps the last call's contents; each call clears the
- * part that must start at zero. Device-side index errors of this variant are
- * not reported through cmp_get_error. */
+ * or events). The array keeps the last call's contents. Its error word starts
+ * at zero when the library is loaded, kernels only set bits in it, and
+ * cmp_get_error reads and clears it: device-side errors (a bad needed table
+ * entry, cu_seqlens or start_pos) are reported by cmp_get_error(stream) on the
+ * same device, once the calls' stream is synchronised (pass that stream).
+ * After a device reset (cudaDeviceReset), call cmp_release_workspaces before
+ * the next call: the array may move when the library image is loaded again,
+ * and that call makes the next one look its address up afresh. */
 CMP_API int cmp_compressor_noalloc(const cmp_bf16* x, float* kv_state, float* score_state,
                                    const int32_t* kv_block_table, const int32_t* state_block_table,
                                    const cmp_bf16* sin, const cmp_bf16* cos, const cmp_bf16* wkv,
@@ -193,7 +198,8 @@ CMP_API int cmp_compressor_noalloc(const cmp_bf16* x, float* kv_state, float* sc
 
 /* Synchronises stream, then returns and clears the error word the kernels of
  * the current device set: CMP_OK, CMP_ERR_DEVICE_INDEX or CMP_ERR_TIMEOUT
- * (CMP_ERR_CUDA if the synchronisation itself fails). */
+ * (CMP_ERR_CUDA if the synchronisation itself fails). Covers the calls made on
+ * `stream` and every cmp_compressor_noalloc call on the current device. */
 CMP_API int cmp_get_error(void* stream);
 
 /* Bytes of device workspace a call with these shapes uses (the two-phase
@@ -201,7 +207,8 @@ CMP_API int cmp_get_error(void* stream);
  * Returns 0 for invalid dims. Host only. */
 CMP_API size_t cmp_workspace_size(const cmp_dims* dims, int32_t ratio);
 
-/* Frees every workspace the library holds (synchronises the devices first).
+/* Frees every workspace the library holds (synchronises the devices first) and
+ * forgets the cached device addresses of cmp_compressor_noalloc's array.
  * Returns CMP_OK or CMP_ERR_CUDA. */
 CMP_API int cmp_release_workspaces(void);
 

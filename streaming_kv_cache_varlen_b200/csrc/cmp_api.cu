@@ -24,6 +24,8 @@ size_t decode_cp_workspace(const Params& p);
 cudaError_t launch_decode_cp(const Params& p, float* ss, void* counter, cudaStream_t s, bool unreachable);
 cudaError_t launch_nsa(const NsaParams& p, cudaStream_t s);
 cudaError_t launch_nsa_scan(const NsaParams& p, cudaStream_t s);
+int noalloc_take_error(int dev, unsigned* word);
+void noalloc_forget_addresses();
 }  // namespace cmp
 
 namespace {
@@ -364,6 +366,7 @@ int cmp_release_workspaces(void) {
   }
   g_ws.clear();
   cudaSetDevice(cur);
+  cmp::noalloc_forget_addresses();  // looked up again by the next allocation-free call
   return rc;
 }
 
@@ -519,6 +522,9 @@ int cmp_get_error(void* stream) {
       word |= v;
     }
   }
+  unsigned na = 0;  // the allocation-free entry point's calls on this device
+  if (cmp::noalloc_take_error(dev, &na) != CMP_OK) return CMP_ERR_CUDA;
+  word |= na;
   if (word & cmp::kErrTimeout) return CMP_ERR_TIMEOUT;
   if (word & cmp::kErrIndex) return CMP_ERR_DEVICE_INDEX;
   return CMP_OK;

@@ -18,8 +18,13 @@
 // cudaGetSymbolAddress and cached; make that first call before any stream
 // capture. Every call on a device shares the array: calls that overlap on the
 // GPU (two streams at once) race on it and must be ordered by the caller. The
-// array keeps the last call's contents; the only part that must start at zero
-// (the error word) is cleared by each call with an asynchronous memset.
+// array keeps the last call's contents. The only part that must start at zero
+// is the error word at its start: it is zero when the library is loaded, the
+// kernels only ever set bits in it, and cmp_get_error reads and clears it, so
+// device-side errors of these calls are reported like those of cmp_compressor.
+// A device reset (cudaDeviceReset) unloads the library image from the device and
+// may move the array when it is loaded again: cmp_release_workspaces forgets
+// the cached addresses, so the next call looks the address up afresh.
 #include <mutex>
 
 #include "cmp_internal.cuh"
@@ -27,6 +32,8 @@
 namespace cmp {
 cudaError_t launch_proj_decode(const Params& p, cudaStream_t s);
 bool proj_decode_supported(const Params& p);
+int noalloc_take_error(int dev, unsigned* word);
+void noalloc_forget_addresses();
 }  // namespace cmp
 
 namespace {
@@ -48,7 +55,7 @@ ScratchLayout scratch_layout(int64_t B, int64_t T, int64_t C) {
     o += (n + 255) & ~size_t(255);
     return r;
   };
-  L.err = take(16);
+  L.err = take(16);  // offset 0: the error word (cmp::noalloc_take_error reads it there)
   L.m_cu = take(sizeof(int32_t) * (B + 1));
   L.m_s = take(sizeof(int32_t) * (B > 0 ? B : 1));
   L.m_off = take(sizeof(int32_t) * (B + 1));
@@ -81,6 +88,30 @@ bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) %
 
 }  // namespace
 
+namespace cmp {
+
+// The error word of this entry point's calls on device `dev` (current), read
+// and cleared; 0 if no call has run on that device. The caller has synchronised
+// the stream the calls ran on.
+int noalloc_take_error(int dev, unsigned* word) {
+  *word = 0;
+  if (dev < 0 || dev >= 64) return CMP_OK;
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (!g_addr[dev]) return CMP_OK;
+  unsigned v = 0;
+  if (cudaMemcpy(&v, g_addr[dev], sizeof(v), cudaMemcpyDeviceToHost) != cudaSuccess) return CMP_ERR_CUDA;
+  if (v && cudaMemset(g_addr[dev], 0, sizeof(v)) != cudaSuccess) return CMP_ERR_CUDA;
+  *word = v;
+  return CMP_OK;
+}
+
+void noalloc_forget_addresses() {
+  std::lock_guard<std::mutex> lk(g_mu);
+  for (auto& a : g_addr) a = nullptr;
+}
+
+}  // namespace cmp
+
 extern "C" int cmp_compressor_noalloc(const cmp_bf16* x, float* kv_state, float* score_state,
                                       const int32_t* kv_block_table, const int32_t* state_block_table,
                                       const cmp_bf16* sin, const cmp_bf16* cos, const cmp_bf16* wkv,
@@ -106,7 +137,9 @@ extern "C" int cmp_compressor_noalloc(const cmp_bf16* x, float* kv_state, float*
     return CMP_ERR_NULLPTR;
   if (!aligned(x, 16) || !aligned(wkv, 16) || !aligned(wgate, 16) || !aligned(kv_state, 16) ||
       !aligned(score_state, 16) || !aligned(ape, 16) || !aligned(out, 8) || !aligned(norm_weight, 8) ||
-      !aligned(sin, 4) || !aligned(cos, 4) || (rotate && !aligned(hadamard, 8)))
+      !aligned(sin, 4) || !aligned(cos, 4) || (rotate && !aligned(hadamard, 8)) ||
+      !aligned(kv_block_table, 4) || !aligned(state_block_table, 4) || !aligned(cu_seqlens, 4) ||
+      (start_pos && !aligned(start_pos, 4)))
     return CMP_ERR_INVALID;
 
   cmp::Params p{};
@@ -150,7 +183,6 @@ extern "C" int cmp_compressor_noalloc(const cmp_bf16* x, float* kv_state, float*
   p.proj = reinterpret_cast<float*>(ws + L.proj);
 
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (cudaMemsetAsync(p.err, 0, sizeof(unsigned), s) != cudaSuccess) return CMP_ERR_CUDA;
   if (cmp::launch_sched(p, s) != cudaSuccess) return CMP_ERR_CUDA;
   if (cmp::launch_proj_decode(p, s) != cudaSuccess) return CMP_ERR_CUDA;
   if (cmp::launch_pool(p, s) != cudaSuccess) return CMP_ERR_CUDA;

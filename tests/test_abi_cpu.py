@@ -109,6 +109,37 @@ def test_host_checks_reject_before_launch(cmp):
     assert _call(cmp, D(**ok), ptr=0x10002) == 2                      # misaligned pointers
 
 
+def _noalloc(cmp, dims, ptrs=None, ptr=0x10000):
+    args = [ptr] * 14 if ptrs is None else ptrs
+    return cmp.lib.cmp_compressor_noalloc(*args, 4, 64, False, ptr, None, ctypes.byref(dims))
+
+
+def test_noalloc_host_checks_reject_before_launch(cmp):
+    """The allocation-free entry point makes the regular call's host checks,
+    the 4-byte alignment of the int32 tables and start_pos included, and rejects
+    calls whose scratch would not fit its fixed 1 MiB array."""
+    D = cmp.cmp_dims
+    ok = dict(B=2, T=10, H=1024, D=512, block_num=4, block_size=128, table_stride=2)
+    names = ["x", "kv_state", "score_state", "kv_block_table", "state_block_table", "sin", "cos",
+             "wkv", "wgate", "ape", "norm_weight", "hadamard", "start_pos", "cu_seqlens"]
+    for name in ("kv_block_table", "state_block_table", "start_pos", "cu_seqlens"):
+        ptrs = [0x10000] * 14
+        ptrs[names.index(name)] = 0x10001      # misaligned int32 array
+        assert _noalloc(cmp, D(**ok), ptrs) == 2, name
+    for name in ("x", "wkv", "kv_state"):
+        ptrs = [0x10000] * 14
+        ptrs[names.index(name)] = 0x10008      # 8 but not 16-byte aligned
+        assert _noalloc(cmp, D(**ok), ptrs) == 2, name
+    # 64 tokens of 2 x 1024 fp32 projection columns take 512 KiB; the three
+    # per-sequence int32 arrays share the rest. 43647 sequences fit, 43648 do not.
+    full = dict(ok, T=64, H=4096, D=512)
+    assert _noalloc(cmp, D(**dict(full, B=43648))) == 2
+    assert _noalloc(cmp, D(**dict(full, T=65))) == 2     # beyond the 64-token limit
+    ptrs = [0x10000] * 14
+    ptrs[names.index("cu_seqlens")] = 0x10002
+    assert _noalloc(cmp, D(**dict(full, B=43647)), ptrs) == 2  # fits; rejected by the alignment
+
+
 def test_empty_calls_are_noops(cmp):
     D = cmp.cmp_dims
     # nothing to do: OK without touching any pointer (all NULL here)
