@@ -330,10 +330,30 @@ def bench_configs(args, ws, local, peaks, peak_src):
         del g
         tf = flops / (us / 1e6) / 1e12
         res[name] = {"calls_per_step": len(calls), "tokens_per_step": int(sum(c.T for c in calls)),
-                     "us_per_step": us, "tflops": tf, "frac_of_bf16_burst": tf / peaks["bf16_tflops"]}
+                     "us_per_step": us, "tflops": tf, "frac_of_bf16_burst": tf / peaks["bf16_tflops"],
+                     "kernel_us": kernel_times(step, side, steps=5)}
         del steps_args, outs
         torch.cuda.empty_cache()
     return res
+
+
+def kernel_times(step, stream, steps: int):
+    """Per-kernel device time of `step`: the library's CUDA events around each of
+    its launches (cmp_profile_start/stop) over `steps` eager steps. The steps are
+    queued behind a ~10 ms sleep kernel so that the host has enqueued them all
+    before the first one runs (launch overhead does not show up between a
+    kernel's events). Returns {kernel: {"us": mean per launch, "launches_per_step": n}}."""
+    import torch
+
+    import streaming_kv_cache_varlen_b200 as cmp
+
+    with torch.cuda.stream(stream):
+        torch.cuda._sleep(20_000_000)
+        cmp.profile_start()
+        for _ in range(steps):
+            step()
+        prof = cmp.profile_stop()
+    return {k: {"us": ms / n * 1e3, "launches_per_step": n / steps} for k, (ms, n) in prof.items() if n}
 
 
 def decode_inputs(device):
@@ -708,6 +728,140 @@ def run_ours(args):
         dist.destroy_process_group()
 
 
+class _Marks:
+    """Time stamps on the device (CUDA events on the current stream) or, on CPU,
+    host clock readings; spans_ms() gives the times between consecutive marks."""
+
+    def __init__(self, cuda: bool):
+        self.cuda = cuda
+        self.m = []
+
+    def mark(self):
+        if self.cuda:
+            import torch
+            e = torch.cuda.Event(enable_timing=True)
+            e.record()
+            self.m.append(e)
+        else:
+            self.m.append(time.perf_counter())
+
+    def spans_ms(self):
+        if self.cuda:
+            import torch
+            torch.cuda.synchronize()
+            return [a.elapsed_time(b) for a, b in zip(self.m, self.m[1:])]
+        return [(b - a) * 1e3 for a, b in zip(self.m, self.m[1:])]
+
+
+def sharded_inputs(device, T: int, H: int, D: int, ratio: int, seed: int):
+    """One sequence of T tokens from position 0, drawn with a seeded torch
+    generator on `device` (identical on every rank): x ~ N(0,1), weights
+    N(0, 1/H), ape N(0, 0.1), norm_weight 1 + N(0, 0.05), and the sin/cos rows of
+    its windows (position w * ratio)."""
+    import numpy as np
+    import torch
+
+    from streaming_kv_cache_varlen_b200 import sharded
+    from workloads import rope_tables
+
+    coff = 2 if ratio == 4 else 1
+    C = coff * D
+    g = torch.Generator(device=device)
+    g.manual_seed(seed)
+    bf = torch.bfloat16
+    x = torch.randn(T, H, generator=g, device=device).to(bf)
+    wkv = (torch.randn(C, H, generator=g, device=device) / H ** 0.5).to(bf)
+    wgate = (torch.randn(C, H, generator=g, device=device) / H ** 0.5).to(bf)
+    ape = torch.randn(ratio, C, generator=g, device=device) * 0.1 ** 0.5
+    norm_w = (1 + torch.randn(D, generator=g, device=device) * 0.05 ** 0.5).to(bf)
+    n_out = sharded.n_out_rows(T, ratio)
+    pos = np.where(np.arange(n_out) < T // ratio, np.arange(n_out) * ratio, 0)
+    cos, sin = rope_tables(pos, 64)
+    to = lambda a: torch.from_numpy(a.view(np.int16)).to(device).view(bf)
+    return dict(x=x, wkv=wkv, wgate=wgate, ape=ape, norm_weight=norm_w, hadamard=None, sin=to(sin),
+                cos=to(cos))
+
+
+def bench_sharded(args, ws: int, rank: int, device, *, T: int, H: int, D: int, ratio: int,
+                  block_size: int = 128, run_call=None):
+    """One long prefill split across the ranks by tokens (the library's sharded
+    prefill: per-rank calls on window-aligned slices with a halo, then one
+    all-gather of the output rows). Per step: this rank's call (with its scratch
+    state) and the all-gather, timed separately; the step time is the max over
+    ranks. Returns (the JSON line's fields, the assembled output of the last step)."""
+    import torch
+
+    from streaming_kv_cache_varlen_b200 import sharded
+
+    cuda = device.type == "cuda"
+    inp = sharded_inputs(device, T, H, D, ratio, seed=1234)
+    shards = sharded.plan(T, ratio, ws)
+    me = shards[rank]
+    C = inp["wkv"].shape[0]
+    if run_call is None:
+        from streaming_kv_cache_varlen_b200 import compressor as run_call
+
+    def step(marks):
+        marks.mark()
+        loc = sharded.local_inputs(me, inp["x"], inp["sin"], inp["cos"], ratio, block_size, C)
+        out_loc = run_call(wkv=inp["wkv"], wgate=inp["wgate"], ape=inp["ape"],
+                           norm_weight=inp["norm_weight"], hadamard=None, ratio=ratio, rope_head_dim=64,
+                           rotate=False, **loc)
+        mine = sharded.own_rows(me, out_loc)
+        marks.mark()
+        rows = sharded.all_gather_rows(shards, mine) if ws > 1 else [mine]
+        out = sharded.assemble(shards, rows, T, ratio, mine)
+        marks.mark()
+        return out
+
+    for _ in range(args.warmup):
+        step(_Marks(cuda))
+    if cuda:
+        torch.cuda.synchronize()
+    barrier(ws)
+    if cuda:
+        torch.cuda.synchronize()
+    marks = _Marks(cuda)
+    for _ in range(args.steps):
+        out = step(marks)
+    spans = marks.spans_ms()
+    barrier(ws)
+    compute = sum(spans[0::3])     # call spans; spans[1::3] all-gather; spans[2::3] between steps
+    gather = sum(spans[1::3])
+    total = sum(spans)
+    total_max = max_over_ranks(total, ws)
+    line = {"metric": METRIC, "value": T * args.steps / (total_max / 1e3), "unit": "tokens/s",
+            "n_gpus": ws, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": total_max / args.steps, "higher_is_better": True, "scaling": "strong",
+            "vs_baseline": None, "dtype": "bf16 in, fp32 accumulate / state, bf16 out",
+            "data": "synthetic",
+            "config": {"workload": f"one sequence x {T} tokens, H={H}, D={D}, ratio={ratio}, "
+                                   f"block_size={block_size}",
+                       "global_batch": 1, "seq_len": T,
+                       "parallelism": f"cp{ws} (token-sharded prefill, one all-gather of the output rows)"},
+            "sharded": {"compute_ms_per_step_max": max_over_ranks(compute, ws) / args.steps,
+                        "gather_ms_per_step_max": max_over_ranks(gather, ws) / args.steps,
+                        "windows_per_rank": [s.n_windows for s in shards],
+                        "backend": "nccl" if cuda else "gloo"}}
+    return line, out
+
+
+def run_sharded(args):
+    """--mode sharded: the token-sharded 128K prefill under torchrun (NCCL)."""
+    import torch
+
+    ws, rank, local = dist_setup()
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    line, _ = bench_sharded(args, ws, rank, device, T=args.prefill_tokens, H=PREFILL["H"],
+                            D=PREFILL["D"], ratio=PREFILL["ratio"], block_size=PREFILL["block_size"])
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if ws > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
 def cpu_baseline(tokens: int):
     """The oracle, as it is, on the first ``tokens`` tokens of the prefill workload
     (drawn on the host with the workload generator), on this host's cores."""
@@ -783,6 +937,9 @@ def main():
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--mode", choices=("replicas", "sharded"), default="replicas",
+                    help="replicas: every rank runs its own copy of the workload (the default); "
+                         "sharded: one 128K prefill split across the ranks by tokens")
     ap.add_argument("--cpu-tokens", type=int, default=None,
                     help="tokens of the CPU-baseline sample (default: about --cpu-seconds of oracle work)")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
@@ -797,6 +954,8 @@ def main():
     PREFILL["T"] = args.prefill_tokens
     if args.impl == "reference":
         run_reference(args)
+    elif args.mode == "sharded":
+        run_sharded(args)
     else:
         run_ours(args)
 

@@ -181,3 +181,65 @@ def test_two_gloo_ranks_gather_the_one_shot_rows(ratio, T):
     for r in range(ws):
         got = np.frombuffer(res[r], dtype=np.uint16).reshape(ref.shape)
         assert np.array_equal(got, ref), f"rank {r}"
+
+
+def oracle_call_bf16(**kw):
+    """oracle_call for bf16 tensors (bench.py's inputs) instead of int16 bits."""
+    kw = {k: (v.view(torch.int16) if isinstance(v, torch.Tensor) and v.dtype == torch.bfloat16 else v)
+          for k, v in kw.items()}
+    return oracle_call(**kw).view(torch.bfloat16)
+
+
+def _bench_worker(rank, ws, port, out):
+    import datetime
+    import types
+
+    import torch.distributed as dist
+
+    import bench
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=ws, timeout=datetime.timedelta(seconds=120))
+    try:
+        args = types.SimpleNamespace(steps=2, warmup=1)
+        line, got = bench.bench_sharded(args, ws, rank, torch.device("cpu"), T=600, H=512, D=128,
+                                        ratio=4, block_size=32, run_call=oracle_call_bf16)
+        out[rank] = (line, got.view(torch.int16).numpy().copy())
+    finally:
+        dist.destroy_process_group()
+
+
+def test_bench_sharded_mode_two_gloo_ranks():
+    """bench.py --mode sharded's step on two gloo ranks with the oracle as the
+    per-rank call: both ranks assemble the one-shot oracle's output exactly, and
+    the line carries the contract's keys with strong scaling."""
+    ws = 2
+    ctx = mp.get_context("spawn")
+    with ctx.Manager() as m:
+        out = m.dict()
+        mp.start_processes(_bench_worker, args=(ws, _free_port(), out), nprocs=ws, join=True,
+                           start_method="spawn")
+        res = dict(out)
+    import bench
+    from oracle import run_inputs
+    from workloads import Inputs
+
+    inp = bench.sharded_inputs(torch.device("cpu"), 600, 512, 128, 4, seed=1234)
+    b = lambda t: t.view(torch.int16).numpy().view(np.uint16)
+    one = Inputs(name="shard_bench", ratio=4, coff=2, D=128, rope_head_dim=64, rotate=False, block_size=32,
+                 x=b(inp["x"]), wkv=b(inp["wkv"]), wgate=b(inp["wgate"]), ape=inp["ape"].numpy(),
+                 norm_weight=b(inp["norm_weight"]), hadamard=None,
+                 start_pos=np.zeros(1, np.int32), cu_seqlens=np.array([0, 600], np.int32),
+                 kv_state=np.zeros((19, 32, 256), np.float32), score_state=np.zeros((19, 32, 256), np.float32),
+                 kv_block_table=np.arange(19, dtype=np.int32)[None], state_block_table=np.arange(19, dtype=np.int32)[None],
+                 sin=b(inp["sin"]), cos=b(inp["cos"]))
+    ref = run_inputs(one).out
+    for rank in range(ws):
+        line, got = res[rank]
+        assert np.array_equal(got.view(np.uint16), ref), rank
+    line = res[0][0]
+    for k in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better",
+              "scaling", "config", "sharded"):
+        assert k in line, k
+    assert line["scaling"] == "strong" and line["n_gpus"] == 2 and line["value"] > 0
+    assert line["sharded"]["windows_per_rank"] == [75, 75]
+    assert res[0][0]["ms_per_step"] == res[1][0]["ms_per_step"]   # max over ranks
