@@ -678,6 +678,53 @@ def bench_nsa(args, ws, local, peaks, peak_src):
                          "traffic": traffic_for("cmp_nsa.cu", "nsa_compress"), "peak_source": peak_src}}
 
 
+PHASE_NAMES = ("entry", "setup_done", "first_stage", "last_mma", "metadata", "acc_complete",
+               "partials_sent", "partials_received", "pooled", "barrier_arrival", "tails_written",
+               "barrier_released", "rms_scales", "end")
+
+
+def run_decode_phases(args):
+    """--only decode-phases: the C4A 32-request decode call run through the
+    phase-stamp build of the library (built beside the normal one if missing),
+    cold (256 MB L2 flush before the call) and warm (the same call again). Per
+    phase, min / median / max over the CTAs of the time since the earliest
+    CTA's entry, in microseconds, medians over `steps` calls of each kind."""
+    import numpy as np
+
+    sys.path.insert(0, os.path.join(ROOT, "streaming_kv_cache_varlen_b200"))
+    import _build
+    os.environ["CMP_LIBRARY"] = _build.build(phases=True)
+    import torch
+
+    import streaming_kv_cache_varlen_b200 as cmp
+    assert cmp.LIB_PATH == os.environ["CMP_LIBRARY"]
+
+    device = torch.device("cuda", 0)
+    dec, _, inp = decode_inputs(device)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=device)
+    dout = torch.empty((cmp.out_rows(inp.B, inp.T, inp.ratio), inp.D), dtype=torch.bfloat16, device=device)
+    n_ctas = (inp.D // 16) * 4
+    res = {}
+    for kind in ("cold", "warm"):
+        runs = []
+        for i in range(args.warmup + args.steps):
+            if kind == "cold":
+                flush.fill_(1)
+            torch.cuda.synchronize()
+            cmp.compressor(**dec, out=dout)
+            st = cmp.debug_phase_stamps(n_ctas).astype(np.int64)
+            assert cmp.get_error() == 0
+            if i >= args.warmup:
+                runs.append((st - st[:, 0].min()) / 1e3)
+        a = np.stack(runs)   # [runs, ctas, 16]
+        res[kind] = {name: {"min": float(np.median(a[:, :, k].min(axis=1))),
+                            "median": float(np.median(np.median(a[:, :, k], axis=1))),
+                            "max": float(np.median(a[:, :, k].max(axis=1)))}
+                     for k, name in enumerate(PHASE_NAMES)}
+    print(json.dumps({"decode_phases_us": res, "ctas": n_ctas, "calls_per_kind": args.steps,
+                      "workload": "c4a_decode: 32 requests x 1 token, H=4096, D=512, ratio 4"}), flush=True)
+
+
 def run_ours(args):
     import torch
 
@@ -944,8 +991,10 @@ def main():
                     help="tokens of the CPU-baseline sample (default: about --cpu-seconds of oracle work)")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--only", choices=("all", "prefill", "decode", "nsa", "configs"), default="all",
-                    help="run only one part (for profiler captures)")
+    ap.add_argument("--only", choices=("all", "prefill", "decode", "nsa", "configs", "decode-phases"),
+                    default="all",
+                    help="run only one part (for profiler captures); decode-phases: the decode "
+                         "kernel's timeline from the phase-stamp build of the library")
     ap.add_argument("--prefill-tokens", type=int, default=PREFILL["T"],
                     help="tokens of the prefill sequence (smaller cases for profiler captures)")
     args = ap.parse_args()
@@ -954,6 +1003,8 @@ def main():
     PREFILL["T"] = args.prefill_tokens
     if args.impl == "reference":
         run_reference(args)
+    elif args.only == "decode-phases":
+        run_decode_phases(args)
     elif args.mode == "sharded":
         run_sharded(args)
     else:

@@ -299,6 +299,18 @@ CMP_API int cmp_profile_start(void);
  * launches[CMP_KERNEL_COUNT] (host arrays; either may be NULL). */
 CMP_API int cmp_profile_stop(double* ms, int64_t* launches);
 
+/* Measurement hook of a library built with -DCMP_PHASE_STAMPS (bench.py
+ * --only decode-phases builds one beside the normal library and runs it): the
+ * channel-group decode kernel writes the global timer (ns) at 14 points of its
+ * timeline; this copies those of its last launch, CTA i's phase k at
+ * dst[i * 16 + k] for the first n entries (host array, n <= 512 * 16), after
+ * synchronising the device. Phases: 0 entry, 1 set-up done, 2 first weight
+ * stage landed, 3 last MMA issued, 4 metadata done, 5 accumulator complete,
+ * 6 partials sent, 7 partials received, 8 pooled, 9 grid-barrier arrival,
+ * 10 tails written, 11 barrier released, 12 RMSNorm scales, 13 end. Other
+ * builds return CMP_ERR_UNSUPPORTED. */
+CMP_API int cmp_debug_phase_stamps(uint64_t* dst, int64_t n);
+
 /* Testing knob: which path calls take. 0 = automatic (for T <= 64 the
  * channel-group decode kernel, or without it (rotate, or a device that cannot
  * hold its clusters) the weight-streaming projection + pooling kernels, else

@@ -14,7 +14,9 @@ import os
 from typing import Dict, Optional, Tuple
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_PKG, "libcmp_b200.so")
+# CMP_LIBRARY selects another build of the same library (the phase-stamp
+# measurement build libcmp_b200_phases.so); by default the one next to this file
+LIB_PATH = os.environ.get("CMP_LIBRARY") or os.path.join(_PKG, "libcmp_b200.so")
 
 CMP_OK = 0
 STATUS = {0: "CMP_OK", 1: "CMP_ERR_NULLPTR", 2: "CMP_ERR_INVALID", 3: "CMP_ERR_UNSUPPORTED",
@@ -55,6 +57,7 @@ def _load() -> ctypes.CDLL:
         "cmp_compressor_noalloc": (ctypes.c_int, [P] * 14 + [I32, I32, ctypes.c_bool, P, P,
                                                            ctypes.POINTER(cmp_dims)]),
         "cmp_get_error": (ctypes.c_int, [P]),
+        "cmp_debug_phase_stamps": (ctypes.c_int, [P, I64]),
         "cmp_workspace_size": (SZ, [ctypes.POINTER(cmp_dims), I32]),
         "cmp_release_workspaces": (ctypes.c_int, []),
         "cmp_status_string": (ctypes.c_char_p, [ctypes.c_int]),
@@ -339,3 +342,16 @@ def set_proj_kernel(which: int) -> int:
     2 tcgen05 projection, 3 weight streaming, 4 fused tcgen05 pooling, 5 K-split
     one-kernel decode, 6 channel-group one-kernel decode. Returns the previous value."""
     return int(lib.cmp_set_proj_kernel(which))
+
+
+def debug_phase_stamps(n_ctas: int):
+    """The channel-group decode kernel's phase stamps of its last launch, as a
+    numpy uint64 array [n_ctas, 16] (global timer, ns). Only the phase-stamp
+    measurement build (CMP_LIBRARY=.../libcmp_b200_phases.so) records them;
+    other builds raise CmpError(CMP_ERR_UNSUPPORTED)."""
+    import numpy as np
+    buf = np.zeros((n_ctas, 16), dtype=np.uint64)
+    st = lib.cmp_debug_phase_stamps(buf.ctypes.data, buf.size)
+    if st != CMP_OK:
+        raise CmpError(st, "cmp_debug_phase_stamps")
+    return buf

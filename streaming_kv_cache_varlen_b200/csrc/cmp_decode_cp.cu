@@ -46,6 +46,24 @@ namespace {
 
 using namespace sm100;
 
+// Phase stamps (a measurement build only, compiled with -DCMP_PHASE_STAMPS):
+// CTA i writes the global timer at phase k to slot i * kStampSlots + k of a
+// device array that cmp_debug_phase_stamps copies out. The normal build has no
+// stamps and no array.
+constexpr int kStampSlots = 16;
+constexpr int kStampCtas = 512;
+#ifdef CMP_PHASE_STAMPS
+__device__ unsigned long long g_cp_stamps[kStampCtas * kStampSlots];
+#define CP_STAMP(cond, k)                                                           \
+  do {                                                                              \
+    if ((cond) && blockIdx.x < kStampCtas) g_cp_stamps[blockIdx.x * kStampSlots + (k)] = globaltimer(); \
+  } while (0)
+#else
+#define CP_STAMP(cond, k) \
+  do {                    \
+  } while (0)
+#endif
+
 constexpr int KQ = 4;             // CTAs per cluster: they split the hidden dimension
 constexpr int GCH = 16;           // channels per cluster
 constexpr int OWN = GCH / KQ;     // channels per CTA after the reduction
@@ -551,6 +569,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   // after the MMAs: the outgoing partials, one block per owner CTA [owner][kind][token][channel]
   float* part = reinterpret_cast<float*>(&sm.a[0][0]);
   const int blk_floats = kinds * p.T * OWN;
+  CP_STAMP(threadIdx.x == 0, 0);  // entry
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -573,6 +592,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = sm.tmem_base;
   volatile int* abort = &sm.abort;
+  CP_STAMP(threadIdx.x == 0, 1);  // set-up done
 
   // ---- 1) stream + MMA (lane 0 of warps 0, 1) / metadata and prefetch (warps 2, 3) ----
   // the metadata's first loads go out before the weight stream (named barrier 3)
@@ -597,6 +617,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool ok = true;
     for (int st = 0; st < nsteps; ++st) {
       if (!mbar_wait(&sm.full[stage], phase, abort)) { ok = false; break; }
+      CP_STAMP(st == 0, 2);  // first stage landed
       tc_fence_after();
 #pragma unroll
       for (int kk = 0; kk < KPS; ++kk) {
@@ -612,18 +633,21 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (++stage == STAGES) { stage = 0; phase ^= 1u; }
     }
     if (ok) mma_commit(&sm.acc_full);
+    CP_STAMP(true, 3);  // last MMA issued
   } else if (warp >= 2) {
     // the grid barrier's target, read here rather than before the stream starts
     // (a cold global load); any time before this CTA's own arrival is correct:
     // the count cannot reach the next multiple while this CTA's share is missing
     if (threadIdx.x == 64) sm.bar_target = grid_target(a.counter) + a.bar_extra;
     call_metadata<MAXT>(p, sm, NT, ch0);
+    CP_STAMP(threadIdx.x == 64, 4);  // metadata and prefetch done
   }
 
   // ---- 2) warps 0-1: TMEM rows -> the owners' blocks, one bulk copy per owner;
   // every CTA then adds the four blocks it received (in rank order) ----
   if (warp < 2) {
     const bool have = mbar_wait(&sm.acc_full, 0, abort);
+    CP_STAMP(threadIdx.x == 0, 5);  // accumulator complete
     __syncwarp();
     if (__all_sync(0xffffffffu, have) && warp * 32 < kinds * GCH) {
       tc_fence_after();
@@ -650,6 +674,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         bulk_copy_to_peer(peer_addr(&sm.recv[q][0], (uint32_t)o), part + o * blk_floats, bytes,
                           peer_addr(&sm.recv_full, (uint32_t)o));
       bulk_commit();
+      CP_STAMP(true, 6);  // partial blocks sent
     }
   }
   if (threadIdx.x == 0) {
@@ -657,6 +682,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // must land before it goes on (and, at the latest, before it exits)
     int never = 0;
     if (!mbar_wait(&sm.recv_full, 0, &never)) atomicOr(p.err, kErrTimeout);
+    CP_STAMP(true, 7);  // the four partial blocks landed
   }
   __syncthreads();  // the partials have landed, and the metadata is complete
   const bool mm_ok = !*abort;
@@ -709,6 +735,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   }
   __syncthreads();
+  CP_STAMP(threadIdx.x == 0, 8);  // pooled
   const int n_cta = gridDim.x;
   const int64_t rep_stride = (int64_t)n_out * n_cta;
   for (int i = threadIdx.x; i < nw * kReplicas; i += kThreads) {
@@ -719,6 +746,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   __syncthreads();
   if (threadIdx.x == 0) grid_arrive(a.counter, n_cta);
+  CP_STAMP(threadIdx.x == 0, 9);  // arrived at the grid barrier
 
   // ---- while the other CTAs arrive: state tails and rows without a window ----
   for (int i = threadIdx.x; i < kinds * p.T && mm_ok; i += kThreads) {
@@ -735,7 +763,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   for (int n = threadIdx.x; n < n_out; n += kThreads)
     if (sm.win[n].w < 0) *reinterpret_cast<uint2*>(p.out + (int64_t)n * p.D + ch0) = make_uint2(0u, 0u);
+  CP_STAMP(threadIdx.x == 0, 10);  // tails written
   if (threadIdx.x == 0) sm.grid_ok = grid_wait(a.counter, sm.bar_target, p.err) ? 1 : 0;
+  CP_STAMP(threadIdx.x == 0, 11);  // grid barrier released
   __syncthreads();
   const bool ok = sm.grid_ok != 0 && mm_ok;
 
@@ -767,6 +797,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   }
   __syncthreads();
+  CP_STAMP(threadIdx.x == 0, 12);  // RMSNorm scales summed
   const bool roped = ch0 >= p.D - p.rope;
   for (int wi = threadIdx.x; wi < nw; wi += kThreads) {
     const int n = sm.wlist[wi];
@@ -800,6 +831,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     tmem_dealloc(tmem, tmem_cols);
   }
   if (threadIdx.x == 0 && sm.abort) atomicOr(p.err, kErrTimeout);
+  CP_STAMP(threadIdx.x == 0, 13);  // end
 }
 
 // x [T, H] as (column in block, row, 64-column block): a box of 64 columns x
@@ -947,3 +979,18 @@ cudaError_t launch_decode_cp(const Params& p, float* ss, void* counter, cudaStre
 }
 
 }  // namespace cmp
+
+// Measurement hook: the phase stamps of the last channel-group decode launch
+// (a -DCMP_PHASE_STAMPS build only; other builds return CMP_ERR_UNSUPPORTED).
+extern "C" int cmp_debug_phase_stamps(uint64_t* dst, int64_t n) {
+#ifdef CMP_PHASE_STAMPS
+  if (!dst || n < 0 || n > (int64_t)cmp::kStampCtas * cmp::kStampSlots) return CMP_ERR_INVALID;
+  if (cudaDeviceSynchronize() != cudaSuccess) return CMP_ERR_CUDA;
+  return cudaMemcpyFromSymbol(dst, cmp::g_cp_stamps, sizeof(uint64_t) * (size_t)n) == cudaSuccess ? CMP_OK
+                                                                                                   : CMP_ERR_CUDA;
+#else
+  (void)dst;
+  (void)n;
+  return CMP_ERR_UNSUPPORTED;
+#endif
+}
