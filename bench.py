@@ -678,9 +678,10 @@ def bench_nsa(args, ws, local, peaks, peak_src):
                          "traffic": traffic_for("cmp_nsa.cu", "nsa_compress"), "peak_source": peak_src}}
 
 
-PHASE_NAMES = ("entry", "setup_done", "first_stage", "last_mma", "metadata", "acc_complete",
-               "partials_sent", "partials_received", "pooled", "barrier_arrival", "tails_written",
-               "barrier_released", "rms_scales", "end")
+PHASE_NAMES = ("entry", "setup_done", "first_stage", "last_mma", "metadata", "partials_sent",
+               "partials_received", "pooled_arrived", "-", "exchange_done", "rows_stored",
+               "all_arrived", "-", "-", "tails_written", "end",
+               "meta_wave1", "meta_windows", "meta_wave2", "meta_wave3")
 
 
 def run_decode_phases(args):
@@ -720,7 +721,7 @@ def run_decode_phases(args):
         res[kind] = {name: {"min": float(np.median(a[:, :, k].min(axis=1))),
                             "median": float(np.median(np.median(a[:, :, k], axis=1))),
                             "max": float(np.median(a[:, :, k].max(axis=1)))}
-                     for k, name in enumerate(PHASE_NAMES)}
+                     for k, name in enumerate(PHASE_NAMES) if name != "-"}
     print(json.dumps({"decode_phases_us": res, "ctas": n_ctas, "calls_per_kind": args.steps,
                       "workload": "c4a_decode: 32 requests x 1 token, H=4096, D=512, ratio 4"}), flush=True)
 

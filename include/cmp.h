@@ -301,14 +301,15 @@ CMP_API int cmp_profile_stop(double* ms, int64_t* launches);
 
 /* Measurement hook of a library built with -DCMP_PHASE_STAMPS (bench.py
  * --only decode-phases builds one beside the normal library and runs it): the
- * channel-group decode kernel writes the global timer (ns) at 14 points of its
- * timeline; this copies those of its last launch, CTA i's phase k at
- * dst[i * 16 + k] for the first n entries (host array, n <= 512 * 16), after
+ * channel-group decode kernel writes the global timer (ns) at up to 32 points
+ * of its timeline; this copies those of its last launch, CTA i's phase k at
+ * dst[i * 32 + k] for the first n entries (host array, n <= 512 * 32), after
  * synchronising the device. Phases: 0 entry, 1 set-up done, 2 first weight
- * stage landed, 3 last MMA issued, 4 metadata done, 5 accumulator complete,
- * 6 partials sent, 7 partials received, 8 pooled, 9 grid-barrier arrival,
- * 10 tails written, 11 barrier released, 12 RMSNorm scales, 13 end. Other
- * builds return CMP_ERR_UNSUPPORTED. */
+ * stage landed, 3 last MMA issued, 4 metadata done, 5 partials sent,
+ * 6 partials received, 7 pooled and arrived, 9 exchange complete, 10 rows
+ * stored, 11 all CTAs arrived, 14 tails written, 15 end; 16-19 the metadata's
+ * first wave, window list, second and third wave. Other builds return
+ * CMP_ERR_UNSUPPORTED. */
 CMP_API int cmp_debug_phase_stamps(uint64_t* dst, int64_t n);
 
 /* Testing knob: which path calls take. 0 = automatic (for T <= 64 the
@@ -324,12 +325,13 @@ CMP_API int cmp_debug_phase_stamps(uint64_t* dst, int64_t n);
 CMP_API int cmp_set_proj_kernel(int which);
 
 /* Testing knob for failure detection: the next `launches` launches of the
- * channel-group decode kernel (CMP_KERNEL_DECODE_CP) wait at their grid barrier
- * for a count no arrival reaches. Each CTA's bounded wait gives up after about
- * one second, the rows of the call come out as zeros, the CTAs free their tensor
- * memory and return, and cmp_get_error then reports CMP_ERR_TIMEOUT and resets
- * the barrier words, so the next call runs normally. Nothing faults or hangs.
- * Returns the previous count, or -1 if launches < 0. */
+ * channel-group decode kernel (CMP_KERNEL_DECODE_CP) wait for the other
+ * clusters' exchange words of an epoch that no cluster publishes. Each CTA's
+ * bounded wait gives up after about one second, the rows of the call come out
+ * as zeros, the CTAs free their tensor memory and return, and cmp_get_error
+ * then reports CMP_ERR_TIMEOUT and resets the exchange words, so the next call
+ * runs normally. Nothing faults or hangs. Returns the previous count, or -1 if
+ * launches < 0. */
 CMP_API int cmp_debug_unreachable_barrier(int launches);
 
 #ifdef __cplusplus

@@ -346,11 +346,11 @@ def set_proj_kernel(which: int) -> int:
 
 def debug_phase_stamps(n_ctas: int):
     """The channel-group decode kernel's phase stamps of its last launch, as a
-    numpy uint64 array [n_ctas, 16] (global timer, ns). Only the phase-stamp
+    numpy uint64 array [n_ctas, 32] (global timer, ns). Only the phase-stamp
     measurement build (CMP_LIBRARY=.../libcmp_b200_phases.so) records them;
     other builds raise CmpError(CMP_ERR_UNSUPPORTED)."""
     import numpy as np
-    buf = np.zeros((n_ctas, 16), dtype=np.uint64)
+    buf = np.zeros((n_ctas, 32), dtype=np.uint64)
     st = lib.cmp_debug_phase_stamps(buf.ctypes.data, buf.size)
     if st != CMP_OK:
         raise CmpError(st, "cmp_debug_phase_stamps")

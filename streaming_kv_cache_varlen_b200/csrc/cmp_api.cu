@@ -20,8 +20,7 @@ bool decode_fused_supported(const Params& p);
 size_t decode_fused_workspace(const Params& p);
 cudaError_t launch_decode_fused(const Params& p, float* part, void* bar, cudaStream_t s);
 bool decode_cp_supported(const Params& p);
-size_t decode_cp_workspace(const Params& p);
-cudaError_t launch_decode_cp(const Params& p, float* ss, void* counter, cudaStream_t s, bool unreachable);
+cudaError_t launch_decode_cp(const Params& p, void* counter, void* xch, cudaStream_t s, bool unreachable);
 cudaError_t launch_nsa(const NsaParams& p, cudaStream_t s);
 cudaError_t launch_nsa_scan(const NsaParams& p, cudaStream_t s);
 int noalloc_take_error(int dev, unsigned* word);
@@ -36,16 +35,18 @@ using cmp::Params;
 
 // The first kHeaderBytes (zeroed when the workspace is created, and after a
 // timeout) hold the error word at offset 0, the K-split decode kernel's
-// grid-barrier words at offset 64 and the channel-group decode kernel's
-// barrier counter at offset 256; only those kernels write there.
-constexpr size_t kHeaderBytes = 2048;
+// grid-barrier words at offset 64, the channel-group decode kernel's arrival
+// counter at offset 256 and its CTAs' sums (64 windows x 128 CTAs x 4 bytes)
+// from offset 4096; only those kernels write there.
 constexpr size_t kGridBarOffset = 64;
 constexpr size_t kCounterOffset = 256;
+constexpr size_t kExchangeOffset = 4096;
+constexpr size_t kHeaderBytes = kExchangeOffset + 64 * 128 * 4;
 
 size_t zeroed_bytes() { return kHeaderBytes; }
 
 struct WsLayout {
-  size_t err, m_cu, m_s, m_off, m_tile, proj, ystat, ylse, part, total;
+  size_t err, m_cu, m_s, m_off, m_tile, had, proj, ystat, ylse, part, total;
 };
 
 // fused: the pooled-halves buffers of the fused path instead of the fp32
@@ -63,6 +64,7 @@ WsLayout ws_layout(int64_t B, int64_t T, int64_t C, int64_t n_out, bool fused, s
   L.m_s = take(sizeof(int32_t) * std::max<int64_t>(B, 1));
   L.m_off = take(sizeof(int32_t) * (B + 1));
   L.m_tile = take(fused ? sizeof(int32_t) * (B + 1) : 0);
+  L.had = take(sizeof(int32_t) * 16);  // the scheduler's verdicts on the hadamard matrix (<= 4 chunks)
   L.proj = take(fused ? 0 : sizeof(float) * (size_t)T * 2 * C);
   L.ystat = take(fused ? sizeof(float) * (size_t)std::max<int64_t>(n_out, 1) * C : 0);
   L.ylse = take(fused ? sizeof(float) * (size_t)std::max<int64_t>(n_out, 1) * C : 0);
@@ -215,7 +217,6 @@ int get_workspace(cudaStream_t s, size_t need, unsigned char** out) {
 // Extra workspace of the one-kernel decode paths.
 size_t decode_part_bytes(const Params& p, int which) {
   if (which == 5) return cmp::decode_fused_workspace(p);
-  if (which == 6) return cmp::decode_cp_workspace(p);
   return 0;
 }
 
@@ -253,19 +254,22 @@ int run_path(Params& p, int which, cudaStream_t s) {
   p.m_s = reinterpret_cast<int32_t*>(ws + L.m_s);
   p.m_off = reinterpret_cast<int32_t*>(ws + L.m_off);
   p.m_tile = fused ? reinterpret_cast<int32_t*>(ws + L.m_tile) : nullptr;
+  // paths with the scheduler kernel check the hadamard matrix there (the pooling
+  // kernels then use the fast transform for a scaled Sylvester matrix)
+  p.had_sylv = (p.rotate && which != 5 && which != 6) ? reinterpret_cast<int32_t*>(ws + L.had) : nullptr;
   p.proj = fused ? nullptr : reinterpret_cast<float*>(ws + L.proj);
   p.ystat = fused ? reinterpret_cast<float*>(ws + L.ystat) : nullptr;
   p.ylse = fused ? reinterpret_cast<float*>(ws + L.ylse) : nullptr;
 
   // ---- kernels ----
   if (which == 6) {  // decode: one cooperative kernel of clusters, no scheduler launch
-    float* ss = reinterpret_cast<float*>(ws + L.part);
     void* counter = ws + L.err + kCounterOffset;
+    void* xch = ws + L.err + kExchangeOffset;
     bool unreachable = false;  // the timeout test's knob, consumed one launch at a time
     for (int v = g_unreachable_barrier.load(); v > 0 && !unreachable;)
       unreachable = g_unreachable_barrier.compare_exchange_weak(v, v - 1);
     const cudaError_t e = launch(CMP_KERNEL_DECODE_CP, s,
-                                 [&] { return cmp::launch_decode_cp(p, ss, counter, s, unreachable); });
+                                 [&] { return cmp::launch_decode_cp(p, counter, xch, s, unreachable); });
     if (e == cudaErrorNotSupported) return kRetryOtherPath;
     return e == cudaSuccess ? CMP_OK : CMP_ERR_CUDA;
   }
@@ -515,7 +519,8 @@ int cmp_get_error(void* stream) {
       if (cudaMemcpy(&v, it->second.ptr, sizeof(v), cudaMemcpyDeviceToHost) != cudaSuccess)
         return CMP_ERR_CUDA;
       if (v && cudaMemset(it->second.ptr, 0, sizeof(v)) != cudaSuccess) return CMP_ERR_CUDA;
-      // a wait that gave up may have left the grid barrier's count behind
+      // a wait that gave up may have left a grid barrier's count behind; the
+      // decode arrival counter restarts from zero with it
       if ((v & cmp::kErrTimeout) &&
           cudaMemset(it->second.ptr + kGridBarOffset, 0, zeroed_bytes() - kGridBarOffset) != cudaSuccess)
         return CMP_ERR_CUDA;

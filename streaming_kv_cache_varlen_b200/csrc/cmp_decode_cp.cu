@@ -3,38 +3,42 @@
 //
 // The per-channel softmax pooling ("compressor torch_extension API", 计算公式
 // 3-5) never mixes channels, so a cluster that holds the complete projections
-// of some channels can pool them on its own:
+// of some channels can pool them on its own. Cluster g owns channels
+// 16g .. 16g+15 of the D; its four CTAs split the hidden dimension, and after
+// an on-chip reduction CTA q holds channels 16g+4q .. 16g+4q+3.
 //
-//  1. Cluster g owns channels 16g .. 16g+15 of the D. Its four CTAs split the
-//     hidden dimension by 64-column blocks (CTA q takes blocks q, q+4, ...: at
-//     any moment the cluster reads 512 contiguous bytes of each weight row).
-//     Per block, one TMA copy brings the wkv and wgate rows of those channels
-//     (both halves for ratio 4, coff 2: 64 rows, else 32; one 4-D tensor map
-//     spans both matrices) and one brings the x columns; tcgen05.mma
-//     accumulates the rows x tokens product in TMEM (M = 128: the A rows past
-//     the loaded ones are whatever shared memory follows and land in TMEM lanes
-//     nobody reads). Clusters start at different blocks so that they spread
-//     over the DRAM channels. Meanwhile warps 2-3 compute the call's metadata
-//     (what the varlen scheduler kernel does on the other paths) and prefetch
-//     what the later steps read: the state rows of every window the call
-//     completes, ape, norm_weight and the RoPE tables, for this CTA's channels.
-//  2. Each CTA pushes, into the shared memory of CTA q of the cluster, its
-//     partial sums of the rows of channels 16g+4q .. 16g+4q+3; after a cluster
-//     barrier CTA q adds the four partials (in quarter order) and holds complete
-//     kv and score projections of 4 channels for every token of the call.
-//  3. It writes those channels of the state tail rows (score + ape), pools the
-//     4 channels of every window the call completes (a max pass, then an
-//     exp-sum pass, so that the rows' loads and exponentials overlap), and
-//     publishes each output row's sum of squares over its channels.
-//  4. Grid barrier (bounded); RMSNorm needs the sum over all D channels. Each
-//     CTA sums the D/4 partials of each row (fixed order), then scales its
-//     channels, applies norm_weight and the interleaved RoPE (a pair never
-//     straddles two CTAs) and stores bf16 ("CANN PyPTO 算子实战", 压缩窗口与状态更新).
+// Projection. Per 64-column K block one TMA copy brings the wkv and wgate rows
+// of the cluster's channels (both halves for ratio 4, coff 2: 64 rows; else 32;
+// one 5-D tensor map spans both matrices) and one brings the x columns; an
+// M = 64 tcgen05.mma accumulates the rows x tokens product in TMEM. An M = 64
+// accumulator puts rows 16i .. 16i+15 in TMEM lanes 32i .. 32i+15, so each of
+// warps 0-3 holds one 16-row block (one half of one matrix). A decode step's
+// weight stream is bound by the number of MMA instructions (each costs about
+// the same at these sizes), so every MMA carries all the rows it can.
 //
-// The weights are read once; x (small) once per cluster. No projection partial
-// leaves the cluster: the only global exchange is n_out x D/4 floats.
-// This call writes state slots of positions >= start_pos only and reads those
-// below, so the prefetch and the tail stores never touch the same slot.
+// Reduction. Each read-out warp pushes every channel's partial sums to the CTA
+// that owns the channel (st.async into its shared memory, completing on its
+// mbarrier); each owner adds the four partials in rank order.
+//
+// Pooling and RMSNorm. Warp 0 pools its 4 channels of every window the call
+// completes (the windows' state rows were pre-reduced per channel while the
+// weights streamed, so only this call's rows remain), stores the windows' sums
+// of squares over its channels to global memory and arrives (release) at a
+// counter. Every CTA waits (acquire, bounded) until all CTAs have arrived, reads
+// every CTA's sums at once, adds them in a fixed order for the RMSNorm ("CANN PyPTO 算子实战", 压缩窗口与状态更新: rms_norm over the D
+// channels), scales its channels, applies norm_weight and the interleaved RoPE
+// (a pair never straddles two CTAs) and stores bf16. Warps 1-3 meanwhile write
+// the state tails.
+//
+// Warps 4-5 compute the call's metadata (what the varlen scheduler kernel does
+// on the other paths) and prefetch what the later steps read: the state rows
+// of every window the call completes, ape, norm_weight and the RoPE tables, for
+// this CTA's channels. Warp 6 issues the TMA copies, warp 7 the MMAs. Waiting
+// warps let one lane poll, so that they do not crowd the shared-memory pipe the
+// other warps and the tensor core use. The weights are read once, x once per
+// cluster. This call writes state slots of positions >= start_pos only and
+// reads those below, so the prefetch and the tail stores never touch the same
+// slot.
 #include <cstddef>
 #include <mutex>
 
@@ -50,9 +54,9 @@ using namespace sm100;
 // CTA i writes the global timer at phase k to slot i * kStampSlots + k of a
 // device array that cmp_debug_phase_stamps copies out. The normal build has no
 // stamps and no array.
-constexpr int kStampSlots = 16;
-constexpr int kStampCtas = 512;
 #ifdef CMP_PHASE_STAMPS
+constexpr int kStampSlots = 32;
+constexpr int kStampCtas = 512;
 __device__ unsigned long long g_cp_stamps[kStampCtas * kStampSlots];
 #define CP_STAMP(cond, k)                                                           \
   do {                                                                              \
@@ -68,23 +72,22 @@ constexpr int KQ = 4;             // CTAs per cluster: they split the hidden dim
 constexpr int GCH = 16;           // channels per cluster
 constexpr int OWN = GCH / KQ;     // channels per CTA after the reduction
 constexpr int BK = 64;
-constexpr int kThreads = 128;     // warp 0: TMA lane, TMEM rows 0-31; warp 1: MMA lane, rows 32-63;
-                                  // warps 2-3: call metadata and prefetch
+constexpr int KPS = 2;            // 64-column K blocks per pipeline stage
+constexpr int kTileA = 4 * GCH * 128;  // one K block of A: 2 matrices x 2 halves x 16 rows x 128 B
+constexpr int kThreads = 256;     // warps 0-3: TMEM read-out (then warp 0: pooling, exchange, stores;
+                                  // warps 1-3: state tails, rows without a window); warps 4-5:
+                                  // metadata; warp 6 lane 0: TMA; warp 7 lane 0: MMA (warp 7 owns the
+                                  // TMEM)
+constexpr int kMetaBase = 128;    // first metadata thread
 constexpr int kMaxSeqs = 256;
 constexpr int kMaxOut = 64;       // n_out <= T <= 64
 constexpr int kHistRows = 256;    // prefetched state rows (this CTA's 4 kv + 4 score channels)
 constexpr int kMaxWinRows = 128;  // coff * ratio
-constexpr int KPS = 2;            // 64-column K blocks per TMA copy (pipeline stage)
-constexpr int kTileA = 8192;      // one K block of A: 2 matrices x 2 halves x 16 rows x 128 B
-constexpr int kSlackA = 16384 - kTileA;  // the 128-row window the MMA reads past the last tile
-constexpr int kReplicas = 16;     // copies of the sum-of-squares partials (spread the readers)
+constexpr int kMaxClusters = 32;  // D / GCH
 
-// Pipeline depth: with 7 stages for T <= 32 each CTA had nearly its whole K
-// range in flight at once; 4 measured 2 % faster (13.23 vs 13.5 us, bit-identical
-// results), 3 slower.
 template <int MAXT>
 struct Cfg {
-  static constexpr int stages = MAXT <= 32 ? 4 : 5;
+  static constexpr int stages = 4;
 };
 
 struct TokInfo {
@@ -106,18 +109,22 @@ struct Win {        // the window of output row n, if the call completes one the
 template <int MAXT>
 struct Smem {
   static constexpr int S = Cfg<MAXT>::stages;
-  // stage s: KPS A tiles (kinds x 16 rows each) and KPS x tiles (NT rows each),
-  // packed as the TMA boxes land them; after the MMAs, a[] holds the TMEM copy
+  // stage s: KPS A tiles (coff x 2 x 16 rows each) and KPS x tiles (NT rows
+  // each), packed as the TMA boxes land them. An M = 64 MMA reads 64 rows from
+  // its A tile on: for coff 1 (32 rows per tile) the last one reads 4 KB past
+  // the A ring, into x
   alignas(1024) unsigned char a[S][KPS * kTileA];
-  unsigned char a_slack[kSlackA];
   alignas(1024) __nv_bfloat16 x[S][KPS * MAXT * BK];
-  alignas(16) float recv[KQ][4 * MAXT * OWN]; // partials from each CTA of the cluster: [kind][token][channel]
-  alignas(16) float hist[kHistRows][2 * OWN];  // state rows: kv c0..c3, score c0..c3
-  alignas(16) float ape[kMaxWinRows][OWN];     // ape of window row j (half * ratio + residue)
-  alignas(16) float rope[kMaxOut][8];          // per pair: cos even, cos odd, sin even, sin odd
+  alignas(16) float recv[2][KQ][2][OWN][MAXT];  // [half][source rank][kv, score][channel][token]
+  alignas(16) float hist[kHistRows][2 * OWN];    // state rows: kv c0..c3, score c0..c3
+  alignas(16) float ape[kMaxWinRows][OWN];       // ape of window row j (half * ratio + residue)
+  alignas(16) float rope[kMaxOut][8];            // per pair: cos even, cos odd, sin even, sin odd
   alignas(16) float ybuf[kMaxOut][OWN];
+  float ss_own[kMaxOut];                         // this CTA's sums of squares per window (list order)
+  float ss_tot[kMaxOut];                         // every CTA's, added
+  alignas(16) float4 hst[kMaxOut][OWN];          // per window and channel: the state rows' running
+                                                 // max, exp-sum and weighted sum
   float norm[OWN];
-  float scale[kMaxOut];
   TokInfo tok[MAXT];
   Win win[kMaxOut];
   int32_t cu[kMaxSeqs + 1];
@@ -128,63 +135,48 @@ struct Smem {
   int32_t n_win;
   uint64_t full[S];
   uint64_t empty[S];
-  uint64_t acc_full;
-  uint64_t recv_full;   // the four partial blocks have landed in recv
+  uint64_t acc_full;        // the accumulator is complete
+  uint64_t recv_full;       // the partial blocks of every source rank have landed in recv
   uint32_t tmem_base;
+  uint32_t target;          // the arrival count at which this launch's sums are all stored
   int abort;
   int rejected;
-  uint32_t bar_target;
-  int grid_ok;
+  int xch_ok;               // the clusters' sums arrived
 };
 
 static_assert(offsetof(Smem<32>, x) % 1024 == 0 && offsetof(Smem<64>, x) % 1024 == 0,
               "TMA swizzled tiles must be 1024-byte aligned");
-static_assert(offsetof(Smem<32>, a_slack) == sizeof(Smem<32>::a) &&
-                  offsetof(Smem<64>, a_slack) == sizeof(Smem<64>::a),
-              "the MMA's 128-row window past the last stage must stay inside the slack");
+static_assert(offsetof(Smem<32>, x) == sizeof(Smem<32>::a) && offsetof(Smem<64>, x) == sizeof(Smem<64>::a) &&
+                  sizeof(Smem<32>::x) >= 32 * 128,
+              "an MMA's 64-row window past the last A tile stays inside x");
 static_assert(offsetof(Smem<32>, recv) % 16 == 0 && offsetof(Smem<64>, recv) % 16 == 0 &&
                   offsetof(Smem<32>, hist) % 16 == 0 && offsetof(Smem<64>, hist) % 16 == 0 &&
                   offsetof(Smem<32>, ape) % 16 == 0 && offsetof(Smem<64>, ape) % 16 == 0 &&
-                  offsetof(Smem<32>, ybuf) % 16 == 0 && offsetof(Smem<64>, ybuf) % 16 == 0,
+                  offsetof(Smem<32>, ybuf) % 16 == 0 && offsetof(Smem<64>, ybuf) % 16 == 0 &&
+                  offsetof(Smem<32>, hst) % 16 == 0 && offsetof(Smem<64>, hst) % 16 == 0,
               "float4 shared-memory rows must be 16-byte aligned");
-static_assert(KQ * 4 * 64 * OWN * 4 <= Cfg<64>::stages * KPS * kTileA &&
-                  KQ * 4 * 32 * OWN * 4 <= Cfg<32>::stages * KPS * kTileA,
-              "the outgoing partial blocks must fit in the stage buffers");
 static_assert(sizeof(Smem<32>) + 1024 <= 232448 && sizeof(Smem<64>) + 1024 <= 232448,
               "shared memory per CTA");
 
-// Grid barrier for a cooperative launch (every CTA is resident), one use per
-// launch: a counter in memory that starts zeroed and only grows. Every launch
-// adds exactly kQuantum to it (each of its n CTAs adds kQuantum / n), so at
-// launch start it is a multiple of kQuantum, and a CTA that reads it before
-// arriving rounds down to that multiple: the launch is complete when the
-// counter reaches the next one. Arrival is a fire-and-forget release-add
-// (publishing the CTA's stores); grid_wait polls with acquire loads, bounded
-// (~1 s, then a timeout is recorded and the CTA goes on without the data).
-// No reset and no last-arriver step: nothing serializes behind one CTA.
-constexpr uint32_t kQuantum = 1024;
+// The CTAs' arrivals: a 32-bit counter in the workspace that starts zeroed and
+// only grows. Every launch adds exactly kPerLaunch to it (each of its n CTAs
+// adds kPerLaunch / n, on every path), so a CTA that reads it at its start,
+// before all CTAs of its launch have arrived (which needs this CTA's own
+// arrival), sees a value whose multiple of kPerLaunch is the launch's base: the
+// launch's sums are all stored once the counter reaches base + kPerLaunch.
+// (Measured alternative: every CTA polling all CTAs' epoch-tagged 64-bit words
+// instead swamped L2 with polls and took about 10 us.)
+constexpr int kMaxCtas = kMaxClusters * KQ;
+constexpr uint32_t kPerLaunch = kMaxCtas;
 
-__device__ __forceinline__ uint32_t grid_target(const unsigned* counter) {
-  uint32_t v;
-  asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(counter) : "memory");
-  return v - v % kQuantum + kQuantum;
+__device__ __forceinline__ uint32_t arrivals_now(const unsigned* counter) {
+  unsigned v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(counter) : "memory");
+  return v;
 }
 
-__device__ __forceinline__ void grid_arrive(unsigned* counter, unsigned nblocks) {
-  asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(counter), "r"(kQuantum / nblocks) : "memory");
-}
-
-__device__ __forceinline__ bool grid_wait(const unsigned* counter, uint32_t target, unsigned* err) {
-  const uint64_t t0 = globaltimer();
-  for (;;) {
-    uint32_t now;
-    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(now) : "l"(counter) : "memory");
-    if ((int32_t)(now - target) >= 0) return true;
-    if (globaltimer() - t0 > 1000000000ull) {
-      atomicOr(err, kErrTimeout);
-      return false;
-    }
-  }
+__device__ __forceinline__ void arrive_release(unsigned* counter, uint32_t n) {
+  asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(counter), "r"(n) : "memory");
 }
 
 __device__ __forceinline__ uint32_t cluster_rank() {
@@ -208,22 +200,14 @@ __device__ __forceinline__ uint32_t peer_addr(const void* local, uint32_t peer) 
   return ra;
 }
 
-// Bulk copy of `bytes` from this CTA's shared memory into a peer's, completing
-// on the peer's mbarrier (both addresses from peer_addr); one destination CTA per copy.
-__device__ __forceinline__ void bulk_copy_to_peer(uint32_t dst, const void* src, uint32_t bytes, uint32_t mbar) {
-  asm volatile(
-      "cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
-      "r"(smem_u32(src)), "r"(bytes), "r"(mbar)
-      : "memory");
-}
-
-__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
-
-__device__ __forceinline__ void bulk_wait_read() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
-
-// Generic-proxy writes to shared memory before async-proxy reads of it.
-__device__ __forceinline__ void fence_proxy_async_smem() {
-  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+// 16 bytes into a peer's shared memory (addresses from peer_addr), completing
+// on the peer's mbarrier.
+__device__ __forceinline__ void st_async4(uint32_t dst, uint32_t a, uint32_t b, uint32_t c, uint32_t d,
+                                          uint32_t mbar) {
+  asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.b32 [%0], {%1, %2, %3, %4}, [%5];" ::"r"(
+                   dst),
+               "r"(a), "r"(b), "r"(c), "r"(d), "r"(mbar)
+               : "memory");
 }
 
 // TMA copy of a 5-D box into shared memory, completing on an mbarrier.
@@ -241,10 +225,11 @@ __device__ __forceinline__ float4 add4(float4 a, float4 b) {
 }
 
 struct CpArgs {
-  float* ss;          // [kReplicas][n_out][D/4] each CTA's sum of squares of its channels, per output row
-  unsigned* counter;  // grid-barrier counter (zeroed at creation)
-  int kv_first;     // the 4-D weight map holds wkv before wgate (else the other way round)
-  uint32_t bar_extra;  // added to the barrier target: kQuantum makes it unreachable (timeout test)
+  unsigned* counter;  // the CTAs' arrivals (zeroed at creation)
+  float* sums;        // [window list entry][CTA]: each CTA's sums of squares
+  int kv_first;       // the 5-D weight map holds wkv before wgate (else the other way round)
+  uint32_t target_extra;  // added to the count the CTAs wait for: kPerLaunch makes it unreachable
+                          // (timeout test)
 };
 
 // Window row j of window w: its absolute position (rows are in rising order).
@@ -268,13 +253,15 @@ __device__ __forceinline__ int table_entry(const Params& p, const int32_t* __res
   return e;
 }
 
-// Warps 2-3: validation, output-row offsets, per-token facts, the window of
+// Warps 4-5: validation, output-row offsets, per-token facts, the window of
 // every output row, and, for this CTA's channels (columns half * D + ch0 .. +3),
 // the state rows of those windows, ape, norm_weight and the RoPE table entries.
 // Loads are grouped in three waves: inputs, block-table entries, state rows.
+// Also pre-reduces every window's state rows per channel, so that the pooling
+// after the stream only adds this call's rows.
 template <int MAXT>
 __device__ void call_metadata(const Params& p, Smem<MAXT>& sm, int NT, int ch0) {
-  const int et = threadIdx.x - 64;  // 0..63
+  const int et = threadIdx.x - kMetaBase;  // 0..63
   const int B = p.B, r = p.ratio;
   const int rows = p.coff * r;
   const int r0 = p.D - p.rope, hr = p.rope / 2;
@@ -314,7 +301,6 @@ __device__ void call_metadata(const Params& p, Smem<MAXT>& sm, int NT, int ch0) 
   }
   // these loads are issued: let the weight stream start behind them
   asm volatile("bar.arrive 3, 96;" ::: "memory");
-  cluster_wait();  // cluster barrier 0 (every CTA of the cluster runs)
 #pragma unroll
   for (int u = 0; u < 5; ++u)
     if (et + 64 * u <= B) sm.cu[et + 64 * u] = cuv[u];
@@ -338,6 +324,7 @@ __device__ void call_metadata(const Params& p, Smem<MAXT>& sm, int NT, int ch0) 
   if (et == 0) sm.rejected = 0;
   for (int n = et; n < kMaxOut; n += 64) sm.win[n].w = -1;
   asm volatile("bar.sync 2, 64;" ::: "memory");
+  CP_STAMP(et == 0, 16);  // first wave landed
 
   // ---- validation, offsets, tokens, windows (shared memory only) ----
   bool bad = false;
@@ -458,6 +445,7 @@ __device__ void call_metadata(const Params& p, Smem<MAXT>& sm, int NT, int ch0) 
   }
   asm volatile("bar.sync 2, 64;" ::: "memory");
 
+  CP_STAMP(et == 0, 17);  // windows and prefetch ranges known
   // ---- second wave of loads: block-table entries (tails, then hist rows i = et + 64u) ----
   const int total = sm.hstart[p.n_out];
   int hb[4], hq[4], hj[4];
@@ -495,6 +483,7 @@ __device__ void call_metadata(const Params& p, Smem<MAXT>& sm, int NT, int ch0) 
     sm.tok[et] = ti;
   }
 
+  CP_STAMP(et == 0, 18);  // second wave landed
   // ---- third wave of loads: the state rows (a row that does not exist: kv 0, score -inf) ----
   float4 v[4][2];
 #pragma unroll
@@ -517,293 +506,237 @@ __device__ void call_metadata(const Params& p, Smem<MAXT>& sm, int NT, int ch0) 
       *reinterpret_cast<float4*>(&sm.hist[i][OWN]) = v[u][1];
     }
   }
-}
+  asm volatile("bar.sync 2, 64;" ::: "memory");
+  CP_STAMP(et == 0, 19);  // third wave landed
 
-// The complete projection of kind k, token t, channel c of this CTA: the four
-// received partial blocks added in rank order.
-template <int MAXT>
-__device__ __forceinline__ float own_value(const Params& p, const Smem<MAXT>& sm, int k, int t, int c) {
-  const int i = (k * p.T + t) * OWN + c;
-  return ((sm.recv[0][i] + sm.recv[1][i]) + sm.recv[2][i]) + sm.recv[3][i];
-}
-
-__device__ __forceinline__ float4 own_value4(const float* r0, const float* r1, const float* r2, const float* r3) {
-  const float4 a = *reinterpret_cast<const float4*>(r0), b = *reinterpret_cast<const float4*>(r1);
-  const float4 c = *reinterpret_cast<const float4*>(r2), d = *reinterpret_cast<const float4*>(r3);
-  return make_float4(((a.x + b.x) + c.x) + d.x, ((a.y + b.y) + c.y) + d.y, ((a.z + b.z) + c.z) + d.z,
-                     ((a.w + b.w) + c.w) + d.w);
-}
-
-// Window row j's kv and score (score + ape for this call's tokens) for channel c.
-template <int MAXT>
-__device__ __forceinline__ void window_row(const Params& p, const Smem<MAXT>& sm, const Win& w, int j, int c,
-                                           float& kv, float& z) {
-  if (j < w.hrows) {
-    kv = sm.hist[w.hist + j][c];
-    z = sm.hist[w.hist + j][OWN + c];
-  } else {
-    const int r = p.ratio;
-    const int half = (p.coff == 2 && j >= r) ? 1 : 0;
-    const int t = w.cu + (window_pos(w.w, j, r, p.coff) - w.s);
-    kv = own_value(p, sm, half, t, c);
-    z = own_value(p, sm, p.coff + half, t, c) + sm.ape[j][c];
-  }
-}
-
-template <int MAXT>
-__global__ void __launch_bounds__(kThreads, 1)
-    decode_cp_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUtensorMap map_w,
-                     Params p, CpArgs a, int NT) {
-  extern __shared__ __align__(1024) unsigned char smem_raw[];
-  using SM = Smem<MAXT>;
-  constexpr int STAGES = SM::S;
-  SM& sm = smem_align1024<SM>(smem_raw);
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const uint32_t q = cluster_rank();          // this CTA's share of the hidden dimension
-  const int g = blockIdx.x / KQ;              // channel group of the cluster
-  const int ch0 = g * GCH + (int)q * OWN;     // this CTA's channels after the reduction
-  const int kinds = 2 * p.coff;               // kv halves, then score halves
-  const int nsteps = p.H / (KQ * KPS * BK);   // pipeline steps per CTA (KPS K blocks each)
-  const uint32_t bytes = KPS * ((uint32_t)kinds * GCH * BK * 2 + (uint32_t)NT * BK * 2);
-  const uint32_t tmem_cols = NT <= 32 ? 32 : 64;
-  // after the MMAs: the outgoing partials, one block per owner CTA [owner][kind][token][channel]
-  float* part = reinterpret_cast<float*>(&sm.a[0][0]);
-  const int blk_floats = kinds * p.T * OWN;
-  CP_STAMP(threadIdx.x == 0, 0);  // entry
-
-  if (threadIdx.x == 0) {
-    for (int s = 0; s < STAGES; ++s) {
-      mbar_init(&sm.full[s], 1);
-      mbar_init(&sm.empty[s], 1);
+  // ---- every window's state rows, pre-reduced per channel (online softmax);
+  // two lanes per (window, channel) take alternate rows and merge ----
+  for (int base = 0; base < sm.n_win * OWN * 2; base += 64) {
+    const int u = (base + et) >> 1, side = et & 1;
+    const bool live = u < sm.n_win * OWN;
+    const int i = live ? u / OWN : 0, c = u % OWN;
+    const Win w = sm.win[sm.wlist[i]];
+    float m = -INFINITY, l = 0.f, acc = 0.f;
+    for (int j = side; j < w.hrows && live; j += 2) {
+      float kv, z;
+      if (w.hist >= 0) {
+        kv = sm.hist[w.hist + j][c];
+        z = sm.hist[w.hist + j][OWN + c];
+      } else {  // more state rows than the prefetch holds: from the paged state
+        const int qp = window_pos(w.w, j, r, p.coff);
+        if (qp < 0) continue;
+        const int rk = table_row(p, p.kv_tbl, w.b, qp);
+        const int rs = table_row(p, p.sc_tbl, w.b, qp);
+        if (rk < 0 || rs < 0) continue;
+        const int col = ((p.coff == 2 && j >= r) ? p.D : 0) + ch0 + c;
+        kv = p.kv_state[((int64_t)rk * p.bs + qp % p.bs) * p.C + col];
+        z = p.score_state[((int64_t)rs * p.bs + qp % p.bs) * p.C + col];
+      }
+      if (z == -INFINITY) continue;  // a row that does not exist
+      const float mn = fmaxf(m, z);
+      const float f = __expf(m - mn), e = __expf(z - mn);
+      l = l * f + e;
+      acc = acc * f + e * kv;
+      m = mn;
     }
-    mbar_init(&sm.acc_full, 1);
-    mbar_init(&sm.recv_full, 1);
-    sm.abort = 0;
-    fence_barrier_init();
-    // the four incoming partial blocks (one of them this CTA's own)
-    mbar_arrive_expect_tx(&sm.recv_full, (uint32_t)(KQ * kinds * p.T * OWN * 4));
-    prefetch_tmap(&map_w);
-    prefetch_tmap(&map_x);
+    {
+      const float m2 = __shfl_xor_sync(0xffffffffu, m, 1);
+      const float l2 = __shfl_xor_sync(0xffffffffu, l, 1);
+      const float a2 = __shfl_xor_sync(0xffffffffu, acc, 1);
+      const float mn = fmaxf(m, m2);
+      const float f1 = m == -INFINITY ? 0.f : __expf(m - mn);
+      const float f2 = m2 == -INFINITY ? 0.f : __expf(m2 - mn);
+      l = l * f1 + l2 * f2;
+      acc = acc * f1 + a2 * f2;
+      m = mn;
+    }
+    if (live && side == 0) sm.hst[i][c] = make_float4(m, l, acc, 0.f);
   }
-  if (warp == 1) tmem_alloc(&sm.tmem_base, tmem_cols);
-  cluster_arrive_relaxed();  // cluster barrier 0: this CTA runs (its barriers are initialized)
-  tc_fence_before();
-  __syncthreads();
+}
+
+// The complete projection of kind k (0 kv, 1 score), half h of the state row
+// (coff 2: 0 = columns [0, D), 1 = [D, 2D); coff 1: 0), channel c and token t:
+// the four received partials added in rank order.
+template <int MAXT>
+__device__ __forceinline__ float own_value(const Smem<MAXT>& sm, int h, int k, int c, int t) {
+  return ((sm.recv[h][0][k][c][t] + sm.recv[h][1][k][c][t]) + sm.recv[h][2][k][c][t]) + sm.recv[h][3][k][c][t];
+}
+
+__device__ __forceinline__ void warp_sync_all() { __syncwarp(0xffffffffu); }
+
+// A warp waits for a phase of an mbarrier: lane 0 polls (a whole warp
+// spinning would crowd the shared-memory pipe), then the warp synchronises. Bounded (~2 s); with `abort` non-null it also
+// gives up when another role aborted, and raises the flag when it times out.
+// Returns the same answer in every lane.
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort) {
+  int ok = 1;
+  if ((threadIdx.x & 31) == 0) {
+    const uint32_t a = smem_u32(bar);
+    const uint64_t t0 = globaltimer();
+    while (!mbar_try_wait(a, parity)) {
+      if (abort && *abort) { ok = 0; break; }
+      if (globaltimer() - t0 > 2000000000ull) {
+        ok = 0;
+        if (abort) *abort = 1;
+        break;
+      }
+    }
+  }
+  ok = __shfl_sync(0xffffffffu, ok, 0);
+  __syncwarp(0xffffffffu);
+  return ok != 0;
+}
+
+// A read-out warp w (0..3) holds accumulator rows 16w .. 16w+15 in its TMEM
+// lanes 0-15 (an M = 64 accumulator, columns = tokens): for coff 2 the rows of
+// matrix w / 2, half w % 2; for coff 1 those of matrix w (warps 0, 1). Each
+// lane pushes its row to the CTA that owns the channel, into its
+// recv[half][this rank][kind][channel][*]. False if the accumulator never
+// completed (nothing is sent).
+template <int MAXT>
+__device__ bool send_partials(Smem<MAXT>& sm, uint32_t tmem, int w, int coff, int NT, int kv_first, uint32_t q,
+                              volatile int* abort) {
+  const int lane = threadIdx.x & 31;
+  const int matrix = coff == 2 ? w >> 1 : w, half = coff == 2 ? w & 1 : 0;
+  if (!warp_wait(&sm.acc_full, 0, abort)) return false;
   tc_fence_after();
-  const uint32_t tmem = sm.tmem_base;
-  volatile int* abort = &sm.abort;
-  CP_STAMP(threadIdx.x == 0, 1);  // set-up done
-
-  // ---- 1) stream + MMA (lane 0 of warps 0, 1) / metadata and prefetch (warps 2, 3) ----
-  // the metadata's first loads go out before the weight stream (named barrier 3)
-  if (warp == 0) asm volatile("bar.sync 3, 96;" ::: "memory");
-  if (warp == 0 && lane == 0) {
-    int stage = 0;
-    uint32_t phase = 0;
-    for (int st = 0; st < nsteps; ++st) {
-      if (!mbar_wait(&sm.empty[stage], phase ^ 1u, abort)) break;
-      mbar_arrive_expect_tx(&sm.full[stage], bytes);
-      // K blocks cb .. cb+KPS-1: clusters start at different steps, the four
-      // CTAs of a cluster take adjacent chunks
-      const int cb = (((st + g) % nsteps) * KQ + (int)q) * KPS;
-      tma_load_5d(sm.a[stage], &map_w, &sm.full[stage], 0, g * GCH, 0, 0, cb);
-      tma_load_3d(sm.x[stage], &map_x, &sm.full[stage], 0, 0, cb);
-      if (++stage == STAGES) { stage = 0; phase ^= 1u; }
-    }
-  } else if (warp == 1 && lane == 0) {
-    int stage = 0;
-    uint32_t phase = 0;
-    const uint32_t idesc = idesc_bf16_f32(128, NT);
-    bool ok = true;
-    for (int st = 0; st < nsteps; ++st) {
-      if (!mbar_wait(&sm.full[stage], phase, abort)) { ok = false; break; }
-      CP_STAMP(st == 0, 2);  // first stage landed
-      tc_fence_after();
+  const int kind = ((matrix == 0) == (kv_first != 0)) ? 0 : 1;
+  const int cg = lane & 15;
+  const uint32_t owner = (uint32_t)(cg / OWN);
+  const uint32_t dst = peer_addr(&sm.recv[half][q][kind][cg % OWN][0], owner);
+  const uint32_t mbar = peer_addr(&sm.recv_full, owner);
+  for (int c0 = 0; c0 < NT; c0 += 32) {
+    uint32_t r[32];
+    tmem_ld32(tmem + ((uint32_t)(32 * w) << 16) + (uint32_t)c0, r);
+    tmem_ld_wait(r);
+    if (lane < 16) {
 #pragma unroll
-      for (int kk = 0; kk < KPS; ++kk) {
-        // the copies land packed: KPS A tiles of kinds x 16 rows, KPS x tiles of NT rows
-        const uint32_t a0 = smem_u32(sm.a[stage]) + kk * kinds * GCH * 128;
-        const uint32_t b0 = smem_u32(sm.x[stage]) + kk * NT * 128;
-#pragma unroll
-        for (int k = 0; k < BK / 16; ++k)
-          mma_bf16(tmem, sw128_kmajor_desc(a0 + k * 32), sw128_kmajor_desc(b0 + k * 32), idesc,
-                   (st > 0 || kk > 0 || k > 0) ? 1u : 0u);
-      }
-      mma_commit(&sm.empty[stage]);
-      if (++stage == STAGES) { stage = 0; phase ^= 1u; }
-    }
-    if (ok) mma_commit(&sm.acc_full);
-    CP_STAMP(true, 3);  // last MMA issued
-  } else if (warp >= 2) {
-    // the grid barrier's target, read here rather than before the stream starts
-    // (a cold global load); any time before this CTA's own arrival is correct:
-    // the count cannot reach the next multiple while this CTA's share is missing
-    if (threadIdx.x == 64) sm.bar_target = grid_target(a.counter) + a.bar_extra;
-    call_metadata<MAXT>(p, sm, NT, ch0);
-    CP_STAMP(threadIdx.x == 64, 4);  // metadata and prefetch done
-  }
-
-  // ---- 2) warps 0-1: TMEM rows -> the owners' blocks, one bulk copy per owner;
-  // every CTA then adds the four blocks it received (in rank order) ----
-  if (warp < 2) {
-    const bool have = mbar_wait(&sm.acc_full, 0, abort);
-    CP_STAMP(threadIdx.x == 0, 5);  // accumulator complete
-    __syncwarp();
-    if (__all_sync(0xffffffffu, have) && warp * 32 < kinds * GCH) {
-      tc_fence_after();
-      // TMEM lane = A row: 16-row block of the tile, channel of the cluster's 16
-      const int row = warp * 32 + lane, b = row / GCH, cg = row % GCH;
-      const int k = a.kv_first ? b : (b + p.coff) % kinds;  // kind of that block
-      float* dst = part + (cg / OWN) * blk_floats + k * p.T * OWN + cg % OWN;
-      for (int c0 = 0; c0 < NT; c0 += 32) {
-        uint32_t r[32];
-        tmem_ld32(tmem + ((uint32_t)(warp * 32) << 16) + c0, r);
-        tmem_ld_wait(r);
-#pragma unroll
-        for (int j = 0; j < 32; ++j)
-          if (c0 + j < p.T) dst[(c0 + j) * OWN] = __uint_as_float(r[j]);
-      }
-    }
-    tc_fence_before();
-    fence_proxy_async_smem();  // the blocks are read by the bulk copies
-    asm volatile("bar.sync 1, 64;" ::: "memory");
-    cluster_wait();  // cluster barrier 0: every CTA of the cluster runs, its barriers initialized
-    if (threadIdx.x == 0) {
-      const uint32_t bytes = (uint32_t)blk_floats * 4;
-      for (int o = 0; o < KQ; ++o)
-        bulk_copy_to_peer(peer_addr(&sm.recv[q][0], (uint32_t)o), part + o * blk_floats, bytes,
-                          peer_addr(&sm.recv_full, (uint32_t)o));
-      bulk_commit();
-      CP_STAMP(true, 6);  // partial blocks sent
+      for (int j = 0; j < 32; j += 4)
+        if (c0 + j < NT) st_async4(dst + (uint32_t)(c0 + j) * 4u, r[j], r[j + 1], r[j + 2], r[j + 3], mbar);
     }
   }
-  if (threadIdx.x == 0) {
-    // not cut short by this CTA's abort flag: the peers' copies into this CTA
-    // must land before it goes on (and, at the latest, before it exits)
-    int never = 0;
-    if (!mbar_wait(&sm.recv_full, 0, &never)) atomicOr(p.err, kErrTimeout);
-    CP_STAMP(true, 7);  // the four partial blocks landed
-  }
-  __syncthreads();  // the partials have landed, and the metadata is complete
-  const bool mm_ok = !*abort;
+  return true;
+}
 
-  // ---- 3) pooling: 16 threads per window (4 channels x 4 row lanes), 8 windows at a time ----
-  const int r = p.ratio, n_out = p.n_out, rows = p.coff * r, nw = sm.n_win;
-  {
-    const int c = (threadIdx.x >> 2) & 3, rl = threadIdx.x & 3;
-    for (int wi = threadIdx.x >> 4; wi < nw + 7 - ((nw + 7) % 8); wi += kThreads / 16) {
-      // every lane runs the shuffles; lanes past the last window compute nothing
-      const bool live = wi < nw && mm_ok;
-      const int n = live ? sm.wlist[wi] : 0;
-      Win w = sm.win[n];
-      float m = -INFINITY, l = 0.f, acc = 0.f;
-      for (int j = rl; j < rows && live; j += 4) {
-        float kv, z;
-        if (j < w.hrows && w.hist < 0) {  // more state rows than the prefetch holds
-          const int qp = window_pos(w.w, j, r, p.coff);
-          if (qp < 0) continue;
-          const int rk = table_row(p, p.kv_tbl, w.b, qp);
-          const int rs = table_row(p, p.sc_tbl, w.b, qp);
-          if (rk < 0 || rs < 0) continue;
-          const int col = ((p.coff == 2 && j >= r) ? p.D : 0) + ch0 + c;
-          kv = p.kv_state[((int64_t)rk * p.bs + qp % p.bs) * p.C + col];
-          z = p.score_state[((int64_t)rs * p.bs + qp % p.bs) * p.C + col];
-        } else {
-          window_row(p, sm, w, j, c, kv, z);
-        }
-        if (z == -INFINITY) continue;  // a row that does not exist
+// A whole warp waits (bounded, ~2 s, not cut short by the CTA's abort flag:
+// pushes into this CTA must land before it goes on) for a phase of pushes.
+__device__ __forceinline__ bool wait_pushes(uint64_t* bar) { return warp_wait(bar, 0, nullptr); }
+
+// Warps 1-3: every (half, kind) pair of this CTA's 4 channels goes to the
+// state tail rows (score rows with ape); warp 1 + f takes pairs f, f + 3.
+template <int MAXT>
+__device__ void write_tails(const Params& p, const Smem<MAXT>& sm, int ch0, int f) {
+  const int r = p.ratio;
+  for (int pair = f; pair < 2 * p.coff; pair += 3) {
+    const int half = pair >> 1, k = pair & 1;
+    for (int t = threadIdx.x & 31; t < p.T; t += 32) {
+      const TokInfo ti = sm.tok[t];
+      const int64_t so = k ? ti.sc_off : ti.kv_off;
+      if (ti.b < 0 || so < 0) continue;
+      float4 v = make_float4(own_value(sm, half, k, 0, t), own_value(sm, half, k, 1, t),
+                             own_value(sm, half, k, 2, t), own_value(sm, half, k, 3, t));
+      if (k) v = add4(v, *reinterpret_cast<const float4*>(&sm.ape[half * r + ti.pos % r][0]));
+      *reinterpret_cast<float4*>((k ? p.score_state : p.kv_state) + so + half * p.D + ch0) = v;
+    }
+  }
+}
+
+// Warp 0, once the partials have landed and the metadata is done: pool,
+// exchange the windows' sums of squares (every CTA stores its sums and arrives
+// at the counter, waits for all arrivals and reads every CTA's sums), then
+// RMSNorm, norm_weight, RoPE and the bf16 store of this CTA's channels.
+template <int MAXT>
+__device__ void pool_and_finish(const Params& p, Smem<MAXT>& sm, const CpArgs& a, int ch0, uint32_t q,
+                                bool ok) {
+  const int lane = threadIdx.x & 31;
+  const int r = p.ratio, rows = p.coff * r;
+  const int nw = sm.n_win;
+  // ---- pooling: lane = 4 * (window mod 8) + channel; the state rows come pre-reduced ----
+  for (int base = 0; base < nw; base += 8) {
+    const int i = base + (lane >> 2), c = lane & 3;
+    const bool live = i < nw;
+    float y = 0.f;
+    int n = 0;
+    if (live) {
+      n = sm.wlist[i];
+      const Win w = sm.win[n];
+      const float4 h = sm.hst[i][c];
+      float m = h.x, l = h.y, acc = h.z;
+      for (int j = w.hrows; j < rows && ok; ++j) {  // this call's rows
+        const int h = (p.coff == 2 && j >= r) ? 1 : 0;
+        const int t = w.cu + (window_pos(w.w, j, r, p.coff) - w.s);
+        const float kv = own_value(sm, h, 0, c, t);
+        const float z = own_value(sm, h, 1, c, t) + sm.ape[j][c];
         const float mn = fmaxf(m, z);
         const float f = __expf(m - mn), e = __expf(z - mn);
         l = l * f + e;
         acc = acc * f + e * kv;
         m = mn;
       }
-      // merge the 4 row lanes of each channel (log-sum-exp)
-#pragma unroll
-      for (int o = 1; o < 4; o <<= 1) {
-        const float m2 = __shfl_xor_sync(0xffffffffu, m, o);
-        const float l2 = __shfl_xor_sync(0xffffffffu, l, o);
-        const float a2 = __shfl_xor_sync(0xffffffffu, acc, o);
-        const float mn = fmaxf(m, m2);
-        const float f1 = m == -INFINITY ? 0.f : __expf(m - mn);
-        const float f2 = m2 == -INFINITY ? 0.f : __expf(m2 - mn);
-        l = l * f1 + l2 * f2;
-        acc = acc * f1 + a2 * f2;
-        m = mn;
+      y = (ok && l > 0.f) ? __fdividef(acc, l) : 0.f;
+      sm.ybuf[n][c] = y;
+    }
+    // the window's sum of squares over this CTA's 4 channels (lanes 4i' .. 4i'+3)
+    float s = y * y;
+    s += __shfl_xor_sync(0xffffffffu, s, 1);
+    s += __shfl_xor_sync(0xffffffffu, s, 2);
+    if (live && c == 0) sm.ss_own[i] = s;
+  }
+  warp_sync_all();
+  // ---- this CTA's sums of squares to global memory, then its arrival (release) ----
+  if (lane == 0) {
+    for (int i = 0; i < nw; ++i) a.sums[(int64_t)i * kMaxCtas + blockIdx.x] = sm.ss_own[i];
+    arrive_release(a.counter, kPerLaunch / gridDim.x);
+  }
+  CP_STAMP(lane == 0, 7);  // pooled, arrived
+  // ---- every CTA's sums once all have arrived: acquire polls by one lane, then
+  // weak loads that bypass L1 (all in flight at once), added in a fixed order ----
+  int got = 1;
+  if (lane == 0) {
+    const uint32_t target = sm.target + a.target_extra;
+    const uint64_t t0 = globaltimer();
+    while ((int32_t)(arrivals_now(a.counter) - target) < 0) {
+      if (globaltimer() - t0 > 1000000000ull) {
+        got = 0;
+        break;
       }
-      if (live && rl == 0) sm.ybuf[n][c] = l > 0.f ? __fdividef(acc, l) : 0.f;
     }
   }
-  __syncthreads();
-  CP_STAMP(threadIdx.x == 0, 8);  // pooled
-  const int n_cta = gridDim.x;
-  const int64_t rep_stride = (int64_t)n_out * n_cta;
-  for (int i = threadIdx.x; i < nw * kReplicas; i += kThreads) {
-    const int n = sm.wlist[i / kReplicas];
-    const float4 y = *reinterpret_cast<const float4*>(&sm.ybuf[n][0]);
-    a.ss[(i % kReplicas) * rep_stride + (int64_t)n * n_cta + blockIdx.x] =
-        y.x * y.x + y.y * y.y + y.z * y.z + y.w * y.w;
-  }
-  __syncthreads();
-  if (threadIdx.x == 0) grid_arrive(a.counter, n_cta);
-  CP_STAMP(threadIdx.x == 0, 9);  // arrived at the grid barrier
-
-  // ---- while the other CTAs arrive: state tails and rows without a window ----
-  for (int i = threadIdx.x; i < kinds * p.T && mm_ok; i += kThreads) {
-    const int k = i / p.T, t = i % p.T;
-    const TokInfo ti = sm.tok[t];
-    const bool score = k >= p.coff;
-    const int64_t so = score ? ti.sc_off : ti.kv_off;
-    if (ti.b < 0 || so < 0) continue;
-    const int half = score ? k - p.coff : k;
-    const int e = (k * p.T + t) * OWN;
-    float4 v = own_value4(&sm.recv[0][e], &sm.recv[1][e], &sm.recv[2][e], &sm.recv[3][e]);
-    if (score) v = add4(v, *reinterpret_cast<const float4*>(&sm.ape[half * r + ti.pos % r][0]));
-    *reinterpret_cast<float4*>((score ? p.score_state : p.kv_state) + so + half * p.D + ch0) = v;
-  }
-  for (int n = threadIdx.x; n < n_out; n += kThreads)
-    if (sm.win[n].w < 0) *reinterpret_cast<uint2*>(p.out + (int64_t)n * p.D + ch0) = make_uint2(0u, 0u);
-  CP_STAMP(threadIdx.x == 0, 10);  // tails written
-  if (threadIdx.x == 0) sm.grid_ok = grid_wait(a.counter, sm.bar_target, p.err) ? 1 : 0;
-  CP_STAMP(threadIdx.x == 0, 11);  // grid barrier released
-  __syncthreads();
-  const bool ok = sm.grid_ok != 0 && mm_ok;
-
-  // ---- 4) RMSNorm scale of each window row (its D/4 partials, fixed order), then this CTA's channels ----
-  if (ok) {
-    const int nq = n_cta / 4;  // float4 per row of partials (<= 32: one per lane)
-    const int mine = nw > warp ? (nw - warp + 3) / 4 : 0;  // list entries warp, warp + 4, ...
-    for (int u0 = 0; u0 < mine; u0 += 8) {
-      float4 v[8];
+  CP_STAMP(lane == 0, 11);  // all CTAs arrived
+  got = __shfl_sync(0xffffffffu, got, 0);
+  warp_sync_all();
+  if (got) {
+    const int per_lane = (int)gridDim.x / 32;  // 1 or 4 partials per lane and window
+    for (int i0 = 0; i0 < nw; i0 += 8) {
+      float v[8][4];
+#pragma unroll
+      for (int u = 0; u < 8; ++u)
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+          v[u][k] = (i0 + u < nw && k < per_lane) ? __ldcg(a.sums + (int64_t)(i0 + u) * kMaxCtas + lane + 32 * k)
+                                                 : 0.f;
 #pragma unroll
       for (int u = 0; u < 8; ++u) {
-        const int n = sm.wlist[warp + 4 * (u0 + u < mine ? u0 + u : u0)];
-        const float* row = a.ss + (int64_t)(blockIdx.x % kReplicas) * rep_stride + (int64_t)n * n_cta;
-        v[u] = lane < nq ? __ldcg(reinterpret_cast<const float4*>(row) + lane) : make_float4(0.f, 0.f, 0.f, 0.f);
-      }
-      float t[8];
+        float t = ((v[u][0] + v[u][1]) + v[u][2]) + v[u][3];
 #pragma unroll
-      for (int u = 0; u < 8; ++u) t[u] = (v[u].x + v[u].y) + (v[u].z + v[u].w);
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) {
-#pragma unroll
-        for (int u = 0; u < 8; ++u) t[u] += __shfl_xor_sync(0xffffffffu, t[u], o);
-      }
-      if (lane == 0) {
-#pragma unroll
-        for (int u = 0; u < 8; ++u)
-          if (u0 + u < mine) sm.scale[sm.wlist[warp + 4 * (u0 + u)]] = rsqrtf(t[u] / (float)p.D + 1e-6f);
+        for (int o = 16; o > 0; o >>= 1) t += __shfl_xor_sync(0xffffffffu, t, o);
+        if (lane == 0 && i0 + u < nw) sm.ss_tot[i0 + u] = t;
       }
     }
+  } else if (lane == 0) {
+    atomicOr(p.err, kErrTimeout);
+    sm.xch_ok = 0;
   }
-  __syncthreads();
-  CP_STAMP(threadIdx.x == 0, 12);  // RMSNorm scales summed
+  warp_sync_all();
+  CP_STAMP(lane == 0, 9);  // exchange complete
+  // ---- RMSNorm scale, norm_weight, RoPE, bf16 store ----
+  const bool fin = ok && sm.xch_ok != 0;
   const bool roped = ch0 >= p.D - p.rope;
-  for (int wi = threadIdx.x; wi < nw; wi += kThreads) {
-    const int n = sm.wlist[wi];
+  for (int i = lane; i < nw; i += 32) {
+    const int n = sm.wlist[i];
     float z[OWN] = {0.f, 0.f, 0.f, 0.f};
-    if (ok) {
-      const float sc = sm.scale[n];
+    if (fin) {
+      const float sc = rsqrtf(sm.ss_tot[i] / (float)p.D + 1e-6f);
 #pragma unroll
       for (int c = 0; c < OWN; ++c) z[c] = sm.ybuf[n][c] * sc * sm.norm[c];
       if (roped) {  // interleaved RoPE: pairs (2j, 2j+1) of the last rope channels
@@ -823,25 +756,147 @@ __global__ void __launch_bounds__(kThreads, 1)
     v.y = *reinterpret_cast<uint32_t*>(&o23);
     *reinterpret_cast<uint2*>(p.out + (int64_t)n * p.D + ch0) = v;
   }
+  CP_STAMP(lane == 0, 10);  // rows stored
+}
 
-  if (threadIdx.x == 0) bulk_wait_read();  // this CTA's outgoing copies have read its blocks
+template <int MAXT>
+__global__ void __launch_bounds__(kThreads, 1)
+    decode_cp_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUtensorMap map_w,
+                     Params p, CpArgs a, int NT) {
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  using SM = Smem<MAXT>;
+  constexpr int STAGES = SM::S;
+  SM& sm = smem_align1024<SM>(smem_raw);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t q = cluster_rank();          // this CTA's share of the hidden dimension
+  const int g = blockIdx.x / KQ;              // channel group of the cluster
+  const int ch0 = g * GCH + (int)q * OWN;     // this CTA's channels after the reduction
+  const int nsteps = p.H / (KQ * KPS * BK);   // pipeline steps per CTA
+  const uint32_t a_tile = (uint32_t)p.coff * 2 * GCH * 128;  // one K block of A as it lands
+  const uint32_t bytes = KPS * (a_tile + (uint32_t)NT * BK * 2);
+  const uint32_t tmem_cols = NT <= 32 ? 32 : 64;
+  CP_STAMP(threadIdx.x == 0, 0);  // entry
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&sm.full[s], 1);
+      mbar_init(&sm.empty[s], 1);
+    }
+    mbar_init(&sm.acc_full, 1);
+    mbar_init(&sm.recv_full, 1);
+    sm.abort = 0;
+    sm.xch_ok = 1;
+    fence_barrier_init();
+    // what lands here from the cluster: every rank's coff halves x 2 kinds x
+    // OWN channels x NT tokens
+    mbar_arrive_expect_tx(&sm.recv_full, (uint32_t)(KQ * p.coff * 2 * OWN * NT * 4));
+    prefetch_tmap(&map_w);
+    prefetch_tmap(&map_x);
+  }
+  if (warp == 7) tmem_alloc(&sm.tmem_base, tmem_cols);
+  cluster_arrive_relaxed();  // cluster barrier 0: this CTA runs (its barriers are initialized)
+  tc_fence_before();
   __syncthreads();
-  if (warp == 1) {
+  tc_fence_after();
+  const uint32_t tmem = sm.tmem_base;
+  volatile int* abort = &sm.abort;
+  CP_STAMP(threadIdx.x == 0, 1);  // set-up done
+
+  if (warp == 6) {
+    // ---- TMA: the metadata's first loads go out before the weight stream (named barrier 3) ----
+    asm volatile("bar.sync 3, 96;" ::: "memory");
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      for (int st = 0; st < nsteps; ++st) {
+        if (!mbar_wait(&sm.empty[stage], phase ^ 1u, abort)) break;
+        mbar_arrive_expect_tx(&sm.full[stage], bytes);
+        // K blocks cb, cb+1: clusters start at different steps, the four CTAs of
+        // a cluster take adjacent chunks
+        const int cb = (((st + g) % nsteps) * KQ + (int)q) * KPS;
+        tma_load_5d(sm.a[stage], &map_w, &sm.full[stage], 0, g * GCH, 0, 0, cb);
+        tma_load_3d(sm.x[stage], &map_x, &sm.full[stage], 0, 0, cb);
+        if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+      }
+    }
+  } else if (warp == 7) {
+    // ---- MMA (M = 64): every A row of the stage in one accumulator ----
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      const uint32_t idesc = idesc_bf16_f32(64, NT);
+      bool ok = true;
+      for (int st = 0; st < nsteps; ++st) {
+        if (!mbar_wait(&sm.full[stage], phase, abort)) { ok = false; break; }
+        CP_STAMP(st == 0, 2);  // first stage landed
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < KPS; ++kk) {
+          // the copies land packed: KPS A tiles of a_tile bytes, KPS x tiles of NT rows
+          const uint32_t a0 = smem_u32(sm.a[stage]) + kk * a_tile;
+          const uint32_t b0 = smem_u32(sm.x[stage]) + kk * NT * 128;
+#pragma unroll
+          for (int k = 0; k < BK / 16; ++k)
+            mma_bf16(tmem, sw128_kmajor_desc(a0 + k * 32), sw128_kmajor_desc(b0 + k * 32), idesc,
+                     (st > 0 || kk > 0 || k > 0) ? 1u : 0u);
+        }
+        mma_commit(&sm.empty[stage]);
+        if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+      }
+      if (ok) mma_commit(&sm.acc_full);
+      CP_STAMP(true, 3);  // last MMA issued
+    }
+  } else if (warp >= 4) {
+    // ---- warps 4-5: metadata and prefetch ----
+    call_metadata<MAXT>(p, sm, NT, ch0);
+    CP_STAMP(threadIdx.x == kMetaBase, 4);  // metadata done
+    asm volatile("bar.arrive 4, 96;" ::: "memory");   // to warp 0
+    asm volatile("bar.arrive 5, 160;" ::: "memory");  // to warps 1-3
+  } else {
+    // ---- warps 0-3: read-out; then warp 0 pools, exchanges and stores the rows,
+    // warps 1-3 write the state tails and the rows without a window ----
+    uint32_t ctr = 0;
+    if (warp == 0) ctr = arrivals_now(a.counter);  // this launch's base (a cold load)
+    cluster_wait();  // cluster barrier 0: every CTA of the cluster runs before a push
+    bool ok = true;
+    if (warp < 2 * p.coff) ok = send_partials(sm, tmem, warp, p.coff, NT, a.kv_first, q, abort);
+    CP_STAMP(threadIdx.x == 0, 5);  // partials sent
+    ok = wait_pushes(&sm.recv_full) && ok;
+    CP_STAMP(threadIdx.x == 0, 6);  // partials received
+    if (warp == 0) {
+      if (lane == 0) sm.target = ctr - ctr % kPerLaunch + kPerLaunch;
+      asm volatile("bar.sync 4, 96;" ::: "memory");  // the metadata is done
+      if (!ok && lane == 0) sm.abort = 1;
+      pool_and_finish(p, sm, a, ch0, q, ok && !*abort);
+    } else {
+      asm volatile("bar.sync 5, 160;" ::: "memory");  // the metadata is done
+      if (warp == 1)
+        for (int n = lane; n < p.n_out; n += 32)
+          if (sm.win[n].w < 0) *reinterpret_cast<uint2*>(p.out + (int64_t)n * p.D + ch0) = make_uint2(0u, 0u);
+      if (ok && !*abort) write_tails(p, sm, ch0, warp - 1);
+      if (!ok && lane == 0) sm.abort = 1;
+      CP_STAMP(threadIdx.x == 32, 14);  // tails written
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 7) {
     tc_fence_after();
     tmem_dealloc(tmem, tmem_cols);
   }
   if (threadIdx.x == 0 && sm.abort) atomicOr(p.err, kErrTimeout);
-  CP_STAMP(threadIdx.x == 0, 13);  // end
+  CP_STAMP(threadIdx.x == 0, 15);  // end
 }
 
 // x [T, H] as (column in block, row, 64-column block): a box of 64 columns x
-// box_rows rows x KPS blocks lands as KPS tiles [block][row][128 B].
-bool make_x_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows) {
+// box_rows rows x kps blocks lands as kps tiles [block][row][128 B].
+bool make_x_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows, int kps) {
   EncodeTiledFn f = encode_fn();
   if (!f) return false;
   const cuuint64_t dims[3] = {(cuuint64_t)BK, rows, cols / BK};
   const cuuint64_t strides[2] = {cols * 2, (cuuint64_t)BK * 2};
-  const cuuint32_t box[3] = {(cuuint32_t)BK, box_rows, (cuuint32_t)KPS};
+  const cuuint32_t box[3] = {(cuuint32_t)BK, box_rows, (cuuint32_t)kps};
   const cuuint32_t estr[3] = {1, 1, 1};
   return f(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -851,9 +906,9 @@ bool make_x_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, 
 // Both weight matrices [C, H] as one 5-D tensor: (column in block, row within a
 // half, half, matrix, 64-column block), the matrix stride being the distance
 // between the two allocations (the lower one first). A box of 64 columns x 16
-// rows x coff halves x 2 matrices x KPS blocks lands as KPS A tiles
+// rows x coff halves x 2 matrices x kps blocks lands as kps A tiles
 // [block][matrix][half][16 rows][128 B].
-bool make_w_map(CUtensorMap* m, const Params& p, int* kv_first) {
+bool make_w_map(CUtensorMap* m, const Params& p, int* kv_first, int kps) {
   EncodeTiledFn f = encode_fn();
   if (!f) return false;
   const uintptr_t a = reinterpret_cast<uintptr_t>(p.wkv), b = reinterpret_cast<uintptr_t>(p.wgate);
@@ -864,7 +919,7 @@ bool make_w_map(CUtensorMap* m, const Params& p, int* kv_first) {
   const cuuint64_t dims[5] = {(cuuint64_t)BK, (cuuint64_t)p.D, (cuuint64_t)p.coff, 2, (cuuint64_t)p.H / BK};
   const cuuint64_t strides[4] = {(cuuint64_t)p.H * 2, (cuuint64_t)p.D * p.H * 2, (cuuint64_t)delta,
                                  (cuuint64_t)BK * 2};
-  const cuuint32_t box[5] = {(cuuint32_t)BK, (cuuint32_t)GCH, (cuuint32_t)p.coff, 2, (cuuint32_t)KPS};
+  const cuuint32_t box[5] = {(cuuint32_t)BK, (cuuint32_t)GCH, (cuuint32_t)p.coff, 2, (cuuint32_t)kps};
   const cuuint32_t estr[5] = {1, 1, 1, 1, 1};
   return f(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, reinterpret_cast<void*>(lo), dims, strides, box, estr,
            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -927,35 +982,31 @@ int max_clusters(int (&conf)[64]) {
 
 bool decode_cp_supported(const Params& p) {
   if (p.T < 1 || p.T > 64 || p.B > kMaxSeqs || p.rotate || p.n_out > kMaxOut || p.rope != 64) return false;
-  if (p.coff * p.ratio > kMaxWinRows || p.H % (KQ * KPS * BK) || p.D % GCH || encode_fn() == nullptr)
+  if (p.coff * p.ratio > kMaxWinRows || p.H % (KQ * KPS * BK) || p.D % GCH || kMaxClusters % (p.D / GCH) ||
+      encode_fn() == nullptr)
     return false;
   CUtensorMap w;
   int kv_first = 0;
-  if (!make_w_map(&w, p, &kv_first)) return false;  // e.g. wkv and wgate at the same address
+  if (!make_w_map(&w, p, &kv_first, KPS)) return false;  // e.g. wkv and wgate at the same address
   const int dev = current_device();
   if (dev < 64 && g_disabled[dev]) return false;
   const int clusters = p.D / GCH;
-  if (kQuantum % (clusters * KQ)) return false;
   const int cap = p.T <= 32 ? max_clusters<32>(g_conf32) : max_clusters<64>(g_conf64);
   return cap >= clusters;
-}
-
-size_t decode_cp_workspace(const Params& p) {
-  return sizeof(float) * kReplicas * (size_t)(p.n_out > 0 ? p.n_out : 1) * (p.D / OWN);
 }
 
 // Launch. If the device refuses the launch form itself (a cooperative launch of
 // clusters), the path is disabled on this device and cudaErrorNotSupported is
 // returned before anything ran, so that the caller can take another path.
-cudaError_t launch_decode_cp(const Params& p, float* ss, void* counter, cudaStream_t s, bool unreachable) {
+cudaError_t launch_decode_cp(const Params& p, void* counter, void* xch, cudaStream_t s, bool unreachable) {
   const int NT = (p.T + 15) / 16 * 16;
-  CUtensorMap mx, mw;
   CpArgs a;
-  if (!make_x_map(&mx, p.x, p.T, p.H, (uint32_t)NT) || !make_w_map(&mw, p, &a.kv_first))
+  CUtensorMap mx, mw;
+  if (!make_x_map(&mx, p.x, p.T, p.H, (uint32_t)NT, KPS) || !make_w_map(&mw, p, &a.kv_first, KPS))
     return cudaErrorInvalidValue;
-  a.ss = ss;
   a.counter = static_cast<unsigned*>(counter);
-  a.bar_extra = unreachable ? kQuantum : 0u;
+  a.sums = static_cast<float*>(xch);
+  a.target_extra = unreachable ? kPerLaunch : 0u;
   const int grid = (p.D / GCH) * KQ;
   cudaLaunchAttribute attr[2];
   cudaError_t e;

@@ -75,7 +75,7 @@ struct Smem {
   int32_t row_w;                        // window of this CTA's output row, or -1
   int32_t nhist;                        // state rows 0..nhist-1 of the window are in hist_*, or -1
   float red[32];
-  float zs[512];
+  float zs[1024];  // 2 D floats: the Hadamard product's exchange buffers
   uint64_t full[S];
   uint64_t empty[S];
   uint64_t acc_full;

@@ -21,7 +21,7 @@ constexpr int kMaxStagedSeqs = 256;
 
 __global__ void __launch_bounds__(128) finish_kernel(Params p) {
   __shared__ float red[32];
-  __shared__ float zs[512];
+  __shared__ float zs[1024];  // 2 D floats: the Hadamard product's exchange buffers
   __shared__ int32_t off_s[kMaxStagedSeqs + 1];
   const int n = blockIdx.x;
   const int D = p.D, r = p.ratio;

@@ -47,7 +47,14 @@ struct Params {
   int32_t* m_tile; // [B+1] first fused work tile of each sequence (fused path), else null
   float* ystat;    // [n_out, coff, D] pooled halves (fused path)
   float* ylse;     // [n_out, coff, D] log-sum-exp of each half's scores (fused path, coff = 2)
+  int32_t* had_sylv;  // rotate: per kHadChunk entries of hadamard, 1 if they are those of
+                      // hadamard[0][0] * (Sylvester H_D) (the scheduler kernel checks), else 0;
+                      // null: not checked (the dense product is used)
 };
+
+// Entries of the hadamard matrix each checking CTA of the scheduler kernel covers.
+constexpr int kHadChunk = 65536;
+__host__ __device__ inline int had_chunks(int D) { return (D * D + kHadChunk - 1) / kHadChunk; }
 
 // Largest b in [0, n] with a[b] <= v, for a non-decreasing a[0..n] with a[0] <= v.
 __device__ __forceinline__ int upper_index(const int32_t* __restrict__ a, int n, int v) {

@@ -44,7 +44,7 @@ constexpr int kMaxTokens = 64;  // the decode projection kernel's limit
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kScratchBytes];
 
 struct ScratchLayout {
-  size_t err, m_cu, m_s, m_off, proj, total;
+  size_t err, m_cu, m_s, m_off, had, proj, total;
 };
 
 ScratchLayout scratch_layout(int64_t B, int64_t T, int64_t C) {
@@ -59,6 +59,7 @@ ScratchLayout scratch_layout(int64_t B, int64_t T, int64_t C) {
   L.m_cu = take(sizeof(int32_t) * (B + 1));
   L.m_s = take(sizeof(int32_t) * (B > 0 ? B : 1));
   L.m_off = take(sizeof(int32_t) * (B + 1));
+  L.had = take(sizeof(int32_t) * 16);  // the scheduler's verdicts on the hadamard matrix
   L.proj = take(sizeof(float) * (size_t)T * 2 * C);
   L.total = o;
   return L;
@@ -181,6 +182,7 @@ extern "C" int cmp_compressor_noalloc(const cmp_bf16* x, float* kv_state, float*
   p.m_s = reinterpret_cast<int32_t*>(ws + L.m_s);
   p.m_off = reinterpret_cast<int32_t*>(ws + L.m_off);
   p.proj = reinterpret_cast<float*>(ws + L.proj);
+  p.had_sylv = p.rotate ? reinterpret_cast<int32_t*>(ws + L.had) : nullptr;
 
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (cmp::launch_sched(p, s) != cudaSuccess) return CMP_ERR_CUDA;

@@ -11,15 +11,69 @@ namespace cmp {
 
 constexpr float kRmsEps = 1e-6f;
 
+// Whether the scheduler kernel found the hadamard matrix to be hadamard[0][0]
+// times the Sylvester matrix H_D (every checked chunk passed). Same answer in
+// every thread of a call.
+__device__ __forceinline__ bool hadamard_is_sylvester(const Params& p) {
+  if (!p.rotate || !p.had_sylv) return false;
+  bool ok = true;
+  for (int i = 0; i < had_chunks(p.D); ++i) ok = ok && p.had_sylv[i] != 0;
+  return ok;
+}
+
+// z @ (c * H_D) for the D values of a row held 4 per thread (thread t of the
+// first D/4: channels 4t .. 4t+3), with the fast Walsh-Hadamard transform in
+// natural order: for every bit b of the channel index, the pair (i, i + 2^b)
+// with bit b clear in i becomes (u + v, u - v); entry (k, j) of the product of
+// those butterflies is (-1)^popcount(k & j), which is H_D. Bits 0-1 are inside
+// a thread, 2-6 across the lanes of a warp (shuffles), 7-8 (D = 512) across
+// warps through shared memory (xs: 2 D floats, two barriers, which every
+// thread of the CTA takes). The result is scaled by c.
+__device__ __forceinline__ void fwht_row(float (&z)[4], int D, bool active, float* xs, float c) {
+  const float a0 = z[0] + z[1], a1 = z[0] - z[1], a2 = z[2] + z[3], a3 = z[2] - z[3];
+  z[0] = a0 + a2;
+  z[1] = a1 + a3;
+  z[2] = a0 - a2;
+  z[3] = a1 - a3;
+  const int lane = threadIdx.x & 31;
+#pragma unroll
+  for (int m = 1; m < 32; m <<= 1) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float v = __shfl_xor_sync(0xffffffffu, z[i], m);
+      z[i] = (lane & m) ? v - z[i] : z[i] + v;
+    }
+  }
+  if (D > 128) {
+    const int c0 = threadIdx.x * 4;
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {  // index bits 7, 8 = bits 0, 1 of the warp
+      const int m = 128 << r;
+      float* buf = xs + r * D;
+      if (active) *reinterpret_cast<float4*>(buf + c0) = make_float4(z[0], z[1], z[2], z[3]);
+      __syncthreads();
+      if (active) {
+        const float4 v = *reinterpret_cast<const float4*>(buf + (c0 ^ m));
+        const float vv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) z[i] = (c0 & m) ? vv[i] - z[i] : z[i] + vv[i];
+      }
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < 4; ++i) z[i] *= c;
+}
+
 // Threads 0 .. D/4-1 of the CTA hold the pooled values y of channels
 // c = 4i .. 4i+3 of output row n (thread i); any further threads only take part
-// in the barriers. red: >= D/128 floats of shared memory, zs: >= D floats of
+// in the barriers. red: >= D/128 floats of shared memory, zs: >= 2 D floats of
 // shared memory. Every thread of the CTA must call it.
 __device__ __forceinline__ void finish_row(const Params& p, int n, int c, const float (&y)[4], float* red,
                                            float* zs) {
   const int D = p.D;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = D / 128;
   const bool active = (int)threadIdx.x < D / 4;
+  const bool sylv = hadamard_is_sylvester(p);
   // RMSNorm over the D channels of the row
   float ss = active ? y[0] * y[0] + y[1] * y[1] + y[2] * y[2] + y[3] * y[3] : 0.f;
 #pragma unroll
@@ -29,8 +83,13 @@ __device__ __forceinline__ void finish_row(const Params& p, int n, int c, const 
   float tot = 0.f;
   for (int i = 0; i < nwarps; ++i) tot += red[i];
   const float inv = rsqrtf(tot / (float)D + kRmsEps);
-  if (!active) {
-    if (p.rotate) __syncthreads();  // the Hadamard product's barrier
+  if (!active) {  // the Hadamard product's barriers
+    if (sylv) {
+      float z[4] = {0.f, 0.f, 0.f, 0.f};
+      if (D > 128) fwht_row(z, D, false, zs, 0.f);
+    } else if (p.rotate) {
+      __syncthreads();
+    }
     return;
   }
   const uint2 wraw = *reinterpret_cast<const uint2*>(p.norm_w + c);
@@ -56,7 +115,9 @@ __device__ __forceinline__ void finish_row(const Params& p, int n, int c, const 
     }
   }
 
-  if (p.rotate) {  // out = z @ hadamard (dense product, any D x D matrix)
+  if (sylv) {  // out = z @ hadamard with hadamard = c * H_D: the fast transform
+    fwht_row(z, D, true, zs, __bfloat162float(p.had[0]));
+  } else if (p.rotate) {  // out = z @ hadamard (dense product, any D x D matrix)
 #pragma unroll
     for (int i = 0; i < 4; ++i) zs[c + i] = z[i];
     __syncthreads();

@@ -4,6 +4,9 @@
 // host synchronisation; this is the role the value-dependent AICPU scheduler
 // plays on "NPU DeepSeek-V4 Ascend C 融合算子优化" (AICPU Scheduler).
 //
+// With rotation it also checks, once per call, whether the hadamard matrix is
+// a scaled Sylvester matrix (classify_hadamard).
+//
 // Output-row layout ("CANN PyPTO 算子实战", 返回值说明 fixes only the row count
 // min(T, T//ratio + B)): sequence b reserves cap_b = min(L_b, L_b / ratio + 1)
 // rows after those of sequences 0..b-1. A sequence covering positions [s, e)
@@ -42,11 +45,39 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int* warp_tot, int* t
   return r;
 }
 
+// CTAs 1.. of a rotating call: is the hadamard matrix c * H_D in natural
+// Sylvester order, c = hadamard[0][0]? Entry (k, j) of H_D is
+// (-1)^popcount(k & j), so its bf16 pattern must be c's with the sign bit
+// flipped by the parity of popcount(k & j). Each CTA checks kHadChunk entries
+// and writes its verdict; the pooling kernels use the in-register fast
+// Walsh-Hadamard transform only if every chunk passed.
+__device__ void classify_hadamard(const Params& p, int chunk) {
+  const int D = p.D;
+  const int64_t lo = (int64_t)chunk * kHadChunk;
+  const int64_t hi = min((int64_t)D * D, lo + kHadChunk);
+  const uint16_t* h = reinterpret_cast<const uint16_t*>(p.had);
+  const uint32_t c = __ldg(h);
+  bool ok = true;
+  for (int64_t e = lo + threadIdx.x * 4; e < hi; e += kThreads * 4) {  // 4 entries of one row
+    const uint2 v = __ldg(reinterpret_cast<const uint2*>(h + e));
+    const int k = (int)(e / D), j0 = (int)(e % D);
+    const uint32_t got[4] = {v.x & 0xFFFFu, v.x >> 16, v.y & 0xFFFFu, v.y >> 16};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) ok = ok && got[i] == (c ^ ((uint32_t)(__popc(k & (j0 + i)) & 1) << 15));
+  }
+  ok = __syncthreads_and(ok);
+  if (threadIdx.x == 0) p.had_sylv[chunk] = ok ? 1 : 0;
+}
+
 __global__ void __launch_bounds__(kThreads) sched_kernel(Params p) {
   __shared__ int bad;
   __shared__ int warp_tot[32];
   __shared__ int chunk_total;
   pdl_trigger();  // the projection kernel may start streaming its inputs now
+  if (blockIdx.x > 0) {
+    classify_hadamard(p, blockIdx.x - 1);
+    return;
+  }
   if (threadIdx.x == 0) bad = 0;
   __syncthreads();
   const int B = p.B;
@@ -103,7 +134,8 @@ __global__ void __launch_bounds__(kThreads) sched_kernel(Params p) {
 }  // namespace
 
 cudaError_t launch_sched(const Params& p, cudaStream_t s) {
-  sched_kernel<<<1, kThreads, 0, s>>>(p);
+  const int grid = 1 + ((p.rotate && p.had_sylv) ? had_chunks(p.D) : 0);
+  sched_kernel<<<grid, kThreads, 0, s>>>(p);
   return cudaGetLastError();
 }
 

@@ -191,6 +191,40 @@ def test_dense_rotation_with_any_matrix(lib):
     check(lib, with_rope(inp))
 
 
+def _rotation(kind, D):
+    """hadamard matrices for the rotation tests: the Sylvester matrix with other
+    scales (the fast transform applies), and ones that are not scaled Sylvester
+    matrices (the dense product applies)."""
+    from workloads import sylvester
+    h = sylvester(D).astype(np.float32)
+    if kind == "sylvester":
+        return bf16_bits(h / np.float32(np.sqrt(D)))
+    if kind == "scaled_quarter":
+        return bf16_bits(h * np.float32(0.25))
+    if kind == "negated":
+        return bf16_bits(-h / np.float32(np.sqrt(D)))
+    if kind == "one_sign_off":       # one entry's sign flipped: not a Sylvester matrix
+        h[77, 3] = -h[77, 3]
+        return bf16_bits(h / np.float32(np.sqrt(D)))
+    if kind == "rows_swapped":       # a Hadamard matrix, but not in Sylvester order
+        h[[5, 9]] = h[[9, 5]]
+        return bf16_bits(h / np.float32(np.sqrt(D)))
+    raise KeyError(kind)
+
+
+@pytest.mark.parametrize("kind", ["sylvester", "scaled_quarter", "negated", "one_sign_off", "rows_swapped"])
+@pytest.mark.parametrize("D", [128, 512])
+def test_rotation_by_sylvester_and_other_matrices(lib, proj_kernel, kind, D):
+    """The scheduler kernel classifies the hadamard matrix once per call; a scaled
+    Sylvester matrix takes the in-register fast Walsh-Hadamard transform (across
+    lanes for D = 128, and across warps too for D = 512), any other matrix the
+    dense product. Both must match the oracle's dense product."""
+    inp = make_inputs(name="rotk", seed=D + len(kind), lengths=[40, 21], start_pos=[0, 6], H=1024, D=D,
+                      coff=2, ratio=4, block_size=16, rotate=True)
+    inp = dataclasses.replace(inp, hadamard=_rotation(kind, D))
+    check(lib, with_rope(inp))
+
+
 def test_empty_and_noop_calls(lib):
     import torch
     inp = with_rope(make_inputs(name="e", seed=1, lengths=[0, 0], start_pos=[3, 4], H=512, D=128,
@@ -335,10 +369,10 @@ def test_output_within_tolerance_of_both_rounding_readings(lib, case):
 
 def test_barrier_timeout_is_reported_and_the_next_call_recovers(lib):
     """Failure detection without a GPU fault: a testing knob makes one launch of
-    the channel-group decode kernel wait at its grid barrier for a count no
-    arrival reaches. Every CTA's bounded wait gives up after about a second, the
-    call reports CMP_ERR_TIMEOUT, get_error resets the barrier words, and the
-    next call runs normally and matches the oracle."""
+    the channel-group decode kernel wait for exchange words of an epoch no CTA
+    publishes. Every CTA's bounded wait gives up after about a second, the call
+    reports CMP_ERR_TIMEOUT, get_error resets the exchange words, and the next
+    call runs normally and matches the oracle."""
     import time
     inp = with_rope(make_config("c4a_decode"))
     prev = lib.set_proj_kernel(6)
