@@ -20,7 +20,8 @@ bool decode_fused_supported(const Params& p);
 size_t decode_fused_workspace(const Params& p);
 cudaError_t launch_decode_fused(const Params& p, float* part, void* bar, cudaStream_t s);
 bool decode_cp_supported(const Params& p);
-cudaError_t launch_decode_cp(const Params& p, void* counter, void* xch, cudaStream_t s, bool unreachable);
+cudaError_t launch_decode_cp(const Params& p, void* counter, void* xch, void* u, cudaStream_t s,
+                             bool unreachable);
 cudaError_t launch_nsa(const NsaParams& p, cudaStream_t s);
 cudaError_t launch_nsa_scan(const NsaParams& p, cudaStream_t s);
 int noalloc_take_error(int dev, unsigned* word);
@@ -36,12 +37,14 @@ using cmp::Params;
 // The first kHeaderBytes (zeroed when the workspace is created, and after a
 // timeout) hold the error word at offset 0, the K-split decode kernel's
 // grid-barrier words at offset 64, the channel-group decode kernel's arrival
-// counter at offset 256 and its CTAs' sums (64 windows x 128 CTAs x 4 bytes)
-// from offset 4096; only those kernels write there.
+// counter at offset 256, its CTAs' sums (64 windows x 128 CTAs x 4 bytes) from
+// offset 4096 and, for the rotation, every channel's u (64 windows x 512 x 4
+// bytes) after them; only those kernels write there.
 constexpr size_t kGridBarOffset = 64;
 constexpr size_t kCounterOffset = 256;
 constexpr size_t kExchangeOffset = 4096;
-constexpr size_t kHeaderBytes = kExchangeOffset + 64 * 128 * 4;
+constexpr size_t kRotateOffset = kExchangeOffset + 64 * 128 * 4;
+constexpr size_t kHeaderBytes = kRotateOffset + 64 * 512 * 4;
 
 size_t zeroed_bytes() { return kHeaderBytes; }
 
@@ -265,11 +268,12 @@ int run_path(Params& p, int which, cudaStream_t s) {
   if (which == 6) {  // decode: one cooperative kernel of clusters, no scheduler launch
     void* counter = ws + L.err + kCounterOffset;
     void* xch = ws + L.err + kExchangeOffset;
+    void* urow = ws + L.err + kRotateOffset;
     bool unreachable = false;  // the timeout test's knob, consumed one launch at a time
     for (int v = g_unreachable_barrier.load(); v > 0 && !unreachable;)
       unreachable = g_unreachable_barrier.compare_exchange_weak(v, v - 1);
     const cudaError_t e = launch(CMP_KERNEL_DECODE_CP, s,
-                                 [&] { return cmp::launch_decode_cp(p, counter, xch, s, unreachable); });
+                                 [&] { return cmp::launch_decode_cp(p, counter, xch, urow, s, unreachable); });
     if (e == cudaErrorNotSupported) return kRetryOtherPath;
     return e == cudaSuccess ? CMP_OK : CMP_ERR_CUDA;
   }

@@ -1,5 +1,5 @@
 // Decode by channel groups, in one cooperative kernel of 4-CTA clusters
-// (T <= 64 tokens, B <= 256 sequences, no Hadamard rotation).
+// (T <= 64 tokens, B <= 256 sequences).
 //
 // The per-channel softmax pooling ("compressor torch_extension API", 计算公式
 // 3-5) never mixes channels, so a cluster that holds the complete projections
@@ -20,15 +20,20 @@
 // that owns the channel (st.async into its shared memory, completing on its
 // mbarrier); each owner adds the four partials in rank order.
 //
-// Pooling and RMSNorm. Warp 0 pools its 4 channels of every window the call
-// completes (the windows' state rows were pre-reduced per channel while the
-// weights streamed, so only this call's rows remain), stores the windows' sums
-// of squares over its channels to global memory and arrives (release) at a
-// counter. Every CTA waits (acquire, bounded) until all CTAs have arrived, reads
-// every CTA's sums at once, adds them in a fixed order for the RMSNorm ("CANN PyPTO 算子实战", 压缩窗口与状态更新: rms_norm over the D
-// channels), scales its channels, applies norm_weight and the interleaved RoPE
-// (a pair never straddles two CTAs) and stores bf16. Warps 1-3 meanwhile write
-// the state tails.
+// Pooling and RMSNorm. Warps 0-3 pool this CTA's 4 channels of every window
+// the call completes (the windows' state rows were pre-reduced per channel
+// while the weights streamed, so only this call's rows remain). Warp 0 then
+// stores the windows' sums of squares over its channels to global memory and
+// arrives (release) at a counter, waits (acquire, bounded) until all CTAs have
+// arrived and reads every CTA's sums at once, while warps 1-3 write the state
+// tails. Warps 0-3 add the sums in a fixed order for the RMSNorm ("CANN PyPTO
+// 算子实战", 压缩窗口与状态更新: rms_norm over the D channels), scale their
+// channels, apply norm_weight and the interleaved RoPE (a pair never straddles
+// two CTAs) and store bf16. With the Hadamard rotation the exchange also
+// carries each CTA's u = RoPE(y * norm_weight) for its channels; the RMSNorm
+// scale commutes with the product, so every CTA forms its own output columns
+// as scale * (u @ hadamard[:, its channels]) from all D values of u ("CANN
+// PyPTO 算子实战", kernel 派发逻辑: out @ hadamard).
 //
 // Warps 4-5 compute the call's metadata (what the varlen scheduler kernel does
 // on the other paths) and prefetch what the later steps read: the state rows
@@ -125,6 +130,7 @@ struct Smem {
   alignas(16) float4 hst[kMaxOut][OWN];          // per window and channel: the state rows' running
                                                  // max, exp-sum and weighted sum
   float norm[OWN];
+  float hcol[512][OWN];     // rotation: this CTA's columns of the hadamard matrix
   TokInfo tok[MAXT];
   Win win[kMaxOut];
   int32_t cu[kMaxSeqs + 1];
@@ -220,6 +226,17 @@ __device__ __forceinline__ void tma_load_5d(void* dst, const CUtensorMap* map, u
       : "memory");
 }
 
+// Interleaved RoPE on 4 consecutive channels (pairs (2j, 2j+1) of the last
+// rope channels; t: per pair cos even, cos odd, sin even, sin odd).
+__device__ __forceinline__ void rope4(float (&z)[4], const float* t) {
+#pragma unroll
+  for (int u = 0; u < 2; ++u) {
+    const float ev = z[2 * u], od = z[2 * u + 1];
+    z[2 * u] = ev * t[4 * u + 0] - od * t[4 * u + 2];
+    z[2 * u + 1] = od * t[4 * u + 1] + ev * t[4 * u + 3];
+  }
+}
+
 __device__ __forceinline__ float4 add4(float4 a, float4 b) {
   return make_float4(a.x + b.x, a.y + b.y, a.z + b.z, a.w + b.w);
 }
@@ -227,6 +244,7 @@ __device__ __forceinline__ float4 add4(float4 a, float4 b) {
 struct CpArgs {
   unsigned* counter;  // the CTAs' arrivals (zeroed at creation)
   float* sums;        // [window list entry][CTA]: each CTA's sums of squares
+  float* u;           // rotation: [window list entry][channel]: RoPE(y * norm_weight) of every channel
   int kv_first;       // the 5-D weight map holds wkv before wgate (else the other way round)
   uint32_t target_extra;  // added to the count the CTAs wait for: kPerLaunch makes it unreachable
                           // (timeout test)
@@ -299,6 +317,15 @@ __device__ void call_metadata(const Params& p, Smem<MAXT>& sm, int NT, int ch0) 
     rp[2] = __ldg(reinterpret_cast<const unsigned int*>(sn + j0));
     rp[3] = __ldg(reinterpret_cast<const unsigned int*>(sn + hr + j0));
   }
+  // rotation: this CTA's 4 columns of the hadamard matrix, rows et, et + 64, ...
+  uint2 hv[8];
+  if (p.rotate) {
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int k = et + 64 * u;
+      hv[u] = k < p.D ? __ldg(reinterpret_cast<const uint2*>(p.had + (int64_t)k * p.D + ch0)) : make_uint2(0u, 0u);
+    }
+  }
   // these loads are issued: let the weight stream start behind them
   asm volatile("bar.arrive 3, 96;" ::: "memory");
 #pragma unroll
@@ -311,6 +338,20 @@ __device__ void call_metadata(const Params& p, Smem<MAXT>& sm, int NT, int ch0) 
   for (int u = 0; u < 2; ++u)
     if (et + 64 * u < rows) *reinterpret_cast<float4*>(&sm.ape[et + 64 * u][0]) = apev[u];
   if (et < OWN) sm.norm[et] = normv;
+  if (p.rotate) {
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int k = et + 64 * u;
+      if (k < p.D) {
+        const __nv_bfloat162 h01 = *reinterpret_cast<const __nv_bfloat162*>(&hv[u].x);
+        const __nv_bfloat162 h23 = *reinterpret_cast<const __nv_bfloat162*>(&hv[u].y);
+        sm.hcol[k][0] = __low2float(h01);
+        sm.hcol[k][1] = __high2float(h01);
+        sm.hcol[k][2] = __low2float(h23);
+        sm.hcol[k][3] = __high2float(h23);
+      }
+    }
+  }
   if (roped && et < p.n_out) {
     float* d = sm.rope[et];
 #pragma unroll
@@ -380,19 +421,28 @@ __device__ void call_metadata(const Params& p, Smem<MAXT>& sm, int NT, int ch0) 
       ttail = tpos >= tail_threshold(s + (sm.cu[lo + 1] - sm.cu[lo]), r, p.coff);
     }
   }
-  // the windows the call completes: rows off[b] .. off[b] + (e/r - s/r) - 1
-  for (int b = et; b < B && !rejected; b += 64) {
-    const int s = sm.sp[b], cu = sm.cu[b], e = s + (sm.cu[b + 1] - cu);
-    for (int k = 0; k < e / r - s / r; ++k) {
-      const int w = s / r + k;
-      Win wi;
-      wi.w = w;
-      wi.b = b;
-      wi.s = s;
-      wi.cu = cu;
-      wi.hrows = max(0, min(rows, s - window_pos(w, 0, r, p.coff)));
-      wi.hist = -1;
-      sm.win[sm.off[b] + k] = wi;
+  // the window of output row n = et (n_out <= 64): the sequence b whose rows
+  // off[b] .. off[b+1]-1 hold it, its k-th completed window if k < e/r - s/r
+  if (et < p.n_out && !rejected) {
+    int lo = 0, hi = B;
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (sm.off[mid] <= et) lo = mid; else hi = mid - 1;
+    }
+    if (lo < B) {
+      const int b = lo, k = et - sm.off[b];
+      const int s = sm.sp[b], cu = sm.cu[b], e = s + (sm.cu[b + 1] - cu);
+      if (k < e / r - s / r) {
+        const int w = s / r + k;
+        Win wi;
+        wi.w = w;
+        wi.b = b;
+        wi.s = s;
+        wi.cu = cu;
+        wi.hrows = max(0, min(rows, s - window_pos(w, 0, r, p.coff)));
+        wi.hist = -1;
+        sm.win[et] = wi;
+      }
     }
   }
   asm volatile("bar.sync 2, 64;" ::: "memory");
@@ -641,28 +691,34 @@ __device__ void write_tails(const Params& p, const Smem<MAXT>& sm, int ch0, int 
   }
 }
 
-// Warp 0, once the partials have landed and the metadata is done: pool,
-// exchange the windows' sums of squares (every CTA stores its sums and arrives
-// at the counter, waits for all arrivals and reads every CTA's sums), then
-// RMSNorm, norm_weight, RoPE and the bf16 store of this CTA's channels.
+__device__ __forceinline__ void epi_sync() { asm volatile("bar.sync 7, 128;" ::: "memory"); }
+
+// Warps 0-3 (128 threads), once the partials have landed and the metadata is
+// done: pool this CTA's 4 channels of every window the call completes. Two
+// threads per (window, channel) take alternate rows of this call (the state
+// rows come pre-reduced) and merge; the windows' sums of squares over the 4
+// channels go to ss_own, RoPE(y * norm_weight) of a rotating call to ybuf.
 template <int MAXT>
-__device__ void pool_and_finish(const Params& p, Smem<MAXT>& sm, const CpArgs& a, int ch0, uint32_t q,
-                                bool ok) {
-  const int lane = threadIdx.x & 31;
-  const int r = p.ratio, rows = p.coff * r;
-  const int nw = sm.n_win;
-  // ---- pooling: lane = 4 * (window mod 8) + channel; the state rows come pre-reduced ----
-  for (int base = 0; base < nw; base += 8) {
-    const int i = base + (lane >> 2), c = lane & 3;
+__device__ void pool_windows(const Params& p, Smem<MAXT>& sm, int ch0, bool ok) {
+  const int tid = threadIdx.x;  // 0..127
+  const int r = p.ratio, rows = p.coff * r, nw = sm.n_win;
+  for (int base = 0; base < nw * OWN * 2; base += 128) {
+    const int u = (base + tid) >> 1, side = tid & 1;
+    const int i = u / OWN, c = u % OWN;
     const bool live = i < nw;
     float y = 0.f;
     int n = 0;
+    float m = -INFINITY, l = 0.f, acc = 0.f;
     if (live) {
       n = sm.wlist[i];
       const Win w = sm.win[n];
-      const float4 h = sm.hst[i][c];
-      float m = h.x, l = h.y, acc = h.z;
-      for (int j = w.hrows; j < rows && ok; ++j) {  // this call's rows
+      if (side == 0) {
+        const float4 h = sm.hst[i][c];
+        m = h.x;
+        l = h.y;
+        acc = h.z;
+      }
+      for (int j = w.hrows + side; j < rows && ok; j += 2) {  // this call's rows
         const int h = (p.coff == 2 && j >= r) ? 1 : 0;
         const int t = w.cu + (window_pos(w.w, j, r, p.coff) - w.s);
         const float kv = own_value(sm, h, 0, c, t);
@@ -673,24 +729,59 @@ __device__ void pool_and_finish(const Params& p, Smem<MAXT>& sm, const CpArgs& a
         acc = acc * f + e * kv;
         m = mn;
       }
-      y = (ok && l > 0.f) ? __fdividef(acc, l) : 0.f;
-      sm.ybuf[n][c] = y;
     }
-    // the window's sum of squares over this CTA's 4 channels (lanes 4i' .. 4i'+3)
-    float s = y * y;
-    s += __shfl_xor_sync(0xffffffffu, s, 1);
+    {  // merge the two sides
+      const float m2 = __shfl_xor_sync(0xffffffffu, m, 1);
+      const float l2 = __shfl_xor_sync(0xffffffffu, l, 1);
+      const float a2 = __shfl_xor_sync(0xffffffffu, acc, 1);
+      const float mn = fmaxf(m, m2);
+      const float f1 = m == -INFINITY ? 0.f : __expf(m - mn);
+      const float f2 = m2 == -INFINITY ? 0.f : __expf(m2 - mn);
+      l = l * f1 + l2 * f2;
+      acc = acc * f1 + a2 * f2;
+    }
+    y = (live && ok && l > 0.f) ? __fdividef(acc, l) : 0.f;
+    if (live && side == 0) sm.ybuf[n][c] = y;
+    // the window's sum of squares over the 4 channels (threads 8i' .. 8i'+7)
+    float s = side == 0 ? y * y : 0.f;
     s += __shfl_xor_sync(0xffffffffu, s, 2);
-    if (live && c == 0) sm.ss_own[i] = s;
+    s += __shfl_xor_sync(0xffffffffu, s, 4);
+    if (live && (tid & 7) == 0) sm.ss_own[i] = s;
   }
-  warp_sync_all();
-  // ---- this CTA's sums of squares to global memory, then its arrival (release) ----
+  epi_sync();
+  if (p.rotate) {  // u = RoPE(y * norm_weight) of this CTA's channels, per window
+    const bool roped = ch0 >= p.D - p.rope;
+    for (int i = tid; i < nw; i += 128) {
+      const int n = sm.wlist[i];
+      float z[OWN];
+#pragma unroll
+      for (int c = 0; c < OWN; ++c) z[c] = sm.ybuf[n][c] * sm.norm[c];
+      if (roped) rope4(z, sm.rope[n]);
+      *reinterpret_cast<float4*>(&sm.ybuf[n][0]) = make_float4(z[0], z[1], z[2], z[3]);
+    }
+    epi_sync();
+  }
+}
+
+// Warp 0: exchange the windows' sums of squares (and, rotating, u) with every
+// CTA: this CTA's go to global memory, one lane arrives (release) at the
+// counter, waits (acquire) for all arrivals, and the warp reads every CTA's sums
+// (weak loads that bypass L1, all in flight at once) and adds them in a fixed
+// order into ss_tot.
+template <int MAXT>
+__device__ void exchange_sums(const Params& p, Smem<MAXT>& sm, const CpArgs& a, int ch0) {
+  const int lane = threadIdx.x & 31;
+  const int nw = sm.n_win;
   if (lane == 0) {
-    for (int i = 0; i < nw; ++i) a.sums[(int64_t)i * kMaxCtas + blockIdx.x] = sm.ss_own[i];
+    for (int i = 0; i < nw; ++i) {
+      a.sums[(int64_t)i * kMaxCtas + blockIdx.x] = sm.ss_own[i];
+      if (p.rotate)
+        *reinterpret_cast<float4*>(a.u + (int64_t)i * 512 + ch0) =
+            *reinterpret_cast<const float4*>(&sm.ybuf[sm.wlist[i]][0]);
+    }
     arrive_release(a.counter, kPerLaunch / gridDim.x);
   }
   CP_STAMP(lane == 0, 7);  // pooled, arrived
-  // ---- every CTA's sums once all have arrived: acquire polls by one lane, then
-  // weak loads that bypass L1 (all in flight at once), added in a fixed order ----
   int got = 1;
   if (lane == 0) {
     const uint32_t target = sm.target + a.target_extra;
@@ -729,25 +820,71 @@ __device__ void pool_and_finish(const Params& p, Smem<MAXT>& sm, const CpArgs& a
   }
   warp_sync_all();
   CP_STAMP(lane == 0, 9);  // exchange complete
-  // ---- RMSNorm scale, norm_weight, RoPE, bf16 store ----
+}
+
+// Warps 0-3: RMSNorm scale, norm_weight, RoPE and the bf16 store of this CTA's
+// channels of every window row; with the rotation, output column ch0 + c of a
+// window is scale * sum_k u[k] * hadamard[k][ch0 + c], one thread per (window,
+// column) adding over k in order (four interleaved partial sums).
+template <int MAXT>
+__device__ void finish_rows(const Params& p, Smem<MAXT>& sm, const CpArgs& a, int ch0, bool ok) {
+  const int tid = threadIdx.x;
+  const int nw = sm.n_win;
   const bool fin = ok && sm.xch_ok != 0;
+  if (p.rotate) {
+    // every window's u (all D channels, published before the arrivals) into
+    // the now idle A ring, rows padded by one float; 8 loads in flight per thread
+    float* uall = reinterpret_cast<float*>(&sm.a[0][0]);
+    if (fin) {
+      const int n4 = nw * p.D / 4;
+      for (int v0 = 0; v0 < n4; v0 += 128 * 8) {
+        float4 x4[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const int v = v0 + tid + 128 * e;
+          if (v < n4)
+            x4[e] = __ldcg(reinterpret_cast<const float4*>(a.u + (int64_t)((4 * v) / p.D) * 512 + (4 * v) % p.D));
+        }
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const int v = v0 + tid + 128 * e;
+          if (v < n4) {
+            float* d = uall + ((4 * v) / p.D) * (p.D + 1) + (4 * v) % p.D;
+            d[0] = x4[e].x;
+            d[1] = x4[e].y;
+            d[2] = x4[e].z;
+            d[3] = x4[e].w;
+          }
+        }
+      }
+    }
+    epi_sync();
+    for (int u = tid; u < nw * OWN; u += 128) {
+      const int i = u / OWN, c = u % OWN;
+      float o = 0.f;
+      if (fin) {
+        const float* ui = uall + i * (p.D + 1);
+        float s4[4] = {0.f, 0.f, 0.f, 0.f};
+        for (int k = 0; k < p.D; k += 4) {
+#pragma unroll
+          for (int e = 0; e < 4; ++e) s4[e] = fmaf(ui[k + e], sm.hcol[k + e][c], s4[e]);
+        }
+        o = ((s4[0] + s4[1]) + (s4[2] + s4[3])) * rsqrtf(sm.ss_tot[i] / (float)p.D + 1e-6f);
+      }
+      p.out[(int64_t)sm.wlist[i] * p.D + ch0 + c] = __float2bfloat16_rn(o);
+    }
+    CP_STAMP(tid == 0, 10);  // rows stored
+    return;
+  }
   const bool roped = ch0 >= p.D - p.rope;
-  for (int i = lane; i < nw; i += 32) {
+  for (int i = tid; i < nw; i += 128) {
     const int n = sm.wlist[i];
     float z[OWN] = {0.f, 0.f, 0.f, 0.f};
     if (fin) {
       const float sc = rsqrtf(sm.ss_tot[i] / (float)p.D + 1e-6f);
 #pragma unroll
       for (int c = 0; c < OWN; ++c) z[c] = sm.ybuf[n][c] * sc * sm.norm[c];
-      if (roped) {  // interleaved RoPE: pairs (2j, 2j+1) of the last rope channels
-        const float* t = sm.rope[n];
-#pragma unroll
-        for (int u = 0; u < 2; ++u) {
-          const float ev = z[2 * u], od = z[2 * u + 1];
-          z[2 * u] = ev * t[4 * u + 0] - od * t[4 * u + 2];
-          z[2 * u + 1] = od * t[4 * u + 1] + ev * t[4 * u + 3];
-        }
-      }
+      if (roped) rope4(z, sm.rope[n]);
     }
     __nv_bfloat162 o01 = __floats2bfloat162_rn(z[0], z[1]);
     __nv_bfloat162 o23 = __floats2bfloat162_rn(z[2], z[3]);
@@ -756,7 +893,7 @@ __device__ void pool_and_finish(const Params& p, Smem<MAXT>& sm, const CpArgs& a
     v.y = *reinterpret_cast<uint32_t*>(&o23);
     *reinterpret_cast<uint2*>(p.out + (int64_t)n * p.D + ch0) = v;
   }
-  CP_STAMP(lane == 0, 10);  // rows stored
+  CP_STAMP(tid == 0, 10);  // rows stored
 }
 
 template <int MAXT>
@@ -850,11 +987,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ---- warps 4-5: metadata and prefetch ----
     call_metadata<MAXT>(p, sm, NT, ch0);
     CP_STAMP(threadIdx.x == kMetaBase, 4);  // metadata done
-    asm volatile("bar.arrive 4, 96;" ::: "memory");   // to warp 0
-    asm volatile("bar.arrive 5, 160;" ::: "memory");  // to warps 1-3
+    asm volatile("bar.arrive 4, 192;" ::: "memory");  // to warps 0-3
   } else {
-    // ---- warps 0-3: read-out; then warp 0 pools, exchanges and stores the rows,
-    // warps 1-3 write the state tails and the rows without a window ----
+    // ---- warps 0-3: read-out, pooling; then warp 0 exchanges the sums while
+    // warps 1-3 write the state tails and the rows without a window; then all
+    // four store the rows ----
     uint32_t ctr = 0;
     if (warp == 0) ctr = arrivals_now(a.counter);  // this launch's base (a cold load)
     cluster_wait();  // cluster barrier 0: every CTA of the cluster runs before a push
@@ -863,20 +1000,23 @@ __global__ void __launch_bounds__(kThreads, 1)
     CP_STAMP(threadIdx.x == 0, 5);  // partials sent
     ok = wait_pushes(&sm.recv_full) && ok;
     CP_STAMP(threadIdx.x == 0, 6);  // partials received
+    if (threadIdx.x == 0) sm.target = ctr - ctr % kPerLaunch + kPerLaunch;
+    asm volatile("bar.sync 4, 192;" ::: "memory");  // the metadata is done
+    if (!ok && lane == 0) sm.abort = 1;
+    epi_sync();
+    const bool good = !*abort;
+    pool_windows(p, sm, ch0, good);
     if (warp == 0) {
-      if (lane == 0) sm.target = ctr - ctr % kPerLaunch + kPerLaunch;
-      asm volatile("bar.sync 4, 96;" ::: "memory");  // the metadata is done
-      if (!ok && lane == 0) sm.abort = 1;
-      pool_and_finish(p, sm, a, ch0, q, ok && !*abort);
+      exchange_sums(p, sm, a, ch0);
     } else {
-      asm volatile("bar.sync 5, 160;" ::: "memory");  // the metadata is done
       if (warp == 1)
         for (int n = lane; n < p.n_out; n += 32)
           if (sm.win[n].w < 0) *reinterpret_cast<uint2*>(p.out + (int64_t)n * p.D + ch0) = make_uint2(0u, 0u);
-      if (ok && !*abort) write_tails(p, sm, ch0, warp - 1);
-      if (!ok && lane == 0) sm.abort = 1;
+      if (good) write_tails(p, sm, ch0, warp - 1);
       CP_STAMP(threadIdx.x == 32, 14);  // tails written
     }
+    epi_sync();
+    finish_rows(p, sm, a, ch0, good);
   }
 
   tc_fence_before();
@@ -981,7 +1121,9 @@ int max_clusters(int (&conf)[64]) {
 }  // namespace
 
 bool decode_cp_supported(const Params& p) {
-  if (p.T < 1 || p.T > 64 || p.B > kMaxSeqs || p.rotate || p.n_out > kMaxOut || p.rope != 64) return false;
+  if (p.T < 1 || p.T > 64 || p.B > kMaxSeqs || p.n_out > kMaxOut || p.rope != 64) return false;
+  // rotation: every window's u (n_out rows of D + 1 floats) fits in the A ring
+  if (p.rotate && (size_t)p.n_out * (p.D + 1) * 4 > sizeof(Smem<32>::a)) return false;
   if (p.coff * p.ratio > kMaxWinRows || p.H % (KQ * KPS * BK) || p.D % GCH || kMaxClusters % (p.D / GCH) ||
       encode_fn() == nullptr)
     return false;
@@ -998,7 +1140,8 @@ bool decode_cp_supported(const Params& p) {
 // Launch. If the device refuses the launch form itself (a cooperative launch of
 // clusters), the path is disabled on this device and cudaErrorNotSupported is
 // returned before anything ran, so that the caller can take another path.
-cudaError_t launch_decode_cp(const Params& p, void* counter, void* xch, cudaStream_t s, bool unreachable) {
+cudaError_t launch_decode_cp(const Params& p, void* counter, void* xch, void* u, cudaStream_t s,
+                             bool unreachable) {
   const int NT = (p.T + 15) / 16 * 16;
   CpArgs a;
   CUtensorMap mx, mw;
@@ -1006,6 +1149,7 @@ cudaError_t launch_decode_cp(const Params& p, void* counter, void* xch, cudaStre
     return cudaErrorInvalidValue;
   a.counter = static_cast<unsigned*>(counter);
   a.sums = static_cast<float*>(xch);
+  a.u = static_cast<float*>(u);
   a.target_extra = unreachable ? kPerLaunch : 0u;
   const int grid = (p.D / GCH) * KQ;
   cudaLaunchAttribute attr[2];

@@ -308,6 +308,35 @@ def test_decode_cp_cases(lib, name):
     assert launched["decode_cp"][1] == 1, launched
 
 
+DECODE_CP_ROTATE_CASES = {
+    # name: lengths, start_pos, D, H, ratio, block_size, hadamard kind
+    "c4li_decode_32way": ([1] * 32, [4 * k + 3 - (k % 4) for k in range(32)], 128, 7168, 4, 128, "sylvester"),
+    "c4li_tiny_one_sequence": ([64], [0], 128, 1024, 4, 16, "sylvester"),
+    "c4li_any_matrix": ([9, 7, 16], [3, 0, 21], 128, 2048, 4, 16, "one_sign_off"),
+    "d512_rotation": ([1] * 24, [4 * k + 3 for k in range(24)], 512, 2048, 4, 64, "scaled_quarter"),
+    "ratio8_rotation": ([13, 2, 31], [5, 6, 3], 128, 1024, 8, 16, "negated"),
+}
+
+
+@pytest.mark.parametrize("name", sorted(DECODE_CP_ROTATE_CASES))
+def test_decode_cp_with_rotation(lib, name):
+    """Path 6 with the Hadamard rotation: each CTA publishes RoPE(y * norm_weight)
+    of its channels and forms its output columns from all D of them."""
+    L, sp, D, H, ratio, bs, kind = DECODE_CP_ROTATE_CASES[name]
+    inp = make_inputs(name=name, seed=17, lengths=L, start_pos=sp, H=H, D=D,
+                      coff=2 if ratio == 4 else 1, ratio=ratio, block_size=bs, rotate=True,
+                      lookback=2 * ratio)
+    inp = with_rope(dataclasses.replace(inp, hadamard=_rotation(kind, D)))
+    prev = lib.set_proj_kernel(6)
+    try:
+        lib.profile_start()
+        check(lib, inp)
+        launched = lib.profile_stop()
+    finally:
+        lib.set_proj_kernel(prev)
+    assert launched["decode_cp"][1] == 1 and sum(n for _, n in launched.values()) == 1, launched
+
+
 def test_decode_cp_is_the_automatic_decode_path(lib):
     inp = with_rope(make_config("c4a_decode"))
     lib.profile_start()
