@@ -726,6 +726,43 @@ def run_decode_phases(args):
                       "workload": "c4a_decode: 32 requests x 1 token, H=4096, D=512, ratio 4"}), flush=True)
 
 
+def run_chunked_calls(args):
+    """--only chunked-calls: the c4li_chunked workload's 4 calls (state carried),
+    run eagerly `warmup` then `steps` times, with the library's per-kernel times
+    (for profiler captures of the projection and pooling kernels on that path;
+    the configs section times the same calls as graph replays)."""
+    import torch
+
+    import streaming_kv_cache_varlen_b200 as cmp
+    from workloads import make_chunked
+
+    device = torch.device("cuda", 0)
+    ch = make_chunked()
+    calls = [with_library_rope(c) for c in ch.calls]
+    first = device_args(calls[0], device)
+    steps_args = [first] + [device_args(c, device, first["kv_state"], first["score_state"]) for c in calls[1:]]
+    outs = [torch.empty((cmp.out_rows(c.B, c.T, c.ratio), c.D), dtype=torch.bfloat16, device=device)
+            for c in calls]
+
+    def step():
+        for a, o in zip(steps_args, outs):
+            cmp.compressor(**a, out=o)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    cmp.profile_start()
+    for _ in range(args.steps):
+        step()
+    prof = cmp.profile_stop()
+    assert cmp.get_error() == 0
+    print(json.dumps({"workload": "c4li_chunked: 8 requests x 4 calls of U[1, 2048] tokens, H=7168, D=128, "
+                                  "ratio 4, rotate", "steps": args.steps,
+                      "tokens_per_step": int(sum(c.T for c in calls)),
+                      "kernel_us": {k: ms / n * 1e3 for k, (ms, n) in prof.items() if n},
+                      "launches": {k: n for k, (ms, n) in prof.items() if n}}), flush=True)
+
+
 def run_ours(args):
     import torch
 
@@ -992,20 +1029,30 @@ def main():
                     help="tokens of the CPU-baseline sample (default: about --cpu-seconds of oracle work)")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--only", choices=("all", "prefill", "decode", "nsa", "configs", "decode-phases"),
+    ap.add_argument("--only", choices=("all", "prefill", "decode", "nsa", "configs", "decode-phases",
+                                       "chunked-calls"),
                     default="all",
                     help="run only one part (for profiler captures); decode-phases: the decode "
                          "kernel's timeline from the phase-stamp build of the library")
     ap.add_argument("--prefill-tokens", type=int, default=PREFILL["T"],
                     help="tokens of the prefill sequence (smaller cases for profiler captures)")
+    ap.add_argument("--path", type=int, default=0,
+                    help="the library's path knob (cmp_set_proj_kernel) for every call: 0 = automatic "
+                         "(the default); others force one path, for comparisons and captures")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
     PREFILL["T"] = args.prefill_tokens
+    if args.path and args.impl == "ours":
+        import streaming_kv_cache_varlen_b200 as cmp
+        if cmp.set_proj_kernel(args.path) < 0:
+            raise SystemExit(f"--path {args.path}: not a path of the library")
     if args.impl == "reference":
         run_reference(args)
     elif args.only == "decode-phases":
         run_decode_phases(args)
+    elif args.only == "chunked-calls":
+        run_chunked_calls(args)
     elif args.mode == "sharded":
         run_sharded(args)
     else:

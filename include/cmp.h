@@ -317,10 +317,11 @@ CMP_API int cmp_debug_phase_stamps(uint64_t* dst, int64_t n);
  * hold its clusters) the weight-streaming projection + pooling kernels, else
  * the K-split one-kernel decode; the fused tcgen05 pooling kernel for long
  * sequences, T >= 1024 and T >= 256*B, when its (T/256)*(C/128) work items
- * fill the SMs twice; else the tcgen05 projection + pooling kernel), 1 = force the mma.sync projection, 2 = the tcgen05 projection,
+ * fill the SMs twice; else the tcgen05 projection + pooling kernel), 1 = force the mma.sync projection, 2 = the tcgen05 projection
+ * (on CTA pairs, cta_group::2, where the device can co-schedule them),
  * 3 = weight streaming, 4 = the fused path, 5 = the K-split one-kernel decode,
- * 6 = the channel-group decode. A forced path a call cannot take falls back
- * to 1.
+ * 6 = the channel-group decode, 7 = the tcgen05 projection on single CTAs.
+ * A forced path a call cannot take falls back to 1.
  * Returns the previous value, or -1 if out of range. */
 CMP_API int cmp_set_proj_kernel(int which);
 

@@ -339,8 +339,9 @@ def debug_unreachable_barrier(launches: int) -> int:
 
 def set_proj_kernel(which: int) -> int:
     """Testing knob, which path calls take: 0 automatic, 1 mma.sync projection,
-    2 tcgen05 projection, 3 weight streaming, 4 fused tcgen05 pooling, 5 K-split
-    one-kernel decode, 6 channel-group one-kernel decode. Returns the previous value."""
+    2 tcgen05 projection (on CTA pairs where the device co-schedules them), 3 weight
+    streaming, 4 fused tcgen05 pooling, 5 K-split one-kernel decode, 6 channel-group
+    one-kernel decode, 7 tcgen05 projection on single CTAs. Returns the previous value."""
     return int(lib.cmp_set_proj_kernel(which))
 
 

@@ -39,12 +39,15 @@ using cmp::Params;
 // grid-barrier words at offset 64, the channel-group decode kernel's arrival
 // counter at offset 256, its CTAs' sums (64 windows x 128 CTAs x 4 bytes) from
 // offset 4096 and, for the rotation, every channel's u (64 windows x 512 x 4
-// bytes) after them; only those kernels write there.
+// bytes) after them, then the one-kernel fused path's per-tile arrival
+// counters (which that kernel puts back to zero); only those kernels write
+// there.
 constexpr size_t kGridBarOffset = 64;
 constexpr size_t kCounterOffset = 256;
 constexpr size_t kExchangeOffset = 4096;
 constexpr size_t kRotateOffset = kExchangeOffset + 64 * 128 * 4;
-constexpr size_t kHeaderBytes = kRotateOffset + 64 * 512 * 4;
+constexpr size_t kTileCntOffset = kRotateOffset + 64 * 512 * 4;
+constexpr size_t kHeaderBytes = kTileCntOffset + cmp::kFusedTileCounters * 4;
 
 size_t zeroed_bytes() { return kHeaderBytes; }
 
@@ -285,9 +288,15 @@ int run_path(Params& p, int which, cudaStream_t s) {
       return CMP_ERR_CUDA;
     return CMP_OK;
   }
+  cudaError_t e;
+  if (fused && cmp::fused_fold_supported(p)) {  // one kernel: metadata and row finish inside
+    p.tile_cnt = reinterpret_cast<unsigned*>(ws + L.err + kTileCntOffset);
+    const int sms = sm_count_cached();
+    e = launch(CMP_KERNEL_FUSED, s, [&] { return cmp::launch_fused(p, s, sms); });
+    return e == cudaSuccess ? CMP_OK : CMP_ERR_CUDA;
+  }
   if (launch(CMP_KERNEL_SCHED, s, [&] { return cmp::launch_sched(p, s); }) != cudaSuccess)
     return CMP_ERR_CUDA;
-  cudaError_t e;
   if (fused) {
     const int sms = sm_count_cached();
     e = launch(CMP_KERNEL_FUSED, s, [&] { return cmp::launch_fused(p, s, sms); });
@@ -356,7 +365,8 @@ size_t cmp_workspace_size(const cmp_dims* dims, int32_t ratio) {
   p.coff = coff;
   p.ratio = ratio;
   p.n_out = (int)cmp_out_rows(p.B, p.T, ratio);
-  const int which = choose_path(p, g_proj_kernel.load());
+  const int knob = g_proj_kernel.load();
+  const int which = choose_path(p, knob == 7 ? 2 : knob);
   return ws_layout(dims->B, dims->T, p.C, p.n_out, which == 4, decode_part_bytes(p, which)).total +
          cmp::proj_decode_workspace(p);
 }
@@ -437,7 +447,9 @@ int cmp_compressor(const cmp_bf16* x, float* kv_state, float* score_state,
   p.n_out = (int)cmp_out_rows(p.B, p.T, ratio);
 
   for (int attempt = 0; attempt < 2; ++attempt) {
-    const int r2 = run_path(p, choose_path(p, g_proj_kernel.load()), s);
+    const int knob = g_proj_kernel.load();
+    p.single_cta = knob == 7 ? 1 : 0;
+    const int r2 = run_path(p, choose_path(p, knob == 7 ? 2 : knob), s);
     // the device refused the channel-group decode's launch form (nothing ran):
     // the path is now disabled there and the next choice is taken
     if (r2 != kRetryOtherPath) return r2;
@@ -597,7 +609,7 @@ int cmp_profile_stop(double* ms, int64_t* launches) {
 }
 
 int cmp_set_proj_kernel(int which) {
-  if (which < 0 || which > 6) return -1;
+  if (which < 0 || which > 7) return -1;
   return g_proj_kernel.exchange(which);
 }
 

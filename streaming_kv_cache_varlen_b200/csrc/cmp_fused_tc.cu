@@ -10,25 +10,47 @@
 // of the same channels ("compressor torch_extension API", 计算公式 1:
 // [kv, score] = X [W^KV, W^Gate]). So TMEM lane i holds channel i's kv
 // (columns 0..255) and score (columns 256..511) for all 256 positions, and one
-// thread owns one channel of every window in the tile.
+// thread owns one channel of every window in a 128-position half of the tile.
 //
 // The epilogue, per channel and window (计算公式 2-5), adds ape[q mod ratio] to
 // the score, takes positions before start_pos from the paged state (only the
 // first window of a sequence has any), and runs the per-channel softmax-
 // weighted sum over the window's rows. It writes the pooled value y (and, for
 // the two halves of a coff = 2 window, the log-sum-exp of its scores so that
-// the finish kernel can merge the previous window's half 0 with this window's
+// the row's finish can merge the previous window's half 0 with this window's
 // half 1 exactly: the softmax over 8 rows splits into two 4-row softmaxes
 // weighted by their exp-sums). The tail rows a later call reads
 // (p >= (e/ratio - coff + 1)*ratio) go to the paged fp32 state from here.
 //
-// Roles (192 threads, one CTA per SM, persistent): warp 0 TMA (3 stages of
+// Roles (320 threads, one CTA per SM, persistent): warp 0 TMA (3 stages of
 // 16 + 16 + 32 KB), warp 1 TMEM owner and MMA issuer (M=128, N=256, K=16, two
-// per k-step), warps 2-5 epilogue. All waits are bounded, as in the plain
-// projection kernel.
+// per k-step), warps 2-9 epilogue: two warps per TMEM lane quarter, one for
+// each 128-position half of the tile (a window never straddles the halves, as
+// ratio divides 128), so the accumulator is drained in half the time and the
+// next item's MMAs start sooner. All waits are bounded: a role that gives up
+// raises the CTA's abort flag and the device error word, and all roles then
+// leave their loops, so the kernel always ends.
+//
+// Folded mode (no rotation, B <= kMetaSeqs, tile counters available): the call
+// is this one kernel.
+//  * Every CTA validates cu_seqlens / start_pos and builds the per-sequence
+//    metadata (token offsets, start positions, first output rows, first work
+//    tiles) in its shared memory, as the scheduler kernel otherwise does.
+//  * Each item, once pooled, arrives on its tile's counter (and, for coff = 2,
+//    on the next tile's, whose first window needs this tile's half 0). The CTA
+//    whose arrival completes a counter finishes that tile's output rows:
+//    merge of the halves (coff = 2), RMSNorm, RoPE, bf16 store. Nobody waits:
+//    the last arriver does the work, then puts the counter back to zero for the
+//    next call (a kernel of the next call touches the counters only after its
+//    griddepcontrol.wait, i.e. after this grid has completed).
+//  * Rows that hold no window are zeroed by the epilogue warps, spread over
+//    the CTAs by sequence.
+// Otherwise the scheduler kernel runs before (metadata, hadamard check) and the
+// finish kernel after this one.
 #include <mutex>
 
 #include "cmp_internal.cuh"
+#include "cmp_rowpost.cuh"
 #include "cmp_sm100.cuh"
 
 namespace cmp {
@@ -40,7 +62,9 @@ constexpr int NTOK = 256;   // positions per tile (MMA N)
 constexpr int BM = 128;     // channels per item (MMA M)
 constexpr int BK = 64;
 constexpr int STAGES = 3;
-constexpr int kThreads = 192;
+constexpr int kThreads = 320;
+constexpr int kEpiThreads = 256;  // warps 2-9
+constexpr int kMetaSeqs = 512;    // folded mode: sequences whose metadata fits in shared memory
 constexpr uint32_t kStageBytes = 2 * BM * BK * 2 + NTOK * BK * 2;  // 64 KB
 constexpr uint32_t kIdesc = idesc_bf16_f32(BM, NTOK);
 
@@ -54,46 +78,165 @@ struct Smem {
   uint64_t acc_empty;
   uint32_t tmem_base;
   int abort;
+  // folded mode: per-sequence metadata, the block scan's scratch, the tiles
+  // this CTA finishes after its current item
+  int32_t m_cu[kMetaSeqs + 1];
+  int32_t m_s[kMetaSeqs];
+  int32_t m_off[kMetaSeqs + 1];
+  int32_t m_tile[kMetaSeqs + 1];
+  int scan_w[32];
+  int scan_tot;
+  int bad;
+  int fin[2];
+  int nfin;
 };
+
+// Per-sequence metadata: in shared memory (folded mode) or in the workspace
+// (written by the scheduler kernel). Plain loads: the pointers may be either.
+struct Meta {
+  const int32_t* cu;    // [B+1] validated token offsets
+  const int32_t* s;     // [B]   start positions
+  const int32_t* off;   // [B+1] first output row of each sequence
+  const int32_t* tile;  // [B+1] first work tile of each sequence
+};
+
+__device__ __forceinline__ int upper_index_plain(const int32_t* a, int n, int v) {
+  int lo = 0, hi = n;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (a[mid] <= v) lo = mid; else hi = mid - 1;
+  }
+  return lo;
+}
+
+__device__ __forceinline__ void epi_bar() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
+
+__device__ __forceinline__ float4 ldcg4(const float* p) { return __ldcg(reinterpret_cast<const float4*>(p)); }
+
+// Exclusive prefix sum over the CTA's threads (every thread calls it); *total
+// gets the sum.
+__device__ __forceinline__ int cta_exclusive_scan(int v, int* wsum, int* total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  constexpr int NW = kThreads / 32;
+  int inc = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int n = __shfl_up_sync(0xffffffffu, inc, o);
+    if (lane >= o) inc += n;
+  }
+  if (lane == 31) wsum[warp] = inc;
+  __syncthreads();
+  if (warp == 0) {
+    const int w = lane < NW ? wsum[lane] : 0;
+    int wi = w;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int n = __shfl_up_sync(0xffffffffu, wi, o);
+      if (lane >= o) wi += n;
+    }
+    wsum[lane] = wi - w;
+    if (lane == 31) *total = wi;
+  }
+  __syncthreads();
+  const int r = wsum[warp] + inc - v;
+  __syncthreads();
+  return r;
+}
+
+// Folded mode: the scheduler's validation and metadata, in this CTA's shared
+// memory (the same rules: cu rises from 0 to T, start_pos >= 0, positions fit in
+// int32; a rejected call gets empty sequences, so every output row is 0;
+// sequence b reserves min(L, L/ratio + 1) output rows; its work tiles cover
+// positions from start_pos rounded down to the ratio to its end).
+__device__ void build_meta(const Params& p, Smem& sm) {
+  const int B = p.B;
+  if (threadIdx.x == 0) sm.bad = 0;
+  __syncthreads();
+  for (int b = threadIdx.x; b <= B; b += kThreads) {
+    const int c = __ldg(p.cu_in + b);
+    bool ok = c >= 0 && c <= p.T;
+    if (b == 0) ok = ok && c == 0;
+    if (b == B) ok = ok && c == p.T;
+    if (b < B) {
+      const int c1 = __ldg(p.cu_in + b + 1);
+      const int s = p.start_pos ? __ldg(p.start_pos + b) : 0;
+      ok = ok && c1 >= c && s >= 0 && (int64_t)s + (int64_t)(c1 - c) <= (int64_t)INT32_MAX;
+    }
+    if (!ok) atomicOr(&sm.bad, 1);
+  }
+  __syncthreads();
+  const bool rejected = sm.bad != 0;
+  if (rejected && threadIdx.x == 0 && blockIdx.x == 0) atomicOr(p.err, kErrIndex);
+  int carry = 0, tcarry = 0;
+  for (int base = 0; base < B; base += kThreads) {
+    const int b = base + threadIdx.x;
+    int c = 0, s = 0, cap = 0, tiles = 0;
+    if (b < B && !rejected) {
+      c = __ldg(p.cu_in + b);
+      const int L = __ldg(p.cu_in + b + 1) - c;
+      s = p.start_pos ? __ldg(p.start_pos + b) : 0;
+      cap = min(L, L / p.ratio + 1);
+      if (L > 0) tiles = (s + L - (s / p.ratio) * p.ratio + NTOK - 1) / NTOK;
+    }
+    const int ex = cta_exclusive_scan(cap, sm.scan_w, &sm.scan_tot);
+    const int cap_total = sm.scan_tot;
+    __syncthreads();
+    const int tex = cta_exclusive_scan(tiles, sm.scan_w, &sm.scan_tot);
+    const int tile_total = sm.scan_tot;
+    if (b < B) {
+      sm.m_cu[b] = c;
+      sm.m_s[b] = s;
+      sm.m_off[b] = carry + ex;
+      sm.m_tile[b] = tcarry + tex;
+    }
+    carry += cap_total;
+    tcarry += tile_total;
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) {
+    sm.m_cu[B] = rejected ? 0 : p.T;
+    sm.m_off[B] = carry;
+    sm.m_tile[B] = tcarry;
+  }
+}
 
 // What one work item covers.
 struct Item {
   int b;      // sequence
+  int k;      // tile of the sequence
   int P0;     // first position of the tile
   int t0;     // x row of position P0 (may lie before the sequence, even < 0)
   int half;   // 0 / 1: which coff half of the state row
   int c0;     // first channel (within the half)
 };
 
-__device__ __forceinline__ Item decode_item(const Params& p, int g, int n_cblk) {
+__device__ __forceinline__ Item decode_item(const Params& p, const Meta& md, int g, int n_cblk) {
   Item it;
   const int tile = g / n_cblk, cb = g % n_cblk;
   const int per_half = p.D / BM;
   it.half = cb / per_half;
   it.c0 = (cb % per_half) * BM;
-  it.b = upper_index(p.m_tile, p.B, tile);
-  const int k = tile - p.m_tile[it.b];
-  const int s = p.m_s[it.b];
-  it.P0 = (s / p.ratio) * p.ratio + k * NTOK;
-  it.t0 = p.m_cu[it.b] + (it.P0 - s);
+  it.b = upper_index_plain(md.tile, p.B, tile);
+  it.k = tile - md.tile[it.b];
+  const int s = md.s[it.b];
+  it.P0 = (s / p.ratio) * p.ratio + it.k * NTOK;
+  it.t0 = md.cu[it.b] + (it.P0 - s);
   return it;
 }
 
-__device__ __forceinline__ int n_items(const Params& p) {
-  return p.m_tile[p.B] * (p.coff * p.D / BM);
-}
-
-// The epilogue of one item for a compile-time ratio R.
+// The epilogue of one item for a compile-time ratio R: the chunks of 32
+// positions of one 128-position half (hp) of the tile.
 template <int R>
-__device__ __forceinline__ void pool_item(const Params& p, const Item& it, uint32_t taddr, int ch) {
+__device__ __forceinline__ void pool_item(const Params& p, const Meta& md, const Item& it, uint32_t taddr,
+                                          int ch, int hp) {
   constexpr int COFF = (R == 4) ? 2 : 1;
   const int b = it.b;
-  const int s = p.m_s[b];
-  const int cu = p.m_cu[b];
-  const int e = s + (p.m_cu[b + 1] - cu);
+  const int s = md.s[b];
+  const int cu = md.cu[b];
+  const int e = s + (md.cu[b + 1] - cu);
   const int w0 = s / R;        // first window this call completes
   const int w_end = e / R;     // windows below this one complete in this call
-  const int off = p.m_off[b];  // output row of window w0
+  const int off = md.off[b];   // output row of window w0
   const int thr = max(s, tail_threshold(e, R, COFF));
   const int col = it.half * p.D + ch;  // column in the coff*D wide state / ape rows
   float* ybase = p.ystat + (int64_t)it.half * p.D + ch;
@@ -107,7 +250,7 @@ __device__ __forceinline__ void pool_item(const Params& p, const Item& it, uint3
   float m = -INFINITY, l = 0.f, acc = 0.f;  // running stats of a window wider than a chunk
 
 #pragma unroll 1
-  for (int c = 0; c < NTOK / 32; ++c) {
+  for (int c = hp * 4; c < hp * 4 + 4; ++c) {
     const int q0 = it.P0 + c * 32;
     if (q0 >= e) break;  // the rest of the tile lies past the sequence
     uint32_t kr[32], sr[32];
@@ -199,11 +342,201 @@ __device__ __forceinline__ void pool_item(const Params& p, const Item& it, uint3
   }
 }
 
+// Folded mode, one warp: output row n = window w of sequence b (first: w is the
+// first window this call completes for b). NG = D / 128; lane l holds channels
+// 128 i + 4 l .. +3 of group i. coff = 2 merges half 0 of window w - 1 (the
+// previous row, or pooled here from the paged state when that window lies
+// wholly before start_pos, or nothing for window 0) with half 1 of window w
+// through their log-sum-exps, which is the 2 ratio-row softmax exactly; then
+// RMSNorm (eps 1e-6) times norm_weight, interleaved RoPE on the last 64
+// channels (pair (2j, 2j+1) takes table columns j and 32 + j) and the bf16
+// store ("CANN PyPTO 算子实战", 压缩窗口与状态更新). Every load of the row is
+// issued before the first use, so a row costs about one memory round trip.
+template <int NG, int COFF>
+__device__ __forceinline__ void finish_window(const Params& p, int b, int w, int64_t n, bool first, int lane,
+                                              const float (&nw)[NG][4]) {
+  constexpr int D = NG * 128;
+  constexpr int kRope = 64;  // rope_head_dim (the only value the library accepts)
+  const bool rope_lane = lane >= 16;  // group NG-1: channels D-64 .. D-1
+  const int j = 2 * (lane - 16);      // its pairs use table columns j, j+1 and 32+j, 33+j
+  __nv_bfloat162 c_lo, c_hi, s_lo, s_hi;
+  if (rope_lane) {
+    const __nv_bfloat16* cs = p.cos + n * kRope;
+    const __nv_bfloat16* sn = p.sin + n * kRope;
+    c_lo = *reinterpret_cast<const __nv_bfloat162*>(cs + j);
+    c_hi = *reinterpret_cast<const __nv_bfloat162*>(cs + 32 + j);
+    s_lo = *reinterpret_cast<const __nv_bfloat162*>(sn + j);
+    s_hi = *reinterpret_cast<const __nv_bfloat162*>(sn + 32 + j);
+  }
+  float4 yb[NG], lb[NG], ya[NG], la[NG];
+  const bool prev_row = COFF == 2 && !first;
+#pragma unroll
+  for (int i = 0; i < NG; ++i) {
+    const int c = i * 128 + lane * 4;
+    if (COFF == 1) {
+      yb[i] = ldcg4(p.ystat + n * D + c);
+    } else {
+      yb[i] = ldcg4(p.ystat + (n * 2 + 1) * D + c);
+      lb[i] = ldcg4(p.ylse + (n * 2 + 1) * D + c);
+      if (prev_row) {
+        ya[i] = ldcg4(p.ystat + (n - 1) * 2 * D + c);
+        la[i] = ldcg4(p.ylse + (n - 1) * 2 * D + c);
+      } else {
+        ya[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+        la[i] = make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
+      }
+    }
+  }
+  if (COFF == 2 && first && w > 0) {  // window w - 1 from the paged state (rare: once per sequence)
+#pragma unroll
+    for (int i = 0; i < NG; ++i) {
+      const int c = i * 128 + lane * 4;
+      float m[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY}, l[4] = {0.f, 0.f, 0.f, 0.f},
+            a[4] = {0.f, 0.f, 0.f, 0.f};
+      for (int jj = 0; jj < p.ratio; ++jj) {
+        const int q = (w - 1) * p.ratio + jj;
+        const int rk = table_row(p, p.kv_tbl, b, q);
+        const int rs = table_row(p, p.sc_tbl, b, q);
+        if (rk < 0 || rs < 0) continue;
+        const float4 kv = __ldcg(reinterpret_cast<const float4*>(
+            p.kv_state + ((int64_t)rk * p.bs + q % p.bs) * p.C + c));
+        const float4 sc = __ldcg(reinterpret_cast<const float4*>(
+            p.score_state + ((int64_t)rs * p.bs + q % p.bs) * p.C + c));
+        const float kk[4] = {kv.x, kv.y, kv.z, kv.w}, zz[4] = {sc.x, sc.y, sc.z, sc.w};
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const float mn = fmaxf(m[u], zz[u]);
+          const float f = __expf(m[u] - mn), pz = __expf(zz[u] - mn);
+          l[u] = l[u] * f + pz;
+          a[u] = a[u] * f + pz * kk[u];
+          m[u] = mn;
+        }
+      }
+      float yv[4] = {0.f, 0.f, 0.f, 0.f}, lv[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+        if (l[u] > 0.f) {
+          yv[u] = a[u] / l[u];
+          lv[u] = m[u] + __logf(l[u]);
+        }
+      ya[i] = make_float4(yv[0], yv[1], yv[2], yv[3]);
+      la[i] = make_float4(lv[0], lv[1], lv[2], lv[3]);
+    }
+  }
+  float y[NG][4];
+  float ss = 0.f;
+#pragma unroll
+  for (int i = 0; i < NG; ++i) {
+    const float ybv[4] = {yb[i].x, yb[i].y, yb[i].z, yb[i].w};
+    if (COFF == 1) {
+#pragma unroll
+      for (int u = 0; u < 4; ++u) y[i][u] = ybv[u];
+    } else {
+      const float lbv[4] = {lb[i].x, lb[i].y, lb[i].z, lb[i].w};
+      const float yav[4] = {ya[i].x, ya[i].y, ya[i].z, ya[i].w};
+      const float lav[4] = {la[i].x, la[i].y, la[i].z, la[i].w};
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const float M = fmaxf(lav[u], lbv[u]);
+        const float wa = __expf(lav[u] - M), wb = __expf(lbv[u] - M);
+        y[i][u] = (yav[u] * wa + ybv[u] * wb) / (wa + wb);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) ss = fmaf(y[i][u], y[i][u], ss);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+  const float inv = rsqrtf(ss / (float)D + kRmsEps);
+#pragma unroll
+  for (int i = 0; i < NG; ++i) {
+    const int c = i * 128 + lane * 4;
+    float z[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) z[u] = y[i][u] * inv * nw[i][u];
+    if (i == NG - 1 && rope_lane) {
+      const float ce[2] = {__low2float(c_lo), __high2float(c_lo)}, co[2] = {__low2float(c_hi), __high2float(c_hi)};
+      const float se[2] = {__low2float(s_lo), __high2float(s_lo)}, so[2] = {__low2float(s_hi), __high2float(s_hi)};
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+        const float ev = z[2 * u], od = z[2 * u + 1];
+        z[2 * u] = ev * ce[u] - od * se[u];
+        z[2 * u + 1] = od * co[u] + ev * so[u];
+      }
+    }
+    __nv_bfloat162 o01 = __floats2bfloat162_rn(z[0], z[1]);
+    __nv_bfloat162 o23 = __floats2bfloat162_rn(z[2], z[3]);
+    uint2 v;
+    v.x = *reinterpret_cast<uint32_t*>(&o01);
+    v.y = *reinterpret_cast<uint32_t*>(&o23);
+    *reinterpret_cast<uint2*>(p.out + n * D + c) = v;
+  }
+}
+
+// Folded mode: the output rows of work tile t (its windows), one per warp of
+// the eight epilogue warps at a time.
+template <int NG, int COFF>
+__device__ void finish_tile_t(const Params& p, const Meta& md, int t, int ew, int lane) {
+  const int b = upper_index_plain(md.tile, p.B, t);
+  const int k = t - md.tile[b];
+  const int s = md.s[b];
+  const int e = s + (md.cu[b + 1] - md.cu[b]);
+  const int R = p.ratio;
+  const int P0 = (s / R) * R + k * NTOK;
+  const int w0 = s / R;
+  const int wa = P0 / R, wb = min((P0 + NTOK) / R, e / R);
+  const int64_t off = md.off[b];
+  float nw[NG][4];  // norm_weight of the lane's channels, shared by the rows
+#pragma unroll
+  for (int i = 0; i < NG; ++i) {
+    const uint2 wraw = *reinterpret_cast<const uint2*>(p.norm_w + i * 128 + lane * 4);
+    const __nv_bfloat162 w01 = *reinterpret_cast<const __nv_bfloat162*>(&wraw.x);
+    const __nv_bfloat162 w23 = *reinterpret_cast<const __nv_bfloat162*>(&wraw.y);
+    nw[i][0] = __low2float(w01);
+    nw[i][1] = __high2float(w01);
+    nw[i][2] = __low2float(w23);
+    nw[i][3] = __high2float(w23);
+  }
+  for (int w = wa + ew; w < wb; w += kEpiThreads / 32)
+    finish_window<NG, COFF>(p, b, w, off + (w - w0), w == w0, lane, nw);
+}
+
+__device__ void finish_tile(const Params& p, const Meta& md, int t, int ew, int lane) {
+  if (p.D == 128) {
+    if (p.coff == 2) finish_tile_t<1, 2>(p, md, t, ew, lane);
+    else finish_tile_t<1, 1>(p, md, t, ew, lane);
+  } else {
+    if (p.coff == 2) finish_tile_t<4, 2>(p, md, t, ew, lane);
+    else finish_tile_t<4, 1>(p, md, t, ew, lane);
+  }
+}
+
+// Folded mode: zero the output rows that hold no window (each sequence's
+// reserved rows past its completed windows, and the rows after the last
+// sequence's), sequences spread over the CTAs; eight warps, 16 bytes a lane.
+__device__ void zero_rows(const Params& p, const Meta& md, int ew, int lane) {
+  const int D = p.D;
+  const int per_row = D * 2 / 16;  // uint4 per row
+  auto zero = [&](int64_t r0, int64_t r1) {
+    const int64_t total = (r1 - r0) * per_row;
+    uint4* base = reinterpret_cast<uint4*>(p.out + r0 * D);
+    for (int64_t i = ew * 32 + lane; i < total; i += kEpiThreads) base[i] = make_uint4(0u, 0u, 0u, 0u);
+  };
+  for (int b = blockIdx.x; b < p.B; b += gridDim.x) {
+    const int s = md.s[b];
+    const int e = s + (md.cu[b + 1] - md.cu[b]);
+    const int nw = e / p.ratio - s / p.ratio;
+    zero(md.off[b] + nw, md.off[b + 1]);
+  }
+  if (blockIdx.x == 0) zero(md.off[p.B], p.n_out);
+}
+
+template <bool FOLD>
 __global__ void __launch_bounds__(kThreads, 1)
     fused_tc_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUtensorMap map_wkv,
                     const __grid_constant__ CUtensorMap map_wg, Params p) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
-  Smem& sm = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  Smem& sm = smem_align1024<Smem>(smem_raw);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int n_cblk = p.coff * p.D / BM;
   const int k_blocks = p.H / BK;
@@ -214,7 +547,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&sm.empty[s], 1);
     }
     mbar_init(&sm.acc_full, 1);
-    mbar_init(&sm.acc_empty, 4);
+    mbar_init(&sm.acc_empty, kEpiThreads / 32);
     sm.abort = 0;
     fence_barrier_init();
     prefetch_tmap(&map_x);
@@ -222,21 +555,28 @@ __global__ void __launch_bounds__(kThreads, 1)
     prefetch_tmap(&map_wg);
   }
   if (warp == 1) tmem_alloc(&sm.tmem_base, 512);
+  if constexpr (FOLD) build_meta(p, sm);  // reads only this call's inputs
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = sm.tmem_base;
   volatile int* abort = &sm.abort;
   pdl_trigger();
-  pdl_wait();  // the tile list comes from the scheduler kernel
-  const int total = n_items(p);
+  Meta md;
+  if constexpr (FOLD) {
+    md = Meta{sm.m_cu, sm.m_s, sm.m_off, sm.m_tile};
+  } else {
+    pdl_wait();  // the metadata comes from the scheduler kernel
+    md = Meta{p.m_cu, p.m_s, p.m_off, p.m_tile};
+  }
+  const int total = md.tile[p.B] * n_cblk;
 
   if (warp == 0) {
     if (lane == 0) {
       int stage = 0;
       uint32_t phase = 0;
       for (int g = blockIdx.x; g < total && !*abort; g += gridDim.x) {
-        const Item it = decode_item(p, g, n_cblk);
+        const Item it = decode_item(p, md, g, n_cblk);
         const int wrow = it.half * p.D + it.c0;
         for (int kb = 0; kb < k_blocks; ++kb) {
           if (!mbar_wait(&sm.empty[stage], phase ^ 1u, abort)) break;
@@ -279,30 +619,66 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
   } else {
-    const int quad = warp & 3;
+    const int ew = warp - 2;                 // 0..7
+    const int e_tid = threadIdx.x - 64;      // 0..255
+    const int quad = warp & 3;               // TMEM lanes this warp may access
+    const int hp = ew >> 2;                  // 128-position half of the tile
     const int row = quad * 32 + lane;
     const uint32_t taddr = tmem + ((uint32_t)(quad * 32) << 16);
+    if constexpr (FOLD) {
+      pdl_wait();  // the epilogue writes the state, the pooled halves and out
+      zero_rows(p, md, ew, lane);
+    }
     uint32_t acc_phase = 0;
     for (int g = blockIdx.x; g < total; g += gridDim.x) {
-      const Item it = decode_item(p, g, n_cblk);
+      const Item it = decode_item(p, md, g, n_cblk);
       const bool ok = mbar_wait(&sm.acc_full, acc_phase, abort);
-      if (!bar_and(1, 128, ok)) break;  // all four warps leave together
+      if (!bar_and(1, kEpiThreads, ok)) break;  // all eight warps leave together
       tc_fence_after();
       const int ch = it.c0 + row;
       switch (p.ratio) {
-        case 1: pool_item<1>(p, it, taddr, ch); break;
-        case 2: pool_item<2>(p, it, taddr, ch); break;
-        case 4: pool_item<4>(p, it, taddr, ch); break;
-        case 8: pool_item<8>(p, it, taddr, ch); break;
-        case 16: pool_item<16>(p, it, taddr, ch); break;
-        case 32: pool_item<32>(p, it, taddr, ch); break;
-        case 64: pool_item<64>(p, it, taddr, ch); break;
-        default: pool_item<128>(p, it, taddr, ch); break;
+        case 1: pool_item<1>(p, md, it, taddr, ch, hp); break;
+        case 2: pool_item<2>(p, md, it, taddr, ch, hp); break;
+        case 4: pool_item<4>(p, md, it, taddr, ch, hp); break;
+        case 8: pool_item<8>(p, md, it, taddr, ch, hp); break;
+        case 16: pool_item<16>(p, md, it, taddr, ch, hp); break;
+        case 32: pool_item<32>(p, md, it, taddr, ch, hp); break;
+        case 64: pool_item<64>(p, md, it, taddr, ch, hp); break;
+        default: pool_item<128>(p, md, it, taddr, ch, hp); break;
       }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&sm.acc_empty);
       acc_phase ^= 1u;
+      if constexpr (FOLD) {
+        // arrive on the tile's counter (coff = 2: also on the next tile's); the
+        // barrier orders every epilogue thread's stores before thread 0's
+        // release fence and atomic, and the finishing CTA's acquire fence
+        // before its loads (the pattern of a cooperative grid barrier)
+        epi_bar();
+        if (e_tid == 0) {
+          const int tile = g / n_cblk;
+          const int ntiles_b = md.tile[it.b + 1] - md.tile[it.b];
+          int nf = 0;
+          __threadfence();
+          const unsigned tgt = (unsigned)n_cblk * ((p.coff == 2 && it.k > 0) ? 2u : 1u);
+          if (atomicAdd(p.tile_cnt + tile, 1u) + 1u == tgt) {
+            atomicExch(p.tile_cnt + tile, 0u);
+            sm.fin[nf++] = tile;
+          }
+          if (p.coff == 2 && it.k + 1 < ntiles_b) {
+            if (atomicAdd(p.tile_cnt + tile + 1, 1u) + 1u == 2u * (unsigned)n_cblk) {
+              atomicExch(p.tile_cnt + tile + 1, 0u);
+              sm.fin[nf++] = tile + 1;
+            }
+          }
+          if (nf) __threadfence();
+          sm.nfin = nf;
+        }
+        epi_bar();
+        const int nf = sm.nfin;
+        for (int i = 0; i < nf; ++i) finish_tile(p, md, sm.fin[i], ew, lane);
+      }
     }
   }
 
@@ -321,11 +697,12 @@ bool fused_supported(const Params& p) {
   return p.H % BK == 0 && p.D % BM == 0 && NTOK % p.ratio == 0 && encode_fn() != nullptr;
 }
 
-// Upper bound of the work items of a call (the exact count is on the device):
+// Upper bound of the work tiles of a call (the exact count is on the device):
 // every sequence adds at most one partial tile at each end.
-int fused_max_items(const Params& p) {
-  const int64_t tiles = ((int64_t)p.T + NTOK - 1) / NTOK + 2LL * p.B;
-  return (int)(tiles * (p.coff * p.D / BM));
+int64_t fused_max_tiles(const Params& p) { return ((int64_t)p.T + NTOK - 1) / NTOK + 2LL * p.B; }
+
+bool fused_fold_supported(const Params& p) {
+  return !p.rotate && p.B <= kMetaSeqs && fused_max_tiles(p) + 1 <= kFusedTileCounters;
 }
 
 cudaError_t launch_fused(const Params& p, cudaStream_t s, int sm_count) {
@@ -334,12 +711,16 @@ cudaError_t launch_fused(const Params& p, cudaStream_t s, int sm_count) {
       !make_tile_map(&mg, p.wgate, p.C, p.H, BM))
     return cudaErrorInvalidValue;
   const size_t smem = sizeof(Smem) + 1024;
-  static int configured[64] = {0};
-  const cudaError_t e = smem_attr_once(fused_tc_kernel, smem, configured);
+  const bool fold = p.tile_cnt != nullptr;
+  static int configured[2][64] = {{0}};
+  const cudaError_t e = fold ? smem_attr_once(fused_tc_kernel<true>, smem, configured[1])
+                             : smem_attr_once(fused_tc_kernel<false>, smem, configured[0]);
   if (e != cudaSuccess) return e;
-  const int items = fused_max_items(p);
-  const int grid = items < sm_count ? items : sm_count;
-  return launch_chained(fused_tc_kernel, dim3(grid), dim3(kThreads), smem, s, 1, mx, mkv, mg, p);
+  const int64_t items = fused_max_tiles(p) * (p.coff * p.D / BM);
+  const int grid = items < sm_count ? (int)items : sm_count;
+  if (fold)
+    return launch_chained(fused_tc_kernel<true>, dim3(grid), dim3(kThreads), smem, s, 1, mx, mkv, mg, p);
+  return launch_chained(fused_tc_kernel<false>, dim3(grid), dim3(kThreads), smem, s, 1, mx, mkv, mg, p);
 }
 
 }  // namespace cmp

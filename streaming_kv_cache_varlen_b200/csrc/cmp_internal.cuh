@@ -50,6 +50,9 @@ struct Params {
   int32_t* had_sylv;  // rotate: per kHadChunk entries of hadamard, 1 if they are those of
                       // hadamard[0][0] * (Sylvester H_D) (the scheduler kernel checks), else 0;
                       // null: not checked (the dense product is used)
+  unsigned* tile_cnt; // fused path in one kernel: per work tile, the arrivals of its items
+                      // (zero between calls), else null (scheduler and finish kernels run)
+  int single_cta;     // tcgen05 projection: 1 = on single CTAs even where CTA pairs would run
 };
 
 // Entries of the hadamard matrix each checking CTA of the scheduler kernel covers.
@@ -161,6 +164,10 @@ cudaError_t launch_pool(const Params& p, cudaStream_t s);
 cudaError_t launch_finish(const Params& p, cudaStream_t s);
 cudaError_t launch_fused(const Params& p, cudaStream_t s, int sm_count);
 bool fused_supported(const Params& p);
+// Whether the fused path can run as one kernel (metadata and row finish inside):
+// no rotation, few enough sequences and work tiles.
+bool fused_fold_supported(const Params& p);
 constexpr int kFusedTile = 256;  // positions per fused work tile
+constexpr int kFusedTileCounters = 8192;  // arrival counters of the one-kernel fused path
 
 }  // namespace cmp

@@ -35,8 +35,8 @@ def check(cmp, inp, rows=None):
     return out, kv, sc, res
 
 
-@pytest.fixture(params=[0, 1, 2, 3, 4, 5, 6],
-                ids=["auto", "mma", "tcgen05", "decode", "fused", "decode1k", "decodecp"])
+@pytest.fixture(params=[0, 1, 2, 3, 4, 5, 6, 7],
+                ids=["auto", "mma", "tcgen05", "decode", "fused", "decode1k", "decodecp", "tcgen05single"])
 def proj_kernel(request, lib):
     prev = lib.set_proj_kernel(request.param)
     yield request.param
@@ -183,6 +183,57 @@ def test_fused_path_history_and_tails(lib, ratio, auto_or_fused):
     check(lib, with_rope(inp))
 
 
+# The fused path runs as one kernel (metadata built per CTA, rows finished by the
+# last CTA to complete each tile) without rotation and for at most 512 sequences;
+# otherwise the scheduler and finish kernels run around it.
+FUSED_ONE_KERNEL_CASES = {
+    "ratio4_512_sequences": (4, 512, False, 1),
+    "ratio4_513_sequences": (4, 513, False, 3),
+    "ratio128_512_sequences": (128, 512, False, 1),
+    "ratio128_513_sequences": (128, 513, False, 3),
+    "ratio4_rotation": (4, 40, True, 3),
+}
+
+
+@pytest.mark.parametrize("name", sorted(FUSED_ONE_KERNEL_CASES))
+def test_fused_one_kernel_and_split_forms(lib, name):
+    ratio, B, rotate, launches = FUSED_ONE_KERNEL_CASES[name]
+    rng = np.random.default_rng(B + ratio)
+    hi = 3 * ratio if ratio == 128 else 40
+    L = [int(v) for v in rng.integers(0, hi, size=B)]
+    sp = [int(v) for v in rng.integers(0, 2 * ratio, size=B)]
+    L[0] = 300  # one sequence over two tiles
+    inp = make_inputs(name=name, seed=B, lengths=L, start_pos=sp, H=512,
+                      D=128, coff=2 if ratio == 4 else 1, ratio=ratio, block_size=32, rotate=rotate)
+    prev = lib.set_proj_kernel(4)
+    try:
+        lib.profile_start()
+        check(lib, with_rope(inp))
+        launched = lib.profile_stop()
+    finally:
+        lib.set_proj_kernel(prev)
+    assert launched["fused_tcgen05"][1] == 1 and sum(n for _, n in launched.values()) == launches, launched
+
+
+def test_fused_one_kernel_repeated_calls(lib):
+    """The per-tile arrival counters go back to zero: the same call three times,
+    then a call with other tiles and channel blocks, agree with the oracle."""
+    prev = lib.set_proj_kernel(4)
+    try:
+        a = with_rope(make_inputs(name="r1", seed=5, lengths=[700, 3, 260], start_pos=[0, 1, 9],
+                                  H=512, D=512, coff=2, ratio=4, block_size=64, rotate=False))
+        first = check(lib, a)[0]
+        for _ in range(2):
+            again = check(lib, a)[0]
+            assert np.array_equal(first, again)
+        b = with_rope(make_inputs(name="r2", seed=6, lengths=[1000, 77], start_pos=[5, 130],
+                                  H=512, D=128, coff=1, ratio=128, block_size=128, rotate=False))
+        check(lib, b)
+        check(lib, a)
+    finally:
+        lib.set_proj_kernel(prev)
+
+
 def test_dense_rotation_with_any_matrix(lib):
     inp = make_inputs(name="rot", seed=3, lengths=[40, 21], start_pos=[0, 6], H=1024, D=128,
                       coff=2, ratio=4, block_size=16, rotate=True)
@@ -255,7 +306,7 @@ def test_projection_kernels_agree(lib):
                                 H=4096, D=512, coff=2, ratio=4, block_size=128, rotate=False))
     res = run_inputs(inp)
     outs = {}
-    for k in (1, 2, 3, 4, 5, 6):
+    for k in (1, 2, 3, 4, 5, 6, 7):
         prev = lib.set_proj_kernel(k)
         try:
             o, kv, sc, err = run(lib, inp)
@@ -267,6 +318,38 @@ def test_projection_kernels_agree(lib):
         assert_out_close(o, res)
         assert_state_close(kv, sc, inp, res)
         outs[k] = o
+
+
+# The tcgen05 projection runs on CTA pairs (cta_group::2, 256 weight rows per
+# pair tile, each CTA holding half of the tile's tokens) unless forced onto
+# single CTAs (knob 7). Cases: a ragged last tile whose second half lies past
+# T, several tiles per pair (double-buffered accumulators), 2C = 256 / 512 / 1024.
+PAIR_CASES = {
+    "ragged_tail_d128": ([1500, 1, 1333], [0, 2, 7], 128, 1024, 4),
+    "two_tiles_per_pair": ([6000, 5111, 900], [3, 0, 129], 128, 512, 4),
+    "d512_ratio4": ([700, 0, 613], [0, 5, 6], 512, 1024, 4),
+    "d512_ratio128": ([1100, 400], [100, 0], 512, 1024, 128),
+    "d128_ratio1": ([300, 20], [0, 3], 128, 1024, 1),
+}
+
+
+@pytest.mark.parametrize("name", sorted(PAIR_CASES))
+@pytest.mark.parametrize("knob", [2, 7], ids=["pairs", "single"])
+def test_tcgen05_projection_pairs_and_single(lib, name, knob):
+    L, sp, D, H, ratio = PAIR_CASES[name]
+    inp = with_rope(make_inputs(name=name, seed=21, lengths=L, start_pos=sp, H=H, D=D,
+                                coff=2 if ratio == 4 else 1, ratio=ratio, block_size=64,
+                                rotate=D == 128))
+    prev = lib.set_proj_kernel(knob)
+    try:
+        lib.profile_start()
+        out = check(lib, inp)[0]
+        launched = lib.profile_stop()
+        again = run(lib, inp)[0]
+    finally:
+        lib.set_proj_kernel(prev)
+    assert launched["proj_tcgen05"][1] == 1, launched
+    assert np.array_equal(out, again)
 
 
 # ---- the channel-group decode kernel -------------------------------------------------
@@ -366,7 +449,7 @@ def test_unneeded_padding_is_not_read(lib):
     check(lib, inp)
 
 
-def test_bad_cu_seqlens_rejected_on_device(lib):
+def test_bad_cu_seqlens_rejected_on_device(lib, auto_or_fused):
     import torch
     inp = with_rope(make_inputs(name="cu", seed=2, lengths=[6, 10], start_pos=[0, 0], H=512, D=128,
                                 coff=2, ratio=4, block_size=16, rotate=False))
@@ -374,7 +457,8 @@ def test_bad_cu_seqlens_rejected_on_device(lib):
     args["cu_seqlens"] = torch.tensor([0, 12, 16], dtype=torch.int32, device="cuda")
     args["cu_seqlens"][1] = 20             # not rising to T: the call is rejected
     kv0 = args["kv_state"].clone()
-    out = lib.compressor(**args)
+    out = torch.full((lib.out_rows(2, 16, 4), 128), 1.0, dtype=torch.bfloat16, device="cuda")
+    lib.compressor(**args, out=out)
     assert lib.get_error() == 5
     assert (bits(out) == 0).all() and torch.equal(args["kv_state"], kv0)
 
