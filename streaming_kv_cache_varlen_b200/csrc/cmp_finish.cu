@@ -52,6 +52,7 @@ __global__ void __launch_bounds__(128) finish_kernel(Params p) {
     *reinterpret_cast<uint2*>(p.out + (int64_t)n * D + c) = make_uint2(0u, 0u);
     return;
   }
+  const RowAux aux = load_row_aux(p, n, c);  // in flight while the halves load
 
   float y[4];
   if (p.coff == 1) {
@@ -103,7 +104,7 @@ __global__ void __launch_bounds__(128) finish_kernel(Params p) {
       y[i] = (ya[i] * wa + ybv[i] * wb) / (wa + wb);
     }
   }
-  finish_row(p, n, c, y, red, zs);
+  finish_row(p, n, c, y, red, zs, aux);
 }
 
 }  // namespace

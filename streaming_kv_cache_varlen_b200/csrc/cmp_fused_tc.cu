@@ -224,11 +224,125 @@ __device__ __forceinline__ Item decode_item(const Params& p, const Meta& md, int
   return it;
 }
 
-// The epilogue of one item for a compile-time ratio R: the chunks of 32
-// positions of one 128-position half (hp) of the tile.
-template <int R>
-__device__ __forceinline__ void pool_item(const Params& p, const Meta& md, const Item& it, uint32_t taddr,
-                                          int ch, int hp) {
+// The epilogue of one item for ratio R in {32, 64, 128} (a window spans 2, 4
+// or 8 sub-chunks of 16 positions): the sub-chunks of one 128-position half
+// (hp) of the tile, with an online softmax per window. The 16 ape values a sub-chunk
+// adds to its scores are loaded one sub-chunk ahead (the first ones before the
+// accumulator is ready), so their L2 latency overlaps the TMEM loads and the
+// previous sub-chunk's math instead of stalling each step while the MMA waits
+// for TMEM.
+template <int R, int D, class Wait>
+__device__ __forceinline__ bool pool_item_wide(const Params& p, const Meta& md, const Item& it, uint32_t taddr,
+                                               int ch, int hp, Wait&& wait_acc) {
+  static_assert(R == 32 || R == 64 || R == 128, "windows of 2, 4 or 8 sub-chunks");
+  constexpr int C = D;  // coff = 1: the state / ape rows are D wide
+  const int b = it.b;
+  const int s = md.s[b];
+  const int cu = md.cu[b];
+  const int e = s + (md.cu[b + 1] - cu);
+  const int w0 = s / R;
+  const int w_end = e / R;
+  const int off = md.off[b];
+  const int thr = max(s, tail_threshold(e, R, 1));
+  const int col = ch;  // coff = 1: one half
+  float* ybase = p.ystat + ch;
+  // the tile starts on a window boundary: position P0 + 16 u + j has ape row (16 u + j) mod R;
+  // the rows of sub-chunk u start at ape + ((16 u) mod R) * C + col (constant offsets j * C)
+  const float* ape_col = p.ape + col;
+  float apn[16];
+#pragma unroll
+  for (int j = 0; j < 16; ++j) apn[j] = __ldg(ape_col + ((hp * 128) % R + j) * C);
+  if (!wait_acc()) return false;
+  float m = -INFINITY, l = 0.f, acc = 0.f;
+
+#pragma unroll 1
+  for (int u = hp * 8; u < hp * 8 + 8; ++u) {
+    const int q0 = it.P0 + u * 16;
+    if (q0 >= e) break;  // the rest of the tile lies past the sequence
+    uint32_t kr[16], sr[16];
+    tmem_ld16(taddr + u * 16, kr);
+    tmem_ld16(taddr + NTOK + u * 16, sr);
+    float apc[16];
+#pragma unroll
+    for (int j = 0; j < 16; ++j) apc[j] = apn[j];
+    if (u + 1 < hp * 8 + 8) {
+      const float* ap_next = ape_col + ((16 * (u + 1)) % R) * C;
+#pragma unroll
+      for (int j = 0; j < 16; ++j) apn[j] = __ldg(ap_next + j * C);
+    }
+    tmem_ld_wait16(kr, sr);
+    float kv[16], z[16];
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+      kv[j] = __uint_as_float(kr[j]);
+      z[j] = __uint_as_float(sr[j]) + apc[j];
+    }
+    if (q0 < s) {  // rows written by earlier calls (the first window of the sequence)
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        const int q = q0 + j;
+        if (q < s) {
+          const int rk = table_row(p, p.kv_tbl, b, q);
+          const int rs = table_row(p, p.sc_tbl, b, q);
+          kv[j] = rk >= 0 ? p.kv_state[((int64_t)rk * p.bs + q % p.bs) * p.C + col] : 0.f;
+          z[j] = rs >= 0 ? p.score_state[((int64_t)rs * p.bs + q % p.bs) * p.C + col] : -INFINITY;
+        }
+      }
+    }
+    if (q0 + 15 >= thr) {  // tail rows: kv and score + ape into the paged state
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        const int q = q0 + j;
+        if (q >= thr && q < e) {
+          const int rk = table_row(p, p.kv_tbl, b, q);
+          const int rs = table_row(p, p.sc_tbl, b, q);
+          if (rk >= 0) p.kv_state[((int64_t)rk * p.bs + q % p.bs) * p.C + col] = kv[j];
+          if (rs >= 0) p.score_state[((int64_t)rs * p.bs + q % p.bs) * p.C + col] = z[j];
+        }
+      }
+    }
+    const int w = q0 / R;  // the sub-chunk is one piece of window w
+    if (w < w_end) {
+      float mx[8];  // tree maximum (short dependency chains)
+#pragma unroll
+      for (int j = 0; j < 8; ++j) mx[j] = fmaxf(z[j], z[j + 8]);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) mx[j] = fmaxf(mx[j], mx[j + 4]);
+      const float mn = fmaxf(m, fmaxf(fmaxf(mx[0], mx[2]), fmaxf(mx[1], mx[3])));
+      const float sc = __expf(m - mn);
+      float l2[2] = {0.f, 0.f}, a2[2] = {0.f, 0.f};  // two independent partial sums
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        const float pz = __expf(z[j] - mn);
+        l2[j & 1] += pz;
+        a2[j & 1] = fmaf(pz, kv[j], a2[j & 1]);
+      }
+      l = fmaf(l, sc, l2[0] + l2[1]);
+      acc = fmaf(acc, sc, a2[0] + a2[1]);
+      m = mn;
+      if (((u + 1) * 16) % R == 0) {  // last sub-chunk of the window
+        const int64_t n = off + (w - w0);
+        ybase[n * p.D] = acc / l;
+        m = -INFINITY;
+        l = 0.f;
+        acc = 0.f;
+      }
+    }
+  }
+  return true;
+}
+
+// The epilogue of one item for ratio R <= 16 (whole windows inside a chunk of
+// 32 positions): the chunks of one 128-position half (hp) of the tile. The R
+// ape rows are loaded before the accumulator is ready. `wait_acc` waits for
+// the accumulator (false: give up).
+template <int R, class Wait>
+__device__ __forceinline__ bool pool_item(const Params& p, const Meta& md, const Item& it, uint32_t taddr,
+                                          int ch, int hp, Wait&& wait_acc) {
+  if constexpr (R >= 32) {
+    if (p.D == 128) return pool_item_wide<R, 128>(p, md, it, taddr, ch, hp, wait_acc);
+    return pool_item_wide<R, 512>(p, md, it, taddr, ch, hp, wait_acc);
+  } else {
   constexpr int COFF = (R == 4) ? 2 : 1;
   const int b = it.b;
   const int s = md.s[b];
@@ -242,12 +356,10 @@ __device__ __forceinline__ void pool_item(const Params& p, const Meta& md, const
   float* ybase = p.ystat + (int64_t)it.half * p.D + ch;
   float* lbase = p.ylse + (int64_t)it.half * p.D + ch;
 
-  float ap[R <= 32 ? R : 1];
-  if constexpr (R <= 32) {
+  float ap[R];
 #pragma unroll
-    for (int j = 0; j < R; ++j) ap[j] = __ldg(p.ape + (int64_t)j * p.C + col);
-  }
-  float m = -INFINITY, l = 0.f, acc = 0.f;  // running stats of a window wider than a chunk
+  for (int j = 0; j < R; ++j) ap[j] = __ldg(p.ape + (int64_t)j * p.C + col);
+  if (!wait_acc()) return false;
 
 #pragma unroll 1
   for (int c = hp * 4; c < hp * 4 + 4; ++c) {
@@ -262,10 +374,7 @@ __device__ __forceinline__ void pool_item(const Params& p, const Meta& md, const
 #pragma unroll
     for (int j = 0; j < 32; ++j) {
       kv[j] = __uint_as_float(kr[j]);
-      float a;
-      if constexpr (R <= 32) a = ap[j % R];
-      else a = __ldg(p.ape + (int64_t)((q0 + j) % R) * p.C + col);
-      z[j] = __uint_as_float(sr[j]) + a;
+      z[j] = __uint_as_float(sr[j]) + ap[j % R];
     }
     if (q0 < s) {  // rows written by earlier calls (the first window of the sequence)
 #pragma unroll
@@ -291,34 +400,7 @@ __device__ __forceinline__ void pool_item(const Params& p, const Meta& md, const
         }
       }
     }
-    if constexpr (R >= 32) {
-      // the chunk is one piece of window q0 / R
-      const int w = q0 / R;
-      if (w < w_end) {
-        float mx = z[0];
-#pragma unroll
-        for (int j = 1; j < 32; ++j) mx = fmaxf(mx, z[j]);
-        const float mn = fmaxf(m, mx);
-        const float sc = __expf(m - mn);
-        l *= sc;
-        acc *= sc;
-#pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          const float pz = __expf(z[j] - mn);
-          l += pz;
-          acc = fmaf(pz, kv[j], acc);
-        }
-        m = mn;
-        if (((c + 1) * 32) % R == 0) {  // last chunk of the window
-          const int64_t n = off + (w - w0);
-          ybase[n * (COFF * p.D)] = acc / l;
-          if (COFF == 2) lbase[n * (COFF * p.D)] = m + __logf(l);
-          m = -INFINITY;
-          l = 0.f;
-          acc = 0.f;
-        }
-      }
-    } else {
+    {
 #pragma unroll
       for (int k = 0; k < 32 / R; ++k) {  // whole windows inside the chunk
         const int w = (q0 + k * R) / R;
@@ -340,6 +422,8 @@ __device__ __forceinline__ void pool_item(const Params& p, const Meta& md, const
       }
     }
   }
+  return true;
+  }
 }
 
 // Folded mode, one warp: output row n = window w of sequence b (first: w is the
@@ -353,8 +437,7 @@ __device__ __forceinline__ void pool_item(const Params& p, const Meta& md, const
 // store ("CANN PyPTO 算子实战", 压缩窗口与状态更新). Every load of the row is
 // issued before the first use, so a row costs about one memory round trip.
 template <int NG, int COFF>
-__device__ __forceinline__ void finish_window(const Params& p, int b, int w, int64_t n, bool first, int lane,
-                                              const float (&nw)[NG][4]) {
+__device__ __forceinline__ void finish_window(const Params& p, int b, int w, int64_t n, bool first, int lane) {
   constexpr int D = NG * 128;
   constexpr int kRope = 64;  // rope_head_dim (the only value the library accepts)
   const bool rope_lane = lane >= 16;  // group NG-1: channels D-64 .. D-1
@@ -368,6 +451,9 @@ __device__ __forceinline__ void finish_window(const Params& p, int b, int w, int
     s_lo = *reinterpret_cast<const __nv_bfloat162*>(sn + j);
     s_hi = *reinterpret_cast<const __nv_bfloat162*>(sn + 32 + j);
   }
+  uint2 wraw[NG];  // norm_weight of the lane's channels
+#pragma unroll
+  for (int i = 0; i < NG; ++i) wraw[i] = *reinterpret_cast<const uint2*>(p.norm_w + i * 128 + lane * 4);
   float4 yb[NG], lb[NG], ya[NG], la[NG];
   const bool prev_row = COFF == 2 && !first;
 #pragma unroll
@@ -451,9 +537,12 @@ __device__ __forceinline__ void finish_window(const Params& p, int b, int w, int
 #pragma unroll
   for (int i = 0; i < NG; ++i) {
     const int c = i * 128 + lane * 4;
+    const __nv_bfloat162 w01 = *reinterpret_cast<const __nv_bfloat162*>(&wraw[i].x);
+    const __nv_bfloat162 w23 = *reinterpret_cast<const __nv_bfloat162*>(&wraw[i].y);
+    const float nw[4] = {__low2float(w01), __high2float(w01), __low2float(w23), __high2float(w23)};
     float z[4];
 #pragma unroll
-    for (int u = 0; u < 4; ++u) z[u] = y[i][u] * inv * nw[i][u];
+    for (int u = 0; u < 4; ++u) z[u] = y[i][u] * inv * nw[u];
     if (i == NG - 1 && rope_lane) {
       const float ce[2] = {__low2float(c_lo), __high2float(c_lo)}, co[2] = {__low2float(c_hi), __high2float(c_hi)};
       const float se[2] = {__low2float(s_lo), __high2float(s_lo)}, so[2] = {__low2float(s_hi), __high2float(s_hi)};
@@ -486,19 +575,8 @@ __device__ void finish_tile_t(const Params& p, const Meta& md, int t, int ew, in
   const int w0 = s / R;
   const int wa = P0 / R, wb = min((P0 + NTOK) / R, e / R);
   const int64_t off = md.off[b];
-  float nw[NG][4];  // norm_weight of the lane's channels, shared by the rows
-#pragma unroll
-  for (int i = 0; i < NG; ++i) {
-    const uint2 wraw = *reinterpret_cast<const uint2*>(p.norm_w + i * 128 + lane * 4);
-    const __nv_bfloat162 w01 = *reinterpret_cast<const __nv_bfloat162*>(&wraw.x);
-    const __nv_bfloat162 w23 = *reinterpret_cast<const __nv_bfloat162*>(&wraw.y);
-    nw[i][0] = __low2float(w01);
-    nw[i][1] = __high2float(w01);
-    nw[i][2] = __low2float(w23);
-    nw[i][3] = __high2float(w23);
-  }
   for (int w = wa + ew; w < wb; w += kEpiThreads / 32)
-    finish_window<NG, COFF>(p, b, w, off + (w - w0), w == w0, lane, nw);
+    finish_window<NG, COFF>(p, b, w, off + (w - w0), w == w0, lane);
 }
 
 __device__ void finish_tile(const Params& p, const Meta& md, int t, int ew, int lane) {
@@ -632,20 +710,25 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint32_t acc_phase = 0;
     for (int g = blockIdx.x; g < total; g += gridDim.x) {
       const Item it = decode_item(p, md, g, n_cblk);
-      const bool ok = mbar_wait(&sm.acc_full, acc_phase, abort);
-      if (!bar_and(1, kEpiThreads, ok)) break;  // all eight warps leave together
-      tc_fence_after();
+      auto wait_acc = [&]() {
+        const bool ok = mbar_wait(&sm.acc_full, acc_phase, abort);
+        if (!bar_and(1, kEpiThreads, ok)) return false;  // all eight warps leave together
+        tc_fence_after();
+        return true;
+      };
       const int ch = it.c0 + row;
+      bool ok;
       switch (p.ratio) {
-        case 1: pool_item<1>(p, md, it, taddr, ch, hp); break;
-        case 2: pool_item<2>(p, md, it, taddr, ch, hp); break;
-        case 4: pool_item<4>(p, md, it, taddr, ch, hp); break;
-        case 8: pool_item<8>(p, md, it, taddr, ch, hp); break;
-        case 16: pool_item<16>(p, md, it, taddr, ch, hp); break;
-        case 32: pool_item<32>(p, md, it, taddr, ch, hp); break;
-        case 64: pool_item<64>(p, md, it, taddr, ch, hp); break;
-        default: pool_item<128>(p, md, it, taddr, ch, hp); break;
+        case 1: ok = pool_item<1>(p, md, it, taddr, ch, hp, wait_acc); break;
+        case 2: ok = pool_item<2>(p, md, it, taddr, ch, hp, wait_acc); break;
+        case 4: ok = pool_item<4>(p, md, it, taddr, ch, hp, wait_acc); break;
+        case 8: ok = pool_item<8>(p, md, it, taddr, ch, hp, wait_acc); break;
+        case 16: ok = pool_item<16>(p, md, it, taddr, ch, hp, wait_acc); break;
+        case 32: ok = pool_item<32>(p, md, it, taddr, ch, hp, wait_acc); break;
+        case 64: ok = pool_item<64>(p, md, it, taddr, ch, hp, wait_acc); break;
+        default: ok = pool_item<128>(p, md, it, taddr, ch, hp, wait_acc); break;
       }
+      if (!ok) break;
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&sm.acc_empty);

@@ -53,16 +53,23 @@ __global__ void __launch_bounds__(128) pool_kernel(Params p) {
   __shared__ float zs[1024];  // 2 D floats: the Hadamard product's exchange buffers
   __shared__ RowSrc src[kMaxRows];
   __shared__ int32_t off_s[kMaxStagedSeqs + 1];
+  __shared__ int32_t cu_s[kMaxStagedSeqs + 1];
+  __shared__ int32_t s_s[kMaxStagedSeqs];
   const int n = blockIdx.x;
   const int D = p.D, C = p.C, r = p.ratio;
   const int c = threadIdx.x * 4;
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
   pdl_wait();  // everything below reads what the earlier kernels of the call wrote
 
-  // which sequence owns row n (search the row offsets; staged when B is small)
-  int b;
-  if (p.B <= kMaxStagedSeqs) {
-    for (int i = threadIdx.x; i <= p.B; i += blockDim.x) off_s[i] = p.m_off[i];
+  // which sequence owns row n: its metadata is staged in one round trip of
+  // independent loads (when B is small), then searched in shared memory
+  int b, s = 0, cu = 0, e = 0;
+  const bool staged = p.B <= kMaxStagedSeqs;
+  if (staged) {
+    for (int i = threadIdx.x; i <= p.B; i += blockDim.x) {
+      off_s[i] = p.m_off[i];
+      cu_s[i] = p.m_cu[i];
+      if (i < p.B) s_s[i] = p.m_s[i];
+    }
     __syncthreads();
     int lo = 0, hi = p.B;
     while (lo < hi) {
@@ -73,12 +80,13 @@ __global__ void __launch_bounds__(128) pool_kernel(Params p) {
   } else {
     b = upper_index(p.m_off, p.B, n);
   }
-  int w = -1, s = 0, cu = 0;
+  int w = -1, off = 0;
   if (b < p.B) {
-    s = p.m_s[b];
-    cu = p.m_cu[b];
-    const int e = s + (p.m_cu[b + 1] - cu);
-    const int k = n - p.m_off[b];
+    s = staged ? s_s[b] : p.m_s[b];
+    cu = staged ? cu_s[b] : p.m_cu[b];
+    e = s + ((staged ? cu_s[b + 1] : p.m_cu[b + 1]) - cu);
+    off = staged ? off_s[b] : p.m_off[b];
+    const int k = n - off;
     if (k < e / r - s / r) w = s / r + k;
   }
   uint2* dst = reinterpret_cast<uint2*>(p.out + (int64_t)n * D + c);
@@ -86,8 +94,10 @@ __global__ void __launch_bounds__(128) pool_kernel(Params p) {
     *dst = make_uint2(0u, 0u);
     return;
   }
+  const RowAux aux = load_row_aux(p, n, c);  // independent of the pooling: in flight meanwhile
 
-  // 1) resolve every row of the window (table lookups in parallel)
+  // 1) resolve every row of the window (table lookups only for rows before
+  //    start_pos, i.e. the first window of the sequence)
   const int rows = p.coff * r;
   for (int j = threadIdx.x; j < rows; j += blockDim.x) {
     const bool bhalf = p.coff == 1 || j >= r;
@@ -153,7 +163,7 @@ __global__ void __launch_bounds__(128) pool_kernel(Params p) {
 #pragma unroll
   for (int i = 0; i < 4; ++i) y[i] = l[i] > 0.f ? a[i] / l[i] : 0.f;
 
-  finish_row(p, n, c, y, red, zs);
+  finish_row(p, n, c, y, red, zs, aux);
 }
 
 }  // namespace

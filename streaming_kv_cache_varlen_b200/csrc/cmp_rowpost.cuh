@@ -64,16 +64,48 @@ __device__ __forceinline__ void fwht_row(float (&z)[4], int D, bool active, floa
   for (int i = 0; i < 4; ++i) z[i] *= c;
 }
 
+// What the row tail of channels c .. c+3 of output row n reads besides the
+// pooled values: norm_weight, and the RoPE table entries when c lies in the
+// last rope_head_dim channels. Loaded before the pooled values are known, so
+// these loads overlap the pooling's.
+struct RowAux {
+  uint2 w;                         // norm_weight[c .. c+3] (bf16)
+  __nv_bfloat162 c_lo, c_hi;       // cos[j], cos[j+1] and cos[rope/2 + j], cos[rope/2 + j + 1]
+  __nv_bfloat162 s_lo, s_hi;       // the same for sin; j = (c - (D - rope)) / 2
+  bool sylv;                       // hadamard_is_sylvester (the same in every thread)
+};
+
+// Every thread of the CTA calls it (sylv must agree across the CTA); the
+// channel loads are made by the threads that hold channels (active).
+__device__ __forceinline__ RowAux load_row_aux(const Params& p, int n, int c, bool active = true) {
+  RowAux a{};
+  a.sylv = hadamard_is_sylvester(p);
+  if (!active) return a;
+  a.w = *reinterpret_cast<const uint2*>(p.norm_w + c);
+  const int r0 = p.D - p.rope;
+  if (c >= r0) {
+    const int j = (c - r0) >> 1;  // even: c - r0 is a multiple of 4
+    const __nv_bfloat16* cs = p.cos + (int64_t)n * p.rope;
+    const __nv_bfloat16* sn = p.sin + (int64_t)n * p.rope;
+    a.c_lo = *reinterpret_cast<const __nv_bfloat162*>(cs + j);
+    a.c_hi = *reinterpret_cast<const __nv_bfloat162*>(cs + p.rope / 2 + j);
+    a.s_lo = *reinterpret_cast<const __nv_bfloat162*>(sn + j);
+    a.s_hi = *reinterpret_cast<const __nv_bfloat162*>(sn + p.rope / 2 + j);
+  }
+  return a;
+}
+
 // Threads 0 .. D/4-1 of the CTA hold the pooled values y of channels
-// c = 4i .. 4i+3 of output row n (thread i); any further threads only take part
-// in the barriers. red: >= D/128 floats of shared memory, zs: >= 2 D floats of
-// shared memory. Every thread of the CTA must call it.
+// c = 4i .. 4i+3 of output row n (thread i) and their RowAux; any further
+// threads only take part in the barriers. red: >= D/128 floats of shared
+// memory, zs: >= 2 D floats of shared memory. Every thread of the CTA must
+// call it.
 __device__ __forceinline__ void finish_row(const Params& p, int n, int c, const float (&y)[4], float* red,
-                                           float* zs) {
+                                           float* zs, const RowAux& aux) {
   const int D = p.D;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = D / 128;
   const bool active = (int)threadIdx.x < D / 4;
-  const bool sylv = hadamard_is_sylvester(p);
+  const bool sylv = aux.sylv;
   // RMSNorm over the D channels of the row
   float ss = active ? y[0] * y[0] + y[1] * y[1] + y[2] * y[2] + y[3] * y[3] : 0.f;
 #pragma unroll
@@ -92,26 +124,23 @@ __device__ __forceinline__ void finish_row(const Params& p, int n, int c, const 
     }
     return;
   }
-  const uint2 wraw = *reinterpret_cast<const uint2*>(p.norm_w + c);
-  const __nv_bfloat162 w01 = *reinterpret_cast<const __nv_bfloat162*>(&wraw.x);
-  const __nv_bfloat162 w23 = *reinterpret_cast<const __nv_bfloat162*>(&wraw.y);
+  const __nv_bfloat162 w01 = *reinterpret_cast<const __nv_bfloat162*>(&aux.w.x);
+  const __nv_bfloat162 w23 = *reinterpret_cast<const __nv_bfloat162*>(&aux.w.y);
   float z[4] = {y[0] * inv * __low2float(w01), y[1] * inv * __high2float(w01),
                 y[2] * inv * __low2float(w23), y[3] * inv * __high2float(w23)};
 
-  // interleaved RoPE on the last rope channels
-  const int r0 = D - p.rope;
-  if (c >= r0) {
-    const int half = p.rope / 2;
-    const __nv_bfloat16* cs = p.cos + (int64_t)n * p.rope;
-    const __nv_bfloat16* sn = p.sin + (int64_t)n * p.rope;
+  // interleaved RoPE on the last rope channels: pair (c + i, c + i + 1) takes
+  // table columns j + i/2 and rope/2 + j + i/2
+  if (c >= D - p.rope) {
+    const float ce[2] = {__low2float(aux.c_lo), __high2float(aux.c_lo)};
+    const float co[2] = {__low2float(aux.c_hi), __high2float(aux.c_hi)};
+    const float se[2] = {__low2float(aux.s_lo), __high2float(aux.s_lo)};
+    const float so[2] = {__low2float(aux.s_hi), __high2float(aux.s_hi)};
 #pragma unroll
-    for (int i = 0; i < 4; i += 2) {
-      const int j = (c + i - r0) >> 1;
-      const float ce = __bfloat162float(cs[j]), se = __bfloat162float(sn[j]);
-      const float co = __bfloat162float(cs[half + j]), so = __bfloat162float(sn[half + j]);
-      const float ev = z[i], od = z[i + 1];
-      z[i] = ev * ce - od * se;
-      z[i + 1] = od * co + ev * so;
+    for (int i = 0; i < 2; ++i) {
+      const float ev = z[2 * i], od = z[2 * i + 1];
+      z[2 * i] = ev * ce[i] - od * se[i];
+      z[2 * i + 1] = od * co[i] + ev * so[i];
     }
   }
 
@@ -142,6 +171,13 @@ __device__ __forceinline__ void finish_row(const Params& p, int n, int c, const 
   v.x = *reinterpret_cast<uint32_t*>(&o01);
   v.y = *reinterpret_cast<uint32_t*>(&o23);
   *reinterpret_cast<uint2*>(p.out + (int64_t)n * D + c) = v;
+}
+
+// The same with the RowAux loads issued here (only the active threads load).
+__device__ __forceinline__ void finish_row(const Params& p, int n, int c, const float (&y)[4], float* red,
+                                           float* zs) {
+  const RowAux aux = load_row_aux(p, n, c, (int)threadIdx.x < p.D / 4);
+  finish_row(p, n, c, y, red, zs, aux);
 }
 
 
