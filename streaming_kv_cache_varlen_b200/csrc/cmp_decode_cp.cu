@@ -130,7 +130,7 @@ struct Smem {
   alignas(16) float4 hst[kMaxOut][OWN];          // per window and channel: the state rows' running
                                                  // max, exp-sum and weighted sum
   float norm[OWN];
-  float hcol[512][OWN];     // rotation: this CTA's columns of the hadamard matrix
+  alignas(16) float hcolT[OWN][512];  // rotation: this CTA's columns of the hadamard matrix (column-major)
   TokInfo tok[MAXT];
   Win win[kMaxOut];
   int32_t cu[kMaxSeqs + 1];
@@ -345,10 +345,10 @@ __device__ void call_metadata(const Params& p, Smem<MAXT>& sm, int NT, int ch0) 
       if (k < p.D) {
         const __nv_bfloat162 h01 = *reinterpret_cast<const __nv_bfloat162*>(&hv[u].x);
         const __nv_bfloat162 h23 = *reinterpret_cast<const __nv_bfloat162*>(&hv[u].y);
-        sm.hcol[k][0] = __low2float(h01);
-        sm.hcol[k][1] = __high2float(h01);
-        sm.hcol[k][2] = __low2float(h23);
-        sm.hcol[k][3] = __high2float(h23);
+        sm.hcolT[0][k] = __low2float(h01);
+        sm.hcolT[1][k] = __high2float(h01);
+        sm.hcolT[2][k] = __low2float(h23);
+        sm.hcolT[3][k] = __high2float(h23);
       }
     }
   }
@@ -795,7 +795,14 @@ __device__ void exchange_sums(const Params& p, Smem<MAXT>& sm, const CpArgs& a, 
   }
   CP_STAMP(lane == 0, 11);  // all CTAs arrived
   got = __shfl_sync(0xffffffffu, got, 0);
+  if (!got && lane == 0) {
+    atomicOr(p.err, kErrTimeout);
+    sm.xch_ok = 0;
+  }
   warp_sync_all();
+  // rotation: warps 1-3 load every window's u while this warp reads the sums
+  // (the barrier carries this warp's acquire to them)
+  if (p.rotate) asm volatile("bar.arrive 5, 128;" ::: "memory");
   if (got) {
     const int per_lane = (int)gridDim.x / 32;  // 1 or 4 partials per lane and window
     for (int i0 = 0; i0 < nw; i0 += 8) {
@@ -814,60 +821,65 @@ __device__ void exchange_sums(const Params& p, Smem<MAXT>& sm, const CpArgs& a, 
         if (lane == 0 && i0 + u < nw) sm.ss_tot[i0 + u] = t;
       }
     }
-  } else if (lane == 0) {
-    atomicOr(p.err, kErrTimeout);
-    sm.xch_ok = 0;
   }
   warp_sync_all();
   CP_STAMP(lane == 0, 9);  // exchange complete
 }
 
+// Rotation, warps 1-3 (96 threads) once every CTA has arrived: every window's
+// u (all D channels, published with the arrivals) into the now idle A ring,
+// rows of D + 4 floats (16-byte aligned, rows on different banks), 8 loads in
+// flight per thread.
+template <int MAXT>
+__device__ void load_u_rows(const Params& p, Smem<MAXT>& sm, const CpArgs& a) {
+  asm volatile("bar.sync 5, 128;" ::: "memory");
+  if (sm.xch_ok == 0) return;
+  const int t = threadIdx.x - 32;
+  const int nw = sm.n_win;
+  const int per_row = p.D / 4;
+  const int n4 = nw * per_row;
+  float* uall = reinterpret_cast<float*>(&sm.a[0][0]);
+  for (int v0 = 0; v0 < n4; v0 += 96 * 8) {
+    float4 x4[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      const int v = v0 + t + 96 * e;
+      if (v < n4) x4[e] = __ldcg(reinterpret_cast<const float4*>(a.u + (int64_t)(v / per_row) * 512 + 4 * (v % per_row)));
+    }
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      const int v = v0 + t + 96 * e;
+      if (v < n4) *reinterpret_cast<float4*>(uall + (v / per_row) * (p.D + 4) + 4 * (v % per_row)) = x4[e];
+    }
+  }
+}
+
 // Warps 0-3: RMSNorm scale, norm_weight, RoPE and the bf16 store of this CTA's
 // channels of every window row; with the rotation, output column ch0 + c of a
 // window is scale * sum_k u[k] * hadamard[k][ch0 + c], one thread per (window,
-// column) adding over k in order (four interleaved partial sums).
+// column) adding over k in order (four interleaved partial sums, four k per
+// step from 16-byte shared-memory loads).
 template <int MAXT>
 __device__ void finish_rows(const Params& p, Smem<MAXT>& sm, const CpArgs& a, int ch0, bool ok) {
   const int tid = threadIdx.x;
   const int nw = sm.n_win;
   const bool fin = ok && sm.xch_ok != 0;
   if (p.rotate) {
-    // every window's u (all D channels, published before the arrivals) into
-    // the now idle A ring, rows padded by one float; 8 loads in flight per thread
-    float* uall = reinterpret_cast<float*>(&sm.a[0][0]);
-    if (fin) {
-      const int n4 = nw * p.D / 4;
-      for (int v0 = 0; v0 < n4; v0 += 128 * 8) {
-        float4 x4[8];
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          const int v = v0 + tid + 128 * e;
-          if (v < n4)
-            x4[e] = __ldcg(reinterpret_cast<const float4*>(a.u + (int64_t)((4 * v) / p.D) * 512 + (4 * v) % p.D));
-        }
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          const int v = v0 + tid + 128 * e;
-          if (v < n4) {
-            float* d = uall + ((4 * v) / p.D) * (p.D + 1) + (4 * v) % p.D;
-            d[0] = x4[e].x;
-            d[1] = x4[e].y;
-            d[2] = x4[e].z;
-            d[3] = x4[e].w;
-          }
-        }
-      }
-    }
-    epi_sync();
+    const float* uall = reinterpret_cast<const float*>(&sm.a[0][0]);
     for (int u = tid; u < nw * OWN; u += 128) {
       const int i = u / OWN, c = u % OWN;
       float o = 0.f;
       if (fin) {
-        const float* ui = uall + i * (p.D + 1);
+        const float* ui = uall + i * (p.D + 4);
+        const float* hc = sm.hcolT[c];
         float s4[4] = {0.f, 0.f, 0.f, 0.f};
         for (int k = 0; k < p.D; k += 4) {
-#pragma unroll
-          for (int e = 0; e < 4; ++e) s4[e] = fmaf(ui[k + e], sm.hcol[k + e][c], s4[e]);
+          const float4 uv = *reinterpret_cast<const float4*>(ui + k);
+          const float4 hv = *reinterpret_cast<const float4*>(hc + k);
+          s4[0] = fmaf(uv.x, hv.x, s4[0]);
+          s4[1] = fmaf(uv.y, hv.y, s4[1]);
+          s4[2] = fmaf(uv.z, hv.z, s4[2]);
+          s4[3] = fmaf(uv.w, hv.w, s4[3]);
         }
         o = ((s4[0] + s4[1]) + (s4[2] + s4[3])) * rsqrtf(sm.ss_tot[i] / (float)p.D + 1e-6f);
       }
@@ -1014,6 +1026,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (sm.win[n].w < 0) *reinterpret_cast<uint2*>(p.out + (int64_t)n * p.D + ch0) = make_uint2(0u, 0u);
       if (good) write_tails(p, sm, ch0, warp - 1);
       CP_STAMP(threadIdx.x == 32, 14);  // tails written
+      if (p.rotate) load_u_rows(p, sm, a);
     }
     epi_sync();
     finish_rows(p, sm, a, ch0, good);
@@ -1122,8 +1135,8 @@ int max_clusters(int (&conf)[64]) {
 
 bool decode_cp_supported(const Params& p) {
   if (p.T < 1 || p.T > 64 || p.B > kMaxSeqs || p.n_out > kMaxOut || p.rope != 64) return false;
-  // rotation: every window's u (n_out rows of D + 1 floats) fits in the A ring
-  if (p.rotate && (size_t)p.n_out * (p.D + 1) * 4 > sizeof(Smem<32>::a)) return false;
+  // rotation: every window's u (n_out rows of D + 4 floats) fits in the A ring
+  if (p.rotate && (size_t)p.n_out * (p.D + 4) * 4 > sizeof(Smem<32>::a)) return false;
   if (p.coff * p.ratio > kMaxWinRows || p.H % (KQ * KPS * BK) || p.D % GCH || kMaxClusters % (p.D / GCH) ||
       encode_fn() == nullptr)
     return false;

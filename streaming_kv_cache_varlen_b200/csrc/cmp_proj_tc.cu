@@ -12,7 +12,7 @@
 // accumulator lane is one channel and its columns are tokens: every epilogue
 // store of a warp is 32 consecutive channels of one token row (128 bytes).
 //
-// BN (128 .. 256 tokens, a multiple of 32) is chosen per call so that the
+// BN (128 .. 256 tokens, a multiple of 16) is chosen per call so that the
 // tiles fill the SMs in whole waves as nearly as possible: with 2C = 512 rows
 // and ~10K tokens, 256-token tiles make 160-200 tiles, i.e. a second wave that
 // keeps only a few SMs busy; narrower tiles spread the same work over all SMs.
@@ -72,11 +72,12 @@ __device__ __forceinline__ void epi_bar() { asm volatile("bar.sync 1, 128;" ::: 
 // Per-token facts of one tile, computed by the 128 epilogue threads while the
 // tile's main loop runs: which tokens are state tail rows and where they go.
 __device__ void fill_tok_info(const Params& p, TokInfo* info, uint32_t* tail_mask, int n0, int e_tid, int bn) {
-  for (int j = e_tid; j < bn; j += 128) {
+  const int bn32 = (bn + 31) & ~31;  // whole warps in the ballot (bn may end on half a chunk)
+  for (int j = e_tid; j < bn32; j += 128) {
     TokInfo ti{0, 0, -1, -1};
     bool tail = false;
     const int t = n0 + j;
-    if (t < p.T) {
+    if (j < bn && t < p.T) {
       const int b = upper_index(p.m_cu, p.B, t);
       if (b < p.B) {
         const int s = p.m_s[b];
@@ -93,7 +94,7 @@ __device__ void fill_tok_info(const Params& p, TokInfo* info, uint32_t* tail_mas
         }
       }
     }
-    info[j] = ti;
+    if (j < bn) info[j] = ti;
     const unsigned m = __ballot_sync(0xffffffffu, tail);  // j = e_tid + 128 i: one warp = one chunk
     if ((j & 31) == 0) tail_mask[j >> 5] = m;
   }
@@ -109,12 +110,23 @@ __device__ __forceinline__ void store_accumulator(const Params& p, uint32_t tadd
   float* proj_col = p.proj + (score ? p.C : 0) + col;
   float* state = score ? p.score_state : p.kv_state;
 #pragma unroll 1
-  for (int c = 0; c < bn / 32; ++c) {
+  for (int c = 0; c < (bn + 31) / 32; ++c) {
     uint32_t r[32];
-    tmem_ld32(taddr + c * 32, r);
-    tmem_ld_wait(r);
+    if (c * 32 + 32 <= bn) {
+      tmem_ld32(taddr + c * 32, r);
+      tmem_ld_wait(r);
+    } else {  // a last chunk of 16 columns (bn = 16 mod 32)
+      uint32_t h[16];
+      tmem_ld16(taddr + c * 32, h);
+      tmem_ld_wait16(h);
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        r[j] = h[j];
+        r[16 + j] = 0u;
+      }
+    }
     const int t0 = n0 + c * 32;
-    const int jmax = p.T - t0;  // tokens past T are padding
+    const int jmax = min(p.T - t0, bn - c * 32);  // tokens past T or past the tile are not stored
     float* dst = proj_col + (int64_t)t0 * (2 * p.C);
 #pragma unroll
     for (int j = 0; j < 32; ++j)
@@ -412,13 +424,13 @@ int sm_count() {
   return n;
 }
 
-// The tile width for T tokens: the fewest waves of tiles over the `slots`
-// concurrent tiles, each wave costing its tile width plus ~32 tokens' worth of
-// per-tile overhead (ties go to the wider tile).
+// The tile width for T tokens (128 .. 256, a multiple of 16): the fewest waves
+// of tiles over the `slots` concurrent tiles, each wave costing its tile width
+// plus ~32 tokens' worth of per-tile overhead (ties go to the wider tile).
 int tile_tokens(int64_t n_m, int T, int slots) {
   int best = BNMAX;
   int64_t best_cost = -1;
-  for (int bn = BNMAX; bn >= 128; bn -= 32) {
+  for (int bn = BNMAX; bn >= 128; bn -= 16) {
     const int64_t tiles = n_m * ((T + bn - 1) / bn);
     const int64_t cost = ((tiles + slots - 1) / slots) * (bn + 32);
     if (best_cost < 0 || cost < best_cost) {
