@@ -14,8 +14,9 @@ Also reported on the same line:
   * decode: the C4A 32-request decode step (one token each), microseconds per
     call, with L2 flushed before every timed call;
   * roofline: the projection kernel's tensor throughput against the measured
-    bf16 peak (with the pooling epilogue's HBM throughput beside it), and the
-    decode call's HBM throughput against measured bandwidth;
+    bf16 peak (with the pooling epilogue's HBM throughput beside it when it is
+    a separate launch), and the decode call's HBM throughput against measured
+    bandwidth;
   * nsa: the NsaCompressWithCache decode step (128 batches), microseconds per
     call with L2 flushed before every timed call, against HBM bandwidth;
   * configs: the other workloads (c4li_tiny, c4a_varlen, c4li_chunked),
@@ -457,8 +458,9 @@ def bench_prefill(args, ws, local, stream, peaks, peak_src):
                 "frac_of_burst": achieved / peaks["bf16_tflops"] if achieved else None,
                 "algorithmic_flops_per_launch": flops,
                 "kernel_ms": {k: (v[0] / v[1] if v[1] else None) for k, v in prof.items()}}
-    # the pooling epilogue that follows the fused projection (merge, RMSNorm,
-    # RoPE, bf16 store): HBM, its algorithmic bytes over its launch time
+    # the pooling epilogue that follows the fused projection when it is a separate
+    # launch (merge, RMSNorm, RoPE, bf16 store): HBM, its algorithmic bytes over its
+    # launch time (calls without rotation finish their rows inside the fused kernel)
     f_ms, f_n = prof["finish"]
     if f_n:
         n_out, coff, D = out.shape[0], (2 if PREFILL["ratio"] == 4 else 1), PREFILL["D"]
