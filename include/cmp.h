@@ -320,7 +320,9 @@ CMP_API int cmp_debug_phase_stamps(uint64_t* dst, int64_t n);
  * fill the SMs twice; else the tcgen05 projection + pooling kernel), 1 = force the mma.sync projection, 2 = the tcgen05 projection
  * (on CTA pairs, cta_group::2, where the device can co-schedule them),
  * 3 = weight streaming, 4 = the fused path, 5 = the K-split one-kernel decode,
- * 6 = the channel-group decode, 7 = the tcgen05 projection on single CTAs.
+ * 6 = the channel-group decode, 7 = the tcgen05 projection on single CTAs,
+ * 8 = the fused path on single CTAs (4 runs on CTA pairs, cta_group::2, when
+ * coff * D / 128 is even and the device co-schedules them).
  * A forced path a call cannot take falls back to 1.
  * Returns the previous value, or -1 if out of range. */
 CMP_API int cmp_set_proj_kernel(int which);

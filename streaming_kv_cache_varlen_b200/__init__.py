@@ -340,8 +340,9 @@ def debug_unreachable_barrier(launches: int) -> int:
 def set_proj_kernel(which: int) -> int:
     """Testing knob, which path calls take: 0 automatic, 1 mma.sync projection,
     2 tcgen05 projection (on CTA pairs where the device co-schedules them), 3 weight
-    streaming, 4 fused tcgen05 pooling, 5 K-split one-kernel decode, 6 channel-group
-    one-kernel decode, 7 tcgen05 projection on single CTAs. Returns the previous value."""
+    streaming, 4 fused tcgen05 pooling (on CTA pairs when the channel blocks pair up),
+    5 K-split one-kernel decode, 6 channel-group one-kernel decode, 7 tcgen05
+    projection on single CTAs, 8 fused path on single CTAs. Returns the previous value."""
     return int(lib.cmp_set_proj_kernel(which))
 
 

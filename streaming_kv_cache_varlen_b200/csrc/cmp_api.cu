@@ -366,7 +366,7 @@ size_t cmp_workspace_size(const cmp_dims* dims, int32_t ratio) {
   p.ratio = ratio;
   p.n_out = (int)cmp_out_rows(p.B, p.T, ratio);
   const int knob = g_proj_kernel.load();
-  const int which = choose_path(p, knob == 7 ? 2 : knob);
+  const int which = choose_path(p, knob == 7 ? 2 : knob == 8 ? 4 : knob);
   return ws_layout(dims->B, dims->T, p.C, p.n_out, which == 4, decode_part_bytes(p, which)).total +
          cmp::proj_decode_workspace(p);
 }
@@ -448,8 +448,8 @@ int cmp_compressor(const cmp_bf16* x, float* kv_state, float* score_state,
 
   for (int attempt = 0; attempt < 2; ++attempt) {
     const int knob = g_proj_kernel.load();
-    p.single_cta = knob == 7 ? 1 : 0;
-    const int r2 = run_path(p, choose_path(p, knob == 7 ? 2 : knob), s);
+    p.single_cta = (knob == 7 || knob == 8) ? 1 : 0;
+    const int r2 = run_path(p, choose_path(p, knob == 7 ? 2 : knob == 8 ? 4 : knob), s);
     // the device refused the channel-group decode's launch form (nothing ran):
     // the path is now disabled there and the next choice is taken
     if (r2 != kRetryOtherPath) return r2;
@@ -609,7 +609,7 @@ int cmp_profile_stop(double* ms, int64_t* launches) {
 }
 
 int cmp_set_proj_kernel(int which) {
-  if (which < 0 || which > 7) return -1;
+  if (which < 0 || which > 8) return -1;
   return g_proj_kernel.exchange(which);
 }
 

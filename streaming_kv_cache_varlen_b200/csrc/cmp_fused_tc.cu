@@ -59,19 +59,28 @@ namespace {
 using namespace sm100;
 
 constexpr int NTOK = 256;   // positions per tile (MMA N)
-constexpr int BM = 128;     // channels per item (MMA M)
+constexpr int BM = 128;     // channels per item (MMA M per CTA)
 constexpr int BK = 64;
-constexpr int STAGES = 3;
 constexpr int kThreads = 320;
 constexpr int kEpiThreads = 256;  // warps 2-9
 constexpr int kMetaSeqs = 512;    // folded mode: sequences whose metadata fits in shared memory
-constexpr uint32_t kStageBytes = 2 * BM * BK * 2 + NTOK * BK * 2;  // 64 KB
-constexpr uint32_t kIdesc = idesc_bf16_f32(BM, NTOK);
 
-struct Smem {
+// Single CTAs: 3 stages of 16 + 16 + 32 KB (the whole 256-position x tile).
+// CTA pairs: 4 stages of 16 + 16 + 16 KB (each CTA holds half of the x tile).
+template <bool PAIR>
+struct Cfg {
+  static constexpr int ST = PAIR ? 4 : 3;
+  static constexpr int NB = PAIR ? NTOK / 2 : NTOK;  // x rows per CTA and stage
+  static constexpr uint32_t kStageBytes = 2 * BM * BK * 2 + NB * BK * 2;
+  static constexpr uint32_t kIdesc = idesc_bf16_f32(PAIR ? 2 * BM : BM, NTOK);
+};
+
+template <bool PAIR>
+struct SmemT {
+  static constexpr int STAGES = Cfg<PAIR>::ST;
   __nv_bfloat16 a_kv[STAGES][BM * BK];
   __nv_bfloat16 a_g[STAGES][BM * BK];
-  __nv_bfloat16 b[STAGES][NTOK * BK];
+  __nv_bfloat16 b[STAGES][Cfg<PAIR>::NB * BK];
   uint64_t full[STAGES];
   uint64_t empty[STAGES];
   uint64_t acc_full;
@@ -148,6 +157,7 @@ __device__ __forceinline__ int cta_exclusive_scan(int v, int* wsum, int* total) 
 // int32; a rejected call gets empty sequences, so every output row is 0;
 // sequence b reserves min(L, L/ratio + 1) output rows; its work tiles cover
 // positions from start_pos rounded down to the ratio to its end).
+template <class Smem>
 __device__ void build_meta(const Params& p, Smem& sm) {
   const int B = p.B;
   if (threadIdx.x == 0) sm.bad = 0;
@@ -609,15 +619,23 @@ __device__ void zero_rows(const Params& p, const Meta& md, int ew, int lane) {
   if (blockIdx.x == 0) zero(md.off[p.B], p.n_out);
 }
 
-template <bool FOLD>
+template <bool FOLD, bool PAIR>
 __global__ void __launch_bounds__(kThreads, 1)
     fused_tc_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUtensorMap map_wkv,
                     const __grid_constant__ CUtensorMap map_wg, Params p) {
+  using C = Cfg<PAIR>;
+  using Smem = SmemT<PAIR>;
+  constexpr int STAGES = C::ST;
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   Smem& sm = smem_align1024<Smem>(smem_raw);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int n_cblk = p.coff * p.D / BM;
   const int k_blocks = p.H / BK;
+  // CTA pairs: rank 0 issues the pair's MMAs; a work unit is two items (channel
+  // blocks 2c and 2c + 1 of one tile), the CTA of rank r pooling item 2u + r
+  const uint32_t rank = PAIR ? cluster_ctarank() : 0u;
+  const int unit0 = PAIR ? (int)(blockIdx.x >> 1) : (int)blockIdx.x;
+  const int ustep = PAIR ? (int)(gridDim.x >> 1) : (int)gridDim.x;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -625,20 +643,26 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&sm.empty[s], 1);
     }
     mbar_init(&sm.acc_full, 1);
-    mbar_init(&sm.acc_empty, kEpiThreads / 32);
+    mbar_init(&sm.acc_empty, (PAIR ? 2 : 1) * kEpiThreads / 32);  // epilogue warps (of both CTAs)
     sm.abort = 0;
     fence_barrier_init();
     prefetch_tmap(&map_x);
     prefetch_tmap(&map_wkv);
     prefetch_tmap(&map_wg);
   }
-  if (warp == 1) tmem_alloc(&sm.tmem_base, 512);
+  if (warp == 1) {
+    if constexpr (PAIR) tmem_alloc_pair(&sm.tmem_base, 512);
+    else tmem_alloc(&sm.tmem_base, 512);
+  }
   if constexpr (FOLD) build_meta(p, sm);  // reads only this call's inputs
   tc_fence_before();
   __syncthreads();
+  if constexpr (PAIR) cluster_sync_all();  // both CTAs' barriers exist before either signals the other's
   tc_fence_after();
   const uint32_t tmem = sm.tmem_base;
   volatile int* abort = &sm.abort;
+  const uint32_t full0 = PAIR ? mapa_shared(smem_u32(&sm.full[0]), 0) : 0u;  // the even CTA's barriers
+  const uint32_t acc_empty0 = PAIR ? mapa_shared(smem_u32(&sm.acc_empty), 0) : 0u;
   pdl_trigger();
   Meta md;
   if constexpr (FOLD) {
@@ -648,30 +672,41 @@ __global__ void __launch_bounds__(kThreads, 1)
     md = Meta{p.m_cu, p.m_s, p.m_off, p.m_tile};
   }
   const int total = md.tile[p.B] * n_cblk;
+  const int n_units = PAIR ? total / 2 : total;
 
   if (warp == 0) {
     if (lane == 0) {
       int stage = 0;
       uint32_t phase = 0;
-      for (int g = blockIdx.x; g < total && !*abort; g += gridDim.x) {
+      for (int u = unit0; u < n_units && !*abort; u += ustep) {
+        const int g = PAIR ? 2 * u + (int)rank : u;
         const Item it = decode_item(p, md, g, n_cblk);
         const int wrow = it.half * p.D + it.c0;
+        const int xrow = it.t0 + (int)rank * C::NB;  // pairs: this CTA's half of the positions
         for (int kb = 0; kb < k_blocks; ++kb) {
           if (!mbar_wait(&sm.empty[stage], phase ^ 1u, abort)) break;
-          mbar_arrive_expect_tx(&sm.full[stage], kStageBytes);
-          tma_load_2d(sm.a_kv[stage], &map_wkv, &sm.full[stage], kb * BK, wrow);
-          tma_load_2d(sm.a_g[stage], &map_wg, &sm.full[stage], kb * BK, wrow);
-          tma_load_2d(sm.b[stage], &map_x, &sm.full[stage], kb * BK, it.t0);
+          if constexpr (PAIR) {
+            if (rank == 0) mbar_arrive_expect_tx(&sm.full[stage], 2 * C::kStageBytes);
+            const uint32_t fb = full0 + 8u * stage;
+            tma_load_2d_pair(sm.a_kv[stage], &map_wkv, fb, kb * BK, wrow);
+            tma_load_2d_pair(sm.a_g[stage], &map_wg, fb, kb * BK, wrow);
+            tma_load_2d_pair(sm.b[stage], &map_x, fb, kb * BK, xrow);
+          } else {
+            mbar_arrive_expect_tx(&sm.full[stage], C::kStageBytes);
+            tma_load_2d(sm.a_kv[stage], &map_wkv, &sm.full[stage], kb * BK, wrow);
+            tma_load_2d(sm.a_g[stage], &map_wg, &sm.full[stage], kb * BK, wrow);
+            tma_load_2d(sm.b[stage], &map_x, &sm.full[stage], kb * BK, xrow);
+          }
           if (++stage == STAGES) { stage = 0; phase ^= 1u; }
         }
       }
     }
   } else if (warp == 1) {
-    if (lane == 0) {
+    if (lane == 0 && rank == 0) {
       int stage = 0;
       uint32_t phase = 0;
       uint32_t acc_phase = 0;
-      for (int g = blockIdx.x; g < total && !*abort; g += gridDim.x) {
+      for (int u = unit0; u < n_units && !*abort; u += ustep) {
         if (!mbar_wait(&sm.acc_empty, acc_phase ^ 1u, abort)) break;
         tc_fence_after();
         bool ok = true;
@@ -685,14 +720,21 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int k = 0; k < BK / 16; ++k) {
             const uint64_t bd = sw128_kmajor_desc(b0 + k * 32);
             const uint32_t accum = (kb > 0 || k > 0) ? 1u : 0u;
-            mma_bf16(tmem, sw128_kmajor_desc(akv + k * 32), bd, kIdesc, accum);
-            mma_bf16(tmem + NTOK, sw128_kmajor_desc(ag + k * 32), bd, kIdesc, accum);
+            if constexpr (PAIR) {
+              mma_bf16_pair(tmem, sw128_kmajor_desc(akv + k * 32), bd, C::kIdesc, accum);
+              mma_bf16_pair(tmem + NTOK, sw128_kmajor_desc(ag + k * 32), bd, C::kIdesc, accum);
+            } else {
+              mma_bf16(tmem, sw128_kmajor_desc(akv + k * 32), bd, C::kIdesc, accum);
+              mma_bf16(tmem + NTOK, sw128_kmajor_desc(ag + k * 32), bd, C::kIdesc, accum);
+            }
           }
-          mma_commit(&sm.empty[stage]);
+          if constexpr (PAIR) mma_commit_pair(&sm.empty[stage], 0x3);  // frees the stage in both CTAs
+          else mma_commit(&sm.empty[stage]);
           if (++stage == STAGES) { stage = 0; phase ^= 1u; }
         }
         if (!ok) break;
-        mma_commit(&sm.acc_full);
+        if constexpr (PAIR) mma_commit_pair(&sm.acc_full, 0x3);
+        else mma_commit(&sm.acc_full);
         acc_phase ^= 1u;
       }
     }
@@ -708,7 +750,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       zero_rows(p, md, ew, lane);
     }
     uint32_t acc_phase = 0;
-    for (int g = blockIdx.x; g < total; g += gridDim.x) {
+    for (int u = unit0; u < n_units; u += ustep) {
+      const int g = PAIR ? 2 * u + (int)rank : u;
       const Item it = decode_item(p, md, g, n_cblk);
       auto wait_acc = [&]() {
         const bool ok = mbar_wait(&sm.acc_full, acc_phase, abort);
@@ -731,7 +774,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!ok) break;
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&sm.acc_empty);
+      if (lane == 0) {
+        if constexpr (PAIR) mbar_arrive_cluster(acc_empty0);
+        else mbar_arrive(&sm.acc_empty);
+      }
       acc_phase ^= 1u;
       if constexpr (FOLD) {
         // arrive on the tile's counter (coff = 2: also on the next tile's); the
@@ -767,9 +813,11 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   tc_fence_before();
   __syncthreads();
+  if constexpr (PAIR) cluster_sync_all();  // neither CTA leaves while the other may still signal it
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, 512);
+    if constexpr (PAIR) tmem_dealloc_pair(tmem, 512);
+    else tmem_dealloc(tmem, 512);
   }
   if (threadIdx.x == 0 && sm.abort) atomicOr(p.err, kErrTimeout);
 }
@@ -788,22 +836,83 @@ bool fused_fold_supported(const Params& p) {
   return !p.rotate && p.B <= kMetaSeqs && fused_max_tiles(p) + 1 <= kFusedTileCounters;
 }
 
-cudaError_t launch_fused(const Params& p, cudaStream_t s, int sm_count) {
+namespace {
+
+// Per device: co-resident 2-CTA clusters of the pair kernels (0: not measured
+// yet, -1: the device refused the cluster form).
+int g_fused_pair_slots[64] = {0};
+
+template <bool FOLD, bool PAIR>
+cudaError_t launch_form(const Params& p, cudaStream_t s, int units) {
   CUtensorMap mx, mkv, mg;
-  if (!make_tile_map(&mx, p.x, p.T, p.H, NTOK) || !make_tile_map(&mkv, p.wkv, p.C, p.H, BM) ||
+  if (!make_tile_map(&mx, p.x, p.T, p.H, Cfg<PAIR>::NB) || !make_tile_map(&mkv, p.wkv, p.C, p.H, BM) ||
       !make_tile_map(&mg, p.wgate, p.C, p.H, BM))
     return cudaErrorInvalidValue;
-  const size_t smem = sizeof(Smem) + 1024;
-  const bool fold = p.tile_cnt != nullptr;
-  static int configured[2][64] = {{0}};
-  const cudaError_t e = fold ? smem_attr_once(fused_tc_kernel<true>, smem, configured[1])
-                             : smem_attr_once(fused_tc_kernel<false>, smem, configured[0]);
+  const size_t smem = sizeof(SmemT<PAIR>) + 1024;
+  static int configured[64] = {0};
+  const cudaError_t e = smem_attr_once(fused_tc_kernel<FOLD, PAIR>, smem, configured);
   if (e != cudaSuccess) return e;
-  const int64_t items = fused_max_tiles(p) * (p.coff * p.D / BM);
+  const int grid = PAIR ? 2 * units : units;
+  return launch_chained(fused_tc_kernel<FOLD, PAIR>, dim3(grid), dim3(kThreads), smem, s, PAIR ? 2 : 1, mx, mkv, mg,
+                        p);
+}
+
+// How many 2-CTA clusters of the pair kernel fit at once (-1: none).
+template <bool FOLD>
+int pair_slots(int dev) {
+  int& slots = g_fused_pair_slots[dev];
+  if (slots != 0) return slots;
+  static int configured[64] = {0};
+  const size_t smem = sizeof(SmemT<true>) + 1024;
+  if (smem_attr_once(fused_tc_kernel<FOLD, true>, smem, configured) != cudaSuccess) {
+    cudaGetLastError();
+    return slots = -1;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = smem;
+  cudaLaunchAttribute attr;
+  attr.id = cudaLaunchAttributeClusterDimension;
+  attr.val.clusterDim.x = 2;
+  attr.val.clusterDim.y = 1;
+  attr.val.clusterDim.z = 1;
+  cfg.attrs = &attr;
+  cfg.numAttrs = 1;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, fused_tc_kernel<FOLD, true>, &cfg) != cudaSuccess || n < 1) {
+    cudaGetLastError();
+    return slots = -1;
+  }
+  return slots = n;
+}
+
+}  // namespace
+
+// CTA pairs (cta_group::2) when the channel blocks pair up (coff * D / 128
+// even) and the device co-schedules the clusters, unless the call asks for
+// single CTAs; the one-kernel form when p.tile_cnt is set.
+cudaError_t launch_fused(const Params& p, cudaStream_t s, int sm_count) {
+  const bool fold = p.tile_cnt != nullptr;
+  const int n_cblk = p.coff * p.D / BM;
+  const int64_t items = fused_max_tiles(p) * n_cblk;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (n_cblk % 2 == 0 && !p.single_cta && dev < 64) {
+    const int slots = fold ? pair_slots<true>(dev) : pair_slots<false>(dev);
+    if (slots > 0) {
+      const int64_t units = items / 2;
+      const int u = units < slots ? (int)units : slots;
+      const cudaError_t e = fold ? launch_form<true, true>(p, s, u) : launch_form<false, true>(p, s, u);
+      if (e == cudaSuccess) return e;
+      // the launch was refused before anything ran (a cluster form this device
+      // will not schedule): single CTAs from now on
+      cudaGetLastError();
+      g_fused_pair_slots[dev] = -1;
+    }
+  }
   const int grid = items < sm_count ? (int)items : sm_count;
-  if (fold)
-    return launch_chained(fused_tc_kernel<true>, dim3(grid), dim3(kThreads), smem, s, 1, mx, mkv, mg, p);
-  return launch_chained(fused_tc_kernel<false>, dim3(grid), dim3(kThreads), smem, s, 1, mx, mkv, mg, p);
+  return fold ? launch_form<true, false>(p, s, grid) : launch_form<false, false>(p, s, grid);
 }
 
 }  // namespace cmp

@@ -521,7 +521,11 @@ cudaError_t launch_proj_tc(const Params& p, cudaStream_t s) {
   const int sms = sm_count();
   if (p.T >= 256 && (2 * p.C) % BMP == 0 && dev < 64 && g_pair_slots[dev] >= 0 && !p.single_cta) {
     const cudaError_t e = launch_pair(p, s, dev);
-    if (e != cudaErrorNotSupported) return e;
+    if (e == cudaSuccess || e == cudaErrorInvalidValue) return e;
+    // refused before anything ran (a cluster form this device will not
+    // schedule): single CTAs from now on
+    cudaGetLastError();
+    g_pair_slots[dev] = -1;
   }
   return launch_single(p, s, sms);
 }

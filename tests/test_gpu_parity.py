@@ -35,8 +35,9 @@ def check(cmp, inp, rows=None):
     return out, kv, sc, res
 
 
-@pytest.fixture(params=[0, 1, 2, 3, 4, 5, 6, 7],
-                ids=["auto", "mma", "tcgen05", "decode", "fused", "decode1k", "decodecp", "tcgen05single"])
+@pytest.fixture(params=[0, 1, 2, 3, 4, 5, 6, 7, 8],
+                ids=["auto", "mma", "tcgen05", "decode", "fused", "decode1k", "decodecp", "tcgen05single",
+                     "fusedsingle"])
 def proj_kernel(request, lib):
     prev = lib.set_proj_kernel(request.param)
     yield request.param
@@ -151,7 +152,7 @@ EDGE_CASES = {
 }
 
 
-@pytest.fixture(params=[0, 4], ids=["auto", "fused"])
+@pytest.fixture(params=[0, 4, 8], ids=["auto", "fused", "fusedsingle"])
 def auto_or_fused(request, lib):
     prev = lib.set_proj_kernel(request.param)
     yield request.param
@@ -306,7 +307,7 @@ def test_projection_kernels_agree(lib):
                                 H=4096, D=512, coff=2, ratio=4, block_size=128, rotate=False))
     res = run_inputs(inp)
     outs = {}
-    for k in (1, 2, 3, 4, 5, 6, 7):
+    for k in (1, 2, 3, 4, 5, 6, 7, 8):
         prev = lib.set_proj_kernel(k)
         try:
             o, kv, sc, err = run(lib, inp)
