@@ -10,7 +10,7 @@
 // of the same channels ("compressor torch_extension API", 计算公式 1:
 // [kv, score] = X [W^KV, W^Gate]). So TMEM lane i holds channel i's kv
 // (columns 0..255) and score (columns 256..511) for all 256 positions, and one
-// thread owns one channel of every window in a 128-position half of the tile.
+// thread owns one channel of every window in a 64-position quarter of the tile.
 //
 // The epilogue, per channel and window (计算公式 2-5), adds ape[q mod ratio] to
 // the score, takes positions before start_pos from the paged state (only the
@@ -22,14 +22,16 @@
 // weighted by their exp-sums). The tail rows a later call reads
 // (p >= (e/ratio - coff + 1)*ratio) go to the paged fp32 state from here.
 //
-// Roles (320 threads, one CTA per SM, persistent): warp 0 TMA (3 stages of
-// 16 + 16 + 32 KB), warp 1 TMEM owner and MMA issuer (M=128, N=256, K=16, two
-// per k-step), warps 2-9 epilogue: two warps per TMEM lane quarter, one for
-// each 128-position half of the tile (a window never straddles the halves, as
-// ratio divides 128), so the accumulator is drained in half the time and the
-// next item's MMAs start sooner. All waits are bounded: a role that gives up
-// raises the CTA's abort flag and the device error word, and all roles then
-// leave their loops, so the kernel always ends.
+// Roles (576 threads, one CTA per SM, persistent): warp 0 TMA (3 stages of
+// 16 + 16 + 32 KB; CTA pairs: 4 of 16 + 16 + 16 KB), warp 1 TMEM owner and MMA
+// issuer (M=128, N=256, K=16, two per k-step; pairs: M=256 over both CTAs),
+// warps 2-17 epilogue: four warps per TMEM lane quarter, one for each
+// 64-position quarter of the tile (a ratio-128 window spans two quarters, whose
+// warps merge their softmax stats through shared memory), so the accumulator —
+// all 512 TMEM columns, which the next item's MMAs must wait for — drains with
+// four independent chains of TMEM loads per lane quarter. All waits are
+// bounded: a role that gives up raises the CTA's abort flag and the device
+// error word, and all roles then leave their loops, so the kernel always ends.
 //
 // Folded mode (no rotation, B <= kMetaSeqs, tile counters available): the call
 // is this one kernel.
@@ -61,8 +63,8 @@ using namespace sm100;
 constexpr int NTOK = 256;   // positions per tile (MMA N)
 constexpr int BM = 128;     // channels per item (MMA M per CTA)
 constexpr int BK = 64;
-constexpr int kThreads = 320;
-constexpr int kEpiThreads = 256;  // warps 2-9
+constexpr int kThreads = 576;
+constexpr int kEpiThreads = 512;  // warps 2-17
 constexpr int kMetaSeqs = 512;    // folded mode: sequences whose metadata fits in shared memory
 
 // Single CTAs: 3 stages of 16 + 16 + 32 KB (the whole 256-position x tile).
@@ -98,6 +100,11 @@ struct SmemT {
   int bad;
   int fin[2];
   int nfin;
+  // ratio 128: running softmax stats of the first 64 positions of each window,
+  // per TMEM lane quarter and lane, handed to the warp that ends the window
+  float part_m[2][4][32];
+  float part_l[2][4][32];
+  float part_a[2][4][32];
 };
 
 // Per-sequence metadata: in shared memory (folded mode) or in the workspace
@@ -118,7 +125,7 @@ __device__ __forceinline__ int upper_index_plain(const int32_t* a, int n, int v)
   return lo;
 }
 
-__device__ __forceinline__ void epi_bar() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
+__device__ __forceinline__ void epi_bar() { asm volatile("bar.sync 1, 512;" ::: "memory"); }
 
 __device__ __forceinline__ float4 ldcg4(const float* p) { return __ldcg(reinterpret_cast<const float4*>(p)); }
 
@@ -234,16 +241,27 @@ __device__ __forceinline__ Item decode_item(const Params& p, const Meta& md, int
   return it;
 }
 
+// Where the first 64 positions of a ratio-128 window leave their running
+// softmax stats for the warp that ends the window (one slot per window of the
+// tile, TMEM lane quarter and lane).
+struct Parts {
+  float* m;  // [2][4][32]
+  float* l;
+  float* a;
+};
+
 // The epilogue of one item for ratio R in {32, 64, 128} (a window spans 2, 4
-// or 8 sub-chunks of 16 positions): the sub-chunks of one 128-position half
-// (hp) of the tile, with an online softmax per window. The 16 ape values a sub-chunk
-// adds to its scores are loaded one sub-chunk ahead (the first ones before the
-// accumulator is ready), so their L2 latency overlaps the TMEM loads and the
-// previous sub-chunk's math instead of stalling each step while the MMA waits
-// for TMEM.
+// or 8 sub-chunks of 16 positions): the four sub-chunks of one 64-position
+// quarter (qt) of the tile, with an online softmax per window; a ratio-128
+// window spans two quarters, and the warp of its second quarter merges the
+// first quarter's stats (after a barrier of all epilogue warps). The 16 ape
+// values a sub-chunk adds to its scores are loaded one sub-chunk ahead (the
+// first ones before the accumulator is ready), so their L2 latency overlaps the
+// TMEM loads and the previous sub-chunk's math instead of stalling each step
+// while the MMA waits for TMEM.
 template <int R, int D, class Wait>
 __device__ __forceinline__ bool pool_item_wide(const Params& p, const Meta& md, const Item& it, uint32_t taddr,
-                                               int ch, int hp, Wait&& wait_acc) {
+                                               int ch, int qt, int quad, const Parts& parts, Wait&& wait_acc) {
   static_assert(R == 32 || R == 64 || R == 128, "windows of 2, 4 or 8 sub-chunks");
   constexpr int C = D;  // coff = 1: the state / ape rows are D wide
   const int b = it.b;
@@ -261,12 +279,12 @@ __device__ __forceinline__ bool pool_item_wide(const Params& p, const Meta& md, 
   const float* ape_col = p.ape + col;
   float apn[16];
 #pragma unroll
-  for (int j = 0; j < 16; ++j) apn[j] = __ldg(ape_col + ((hp * 128) % R + j) * C);
+  for (int j = 0; j < 16; ++j) apn[j] = __ldg(ape_col + ((qt * 64) % R + j) * C);
   if (!wait_acc()) return false;
   float m = -INFINITY, l = 0.f, acc = 0.f;
 
 #pragma unroll 1
-  for (int u = hp * 8; u < hp * 8 + 8; ++u) {
+  for (int u = qt * 4; u < qt * 4 + 4; ++u) {
     const int q0 = it.P0 + u * 16;
     if (q0 >= e) break;  // the rest of the tile lies past the sequence
     uint32_t kr[16], sr[16];
@@ -275,7 +293,7 @@ __device__ __forceinline__ bool pool_item_wide(const Params& p, const Meta& md, 
     float apc[16];
 #pragma unroll
     for (int j = 0; j < 16; ++j) apc[j] = apn[j];
-    if (u + 1 < hp * 8 + 8) {
+    if (u + 1 < qt * 4 + 4) {
       const float* ap_next = ape_col + ((16 * (u + 1)) % R) * C;
 #pragma unroll
       for (int j = 0; j < 16; ++j) apn[j] = __ldg(ap_next + j * C);
@@ -330,7 +348,7 @@ __device__ __forceinline__ bool pool_item_wide(const Params& p, const Meta& md, 
       l = fmaf(l, sc, l2[0] + l2[1]);
       acc = fmaf(acc, sc, a2[0] + a2[1]);
       m = mn;
-      if (((u + 1) * 16) % R == 0) {  // last sub-chunk of the window
+      if (R < 128 && ((u + 1) * 16) % R == 0) {  // last sub-chunk of the window
         const int64_t n = off + (w - w0);
         ybase[n * p.D] = acc / l;
         m = -INFINITY;
@@ -339,19 +357,41 @@ __device__ __forceinline__ bool pool_item_wide(const Params& p, const Meta& md, 
       }
     }
   }
+  if constexpr (R == 128) {  // window qt / 2 of the tile: quarters 2 wi and 2 wi + 1
+    const int wi = qt >> 1;
+    const int slot = (wi * 4 + quad) * 32 + (threadIdx.x & 31);
+    if ((qt & 1) == 0) {
+      parts.m[slot] = m;
+      parts.l[slot] = l;
+      parts.a[slot] = acc;
+    }
+    epi_bar();
+    const int w = (it.P0 + wi * 128) / R;
+    if ((qt & 1) && w < w_end) {
+      const float m1 = parts.m[slot], l1 = parts.l[slot], a1 = parts.a[slot];
+      const float mn = fmaxf(m1, m);
+      const float f1 = m1 == -INFINITY ? 0.f : __expf(m1 - mn);
+      const float f2 = m == -INFINITY ? 0.f : __expf(m - mn);
+      const float lt = fmaf(l1, f1, l * f2);
+      const float at = fmaf(a1, f1, acc * f2);
+      const int64_t n = off + (w - w0);
+      ybase[n * p.D] = at / lt;
+    }
+    epi_bar();  // the slots are free for the next item
+  }
   return true;
 }
 
-// The epilogue of one item for ratio R <= 16 (whole windows inside a chunk of
-// 32 positions): the chunks of one 128-position half (hp) of the tile. The R
-// ape rows are loaded before the accumulator is ready. `wait_acc` waits for
-// the accumulator (false: give up).
+// The epilogue of one item for ratio R <= 16 (whole windows inside a sub-chunk
+// of 16 positions): the four sub-chunks of one 64-position quarter (qt) of the tile.
+// The R ape rows are loaded before the accumulator is ready. `wait_acc` waits
+// for the accumulator (false: give up).
 template <int R, class Wait>
 __device__ __forceinline__ bool pool_item(const Params& p, const Meta& md, const Item& it, uint32_t taddr,
-                                          int ch, int hp, Wait&& wait_acc) {
+                                          int ch, int qt, int quad, const Parts& parts, Wait&& wait_acc) {
   if constexpr (R >= 32) {
-    if (p.D == 128) return pool_item_wide<R, 128>(p, md, it, taddr, ch, hp, wait_acc);
-    return pool_item_wide<R, 512>(p, md, it, taddr, ch, hp, wait_acc);
+    if (p.D == 128) return pool_item_wide<R, 128>(p, md, it, taddr, ch, qt, quad, parts, wait_acc);
+    return pool_item_wide<R, 512>(p, md, it, taddr, ch, qt, quad, parts, wait_acc);
   } else {
   constexpr int COFF = (R == 4) ? 2 : 1;
   const int b = it.b;
@@ -372,23 +412,22 @@ __device__ __forceinline__ bool pool_item(const Params& p, const Meta& md, const
   if (!wait_acc()) return false;
 
 #pragma unroll 1
-  for (int c = hp * 4; c < hp * 4 + 4; ++c) {
-    const int q0 = it.P0 + c * 32;
+  for (int c = qt * 4; c < qt * 4 + 4; ++c) {
+    const int q0 = it.P0 + c * 16;
     if (q0 >= e) break;  // the rest of the tile lies past the sequence
-    uint32_t kr[32], sr[32];
-    tmem_ld32(taddr + c * 32, kr);
-    tmem_ld32(taddr + NTOK + c * 32, sr);
-    tmem_ld_wait(kr);
-    tmem_ld_wait(sr);
-    float kv[32], z[32];
+    uint32_t kr[16], sr[16];
+    tmem_ld16(taddr + c * 16, kr);
+    tmem_ld16(taddr + NTOK + c * 16, sr);
+    tmem_ld_wait16(kr, sr);
+    float kv[16], z[16];
 #pragma unroll
-    for (int j = 0; j < 32; ++j) {
+    for (int j = 0; j < 16; ++j) {
       kv[j] = __uint_as_float(kr[j]);
       z[j] = __uint_as_float(sr[j]) + ap[j % R];
     }
     if (q0 < s) {  // rows written by earlier calls (the first window of the sequence)
 #pragma unroll
-      for (int j = 0; j < 32; ++j) {
+      for (int j = 0; j < 16; ++j) {
         const int q = q0 + j;
         if (q < s) {
           const int rk = table_row(p, p.kv_tbl, b, q);
@@ -398,9 +437,9 @@ __device__ __forceinline__ bool pool_item(const Params& p, const Meta& md, const
         }
       }
     }
-    if (q0 + 31 >= thr) {  // tail rows: kv and score + ape into the paged state
+    if (q0 + 15 >= thr) {  // tail rows: kv and score + ape into the paged state
 #pragma unroll
-      for (int j = 0; j < 32; ++j) {
+      for (int j = 0; j < 16; ++j) {
         const int q = q0 + j;
         if (q >= thr && q < e) {
           const int rk = table_row(p, p.kv_tbl, b, q);
@@ -412,7 +451,7 @@ __device__ __forceinline__ bool pool_item(const Params& p, const Meta& md, const
     }
     {
 #pragma unroll
-      for (int k = 0; k < 32 / R; ++k) {  // whole windows inside the chunk
+      for (int k = 0; k < 16 / R; ++k) {  // whole windows inside the sub-chunk
         const int w = (q0 + k * R) / R;
         if (w < w_end) {
           float mx = z[k * R];
@@ -464,73 +503,69 @@ __device__ __forceinline__ void finish_window(const Params& p, int b, int w, int
   uint2 wraw[NG];  // norm_weight of the lane's channels
 #pragma unroll
   for (int i = 0; i < NG; ++i) wraw[i] = *reinterpret_cast<const uint2*>(p.norm_w + i * 128 + lane * 4);
-  float4 yb[NG], lb[NG], ya[NG], la[NG];
+  // per group of 128 channels: the pooled halves (coff = 2: and the previous
+  // window's half 0), merged right away so that only one group's loads are
+  // live at a time
   const bool prev_row = COFF == 2 && !first;
-#pragma unroll
-  for (int i = 0; i < NG; ++i) {
-    const int c = i * 128 + lane * 4;
-    if (COFF == 1) {
-      yb[i] = ldcg4(p.ystat + n * D + c);
-    } else {
-      yb[i] = ldcg4(p.ystat + (n * 2 + 1) * D + c);
-      lb[i] = ldcg4(p.ylse + (n * 2 + 1) * D + c);
-      if (prev_row) {
-        ya[i] = ldcg4(p.ystat + (n - 1) * 2 * D + c);
-        la[i] = ldcg4(p.ylse + (n - 1) * 2 * D + c);
-      } else {
-        ya[i] = make_float4(0.f, 0.f, 0.f, 0.f);
-        la[i] = make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
-      }
-    }
-  }
-  if (COFF == 2 && first && w > 0) {  // window w - 1 from the paged state (rare: once per sequence)
-#pragma unroll
-    for (int i = 0; i < NG; ++i) {
-      const int c = i * 128 + lane * 4;
-      float m[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY}, l[4] = {0.f, 0.f, 0.f, 0.f},
-            a[4] = {0.f, 0.f, 0.f, 0.f};
-      for (int jj = 0; jj < p.ratio; ++jj) {
-        const int q = (w - 1) * p.ratio + jj;
-        const int rk = table_row(p, p.kv_tbl, b, q);
-        const int rs = table_row(p, p.sc_tbl, b, q);
-        if (rk < 0 || rs < 0) continue;
-        const float4 kv = __ldcg(reinterpret_cast<const float4*>(
-            p.kv_state + ((int64_t)rk * p.bs + q % p.bs) * p.C + c));
-        const float4 sc = __ldcg(reinterpret_cast<const float4*>(
-            p.score_state + ((int64_t)rs * p.bs + q % p.bs) * p.C + c));
-        const float kk[4] = {kv.x, kv.y, kv.z, kv.w}, zz[4] = {sc.x, sc.y, sc.z, sc.w};
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const float mn = fmaxf(m[u], zz[u]);
-          const float f = __expf(m[u] - mn), pz = __expf(zz[u] - mn);
-          l[u] = l[u] * f + pz;
-          a[u] = a[u] * f + pz * kk[u];
-          m[u] = mn;
-        }
-      }
-      float yv[4] = {0.f, 0.f, 0.f, 0.f}, lv[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-#pragma unroll
-      for (int u = 0; u < 4; ++u)
-        if (l[u] > 0.f) {
-          yv[u] = a[u] / l[u];
-          lv[u] = m[u] + __logf(l[u]);
-        }
-      ya[i] = make_float4(yv[0], yv[1], yv[2], yv[3]);
-      la[i] = make_float4(lv[0], lv[1], lv[2], lv[3]);
-    }
-  }
   float y[NG][4];
   float ss = 0.f;
 #pragma unroll
   for (int i = 0; i < NG; ++i) {
-    const float ybv[4] = {yb[i].x, yb[i].y, yb[i].z, yb[i].w};
+    const int c = i * 128 + lane * 4;
+    float4 yb, lb, ya, la;
+    if (COFF == 1) {
+      yb = ldcg4(p.ystat + n * D + c);
+    } else {
+      yb = ldcg4(p.ystat + (n * 2 + 1) * D + c);
+      lb = ldcg4(p.ylse + (n * 2 + 1) * D + c);
+      if (prev_row) {
+        ya = ldcg4(p.ystat + (n - 1) * 2 * D + c);
+        la = ldcg4(p.ylse + (n - 1) * 2 * D + c);
+      } else {
+        ya = make_float4(0.f, 0.f, 0.f, 0.f);
+        la = make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
+      }
+      if (first && w > 0) {  // window w - 1 from the paged state (rare: once per sequence)
+        float m[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY}, l[4] = {0.f, 0.f, 0.f, 0.f},
+              a[4] = {0.f, 0.f, 0.f, 0.f};
+        for (int jj = 0; jj < p.ratio; ++jj) {
+          const int q = (w - 1) * p.ratio + jj;
+          const int rk = table_row(p, p.kv_tbl, b, q);
+          const int rs = table_row(p, p.sc_tbl, b, q);
+          if (rk < 0 || rs < 0) continue;
+          const float4 kv = __ldcg(reinterpret_cast<const float4*>(
+              p.kv_state + ((int64_t)rk * p.bs + q % p.bs) * p.C + c));
+          const float4 sc = __ldcg(reinterpret_cast<const float4*>(
+              p.score_state + ((int64_t)rs * p.bs + q % p.bs) * p.C + c));
+          const float kk[4] = {kv.x, kv.y, kv.z, kv.w}, zz[4] = {sc.x, sc.y, sc.z, sc.w};
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const float mn = fmaxf(m[u], zz[u]);
+            const float f = __expf(m[u] - mn), pz = __expf(zz[u] - mn);
+            l[u] = l[u] * f + pz;
+            a[u] = a[u] * f + pz * kk[u];
+            m[u] = mn;
+          }
+        }
+        float yv[4] = {0.f, 0.f, 0.f, 0.f}, lv[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+          if (l[u] > 0.f) {
+            yv[u] = a[u] / l[u];
+            lv[u] = m[u] + __logf(l[u]);
+          }
+        ya = make_float4(yv[0], yv[1], yv[2], yv[3]);
+        la = make_float4(lv[0], lv[1], lv[2], lv[3]);
+      }
+    }
+    const float ybv[4] = {yb.x, yb.y, yb.z, yb.w};
     if (COFF == 1) {
 #pragma unroll
       for (int u = 0; u < 4; ++u) y[i][u] = ybv[u];
     } else {
-      const float lbv[4] = {lb[i].x, lb[i].y, lb[i].z, lb[i].w};
-      const float yav[4] = {ya[i].x, ya[i].y, ya[i].z, ya[i].w};
-      const float lav[4] = {la[i].x, la[i].y, la[i].z, la[i].w};
+      const float lbv[4] = {lb.x, lb.y, lb.z, lb.w};
+      const float yav[4] = {ya.x, ya.y, ya.z, ya.w};
+      const float lav[4] = {la.x, la.y, la.z, la.w};
 #pragma unroll
       for (int u = 0; u < 4; ++u) {
         const float M = fmaxf(lav[u], lbv[u]);
@@ -573,7 +608,7 @@ __device__ __forceinline__ void finish_window(const Params& p, int b, int w, int
 }
 
 // Folded mode: the output rows of work tile t (its windows), one per warp of
-// the eight epilogue warps at a time.
+// the sixteen epilogue warps at a time.
 template <int NG, int COFF>
 __device__ void finish_tile_t(const Params& p, const Meta& md, int t, int ew, int lane) {
   const int b = upper_index_plain(md.tile, p.B, t);
@@ -601,7 +636,7 @@ __device__ void finish_tile(const Params& p, const Meta& md, int t, int ew, int 
 
 // Folded mode: zero the output rows that hold no window (each sequence's
 // reserved rows past its completed windows, and the rows after the last
-// sequence's), sequences spread over the CTAs; eight warps, 16 bytes a lane.
+// sequence's), sequences spread over the CTAs; sixteen warps, 16 bytes a lane.
 __device__ void zero_rows(const Params& p, const Meta& md, int ew, int lane) {
   const int D = p.D;
   const int per_row = D * 2 / 16;  // uint4 per row
@@ -739,10 +774,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
   } else {
-    const int ew = warp - 2;                 // 0..7
-    const int e_tid = threadIdx.x - 64;      // 0..255
+    const int ew = warp - 2;                 // 0..15
+    const int e_tid = threadIdx.x - 64;      // 0..511
     const int quad = warp & 3;               // TMEM lanes this warp may access
-    const int hp = ew >> 2;                  // 128-position half of the tile
+    const int qt = ew >> 2;                  // 64-position quarter of the tile
+    const Parts parts{&sm.part_m[0][0][0], &sm.part_l[0][0][0], &sm.part_a[0][0][0]};
     const int row = quad * 32 + lane;
     const uint32_t taddr = tmem + ((uint32_t)(quad * 32) << 16);
     if constexpr (FOLD) {
@@ -755,21 +791,21 @@ __global__ void __launch_bounds__(kThreads, 1)
       const Item it = decode_item(p, md, g, n_cblk);
       auto wait_acc = [&]() {
         const bool ok = mbar_wait(&sm.acc_full, acc_phase, abort);
-        if (!bar_and(1, kEpiThreads, ok)) return false;  // all eight warps leave together
+        if (!bar_and(1, kEpiThreads, ok)) return false;  // all epilogue warps leave together
         tc_fence_after();
         return true;
       };
       const int ch = it.c0 + row;
       bool ok;
       switch (p.ratio) {
-        case 1: ok = pool_item<1>(p, md, it, taddr, ch, hp, wait_acc); break;
-        case 2: ok = pool_item<2>(p, md, it, taddr, ch, hp, wait_acc); break;
-        case 4: ok = pool_item<4>(p, md, it, taddr, ch, hp, wait_acc); break;
-        case 8: ok = pool_item<8>(p, md, it, taddr, ch, hp, wait_acc); break;
-        case 16: ok = pool_item<16>(p, md, it, taddr, ch, hp, wait_acc); break;
-        case 32: ok = pool_item<32>(p, md, it, taddr, ch, hp, wait_acc); break;
-        case 64: ok = pool_item<64>(p, md, it, taddr, ch, hp, wait_acc); break;
-        default: ok = pool_item<128>(p, md, it, taddr, ch, hp, wait_acc); break;
+        case 1: ok = pool_item<1>(p, md, it, taddr, ch, qt, quad, parts, wait_acc); break;
+        case 2: ok = pool_item<2>(p, md, it, taddr, ch, qt, quad, parts, wait_acc); break;
+        case 4: ok = pool_item<4>(p, md, it, taddr, ch, qt, quad, parts, wait_acc); break;
+        case 8: ok = pool_item<8>(p, md, it, taddr, ch, qt, quad, parts, wait_acc); break;
+        case 16: ok = pool_item<16>(p, md, it, taddr, ch, qt, quad, parts, wait_acc); break;
+        case 32: ok = pool_item<32>(p, md, it, taddr, ch, qt, quad, parts, wait_acc); break;
+        case 64: ok = pool_item<64>(p, md, it, taddr, ch, qt, quad, parts, wait_acc); break;
+        default: ok = pool_item<128>(p, md, it, taddr, ch, qt, quad, parts, wait_acc); break;
       }
       if (!ok) break;
       tc_fence_before();
