@@ -957,9 +957,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       int stage = 0;
       uint32_t phase = 0;
+      Armed armed;
       for (int st = 0; st < nsteps; ++st) {
         if (!mbar_wait(&sm.empty[stage], phase ^ 1u, abort)) break;
         mbar_arrive_expect_tx(&sm.full[stage], bytes);
+        armed.note(stage, phase);
         // K blocks cb, cb+1: clusters start at different steps, the four CTAs of
         // a cluster take adjacent chunks
         const int cb = (((st + g) % nsteps) * KQ + (int)q) * KPS;
@@ -967,6 +969,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tma_load_3d(sm.x[stage], &map_x, &sm.full[stage], 0, 0, cb);
         if (++stage == STAGES) { stage = 0; phase ^= 1u; }
       }
+      drain_armed(sm.full, STAGES, armed);  // no copy still landing when the CTA leaves
     }
   } else if (warp == 7) {
     // ---- MMA (M = 64): every A row of the stage in one accumulator ----

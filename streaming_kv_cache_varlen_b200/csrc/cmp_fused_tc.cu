@@ -713,6 +713,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       int stage = 0;
       uint32_t phase = 0;
+      Armed armed;
       for (int u = unit0; u < n_units && !*abort; u += ustep) {
         const int g = PAIR ? 2 * u + (int)rank : u;
         const Item it = decode_item(p, md, g, n_cblk);
@@ -721,13 +722,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int kb = 0; kb < k_blocks; ++kb) {
           if (!mbar_wait(&sm.empty[stage], phase ^ 1u, abort)) break;
           if constexpr (PAIR) {
-            if (rank == 0) mbar_arrive_expect_tx(&sm.full[stage], 2 * C::kStageBytes);
+            if (rank == 0) {
+              mbar_arrive_expect_tx(&sm.full[stage], 2 * C::kStageBytes);
+              armed.note(stage, phase);
+            }
             const uint32_t fb = full0 + 8u * stage;
             tma_load_2d_pair(sm.a_kv[stage], &map_wkv, fb, kb * BK, wrow);
             tma_load_2d_pair(sm.a_g[stage], &map_wg, fb, kb * BK, wrow);
             tma_load_2d_pair(sm.b[stage], &map_x, fb, kb * BK, xrow);
           } else {
             mbar_arrive_expect_tx(&sm.full[stage], C::kStageBytes);
+            armed.note(stage, phase);
             tma_load_2d(sm.a_kv[stage], &map_wkv, &sm.full[stage], kb * BK, wrow);
             tma_load_2d(sm.a_g[stage], &map_wg, &sm.full[stage], kb * BK, wrow);
             tma_load_2d(sm.b[stage], &map_x, &sm.full[stage], kb * BK, xrow);
@@ -735,6 +740,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (++stage == STAGES) { stage = 0; phase ^= 1u; }
         }
       }
+      drain_armed(sm.full, STAGES, armed);  // no copy still landing when the CTA leaves
     }
   } else if (warp == 1) {
     if (lane == 0 && rank == 0) {

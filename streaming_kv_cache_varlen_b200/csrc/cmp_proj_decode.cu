@@ -123,13 +123,16 @@ __global__ void __launch_bounds__(kThreads)
   if (warp == 0 && lane == 0) {
     int stage = 0;
     uint32_t phase = 0;
+    Armed armed;
     for (int kb = kb_lo; kb < kb_hi; ++kb) {
       if (!mbar_wait(&sm.empty[stage], phase ^ 1u, abort)) break;
       mbar_arrive_expect_tx(&sm.full[stage], BM * BK * 2 + x_bytes);
+      armed.note(stage, phase);
       tma_load_2d(sm.w[stage], wmap, &sm.full[stage], kb * BK, wrow);
       tma_load_2d(sm.x[stage], &map_x, &sm.full[stage], kb * BK, 0);
       if (++stage == STAGES) { stage = 0; phase ^= 1u; }
     }
+    drain_armed(sm.full, STAGES, armed);  // no copy still landing when the CTA leaves
   } else if (warp == 1 && lane == 0) {
     int stage = 0;
     uint32_t phase = 0;

@@ -190,6 +190,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       int stage = 0;
       uint32_t phase = 0;
+      Armed armed;
       for (int tile = blockIdx.x; tile < n_tiles && !*abort; tile += gridDim.x) {
         const int m0 = (tile % n_m) * BM;
         const int n0 = (tile / n_m) * bn;
@@ -198,12 +199,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int kb = 0; kb < k_blocks; ++kb) {
           if (!mbar_wait(&sm.empty[stage], phase ^ 1u, abort)) break;
           mbar_arrive_expect_tx(&sm.full[stage], sbytes);
+          armed.note(stage, phase);
           unsigned char* st = ring + (size_t)stage * sbytes;
           tma_load_2d(st, wmap, &sm.full[stage], kb * BK, wrow);
           tma_load_2d(st + kStageBytesA, &map_x, &sm.full[stage], kb * BK, n0);
           if (++stage == stages) { stage = 0; phase ^= 1u; }
         }
       }
+      drain_armed(sm.full, stages, armed);  // no copy still landing when the CTA leaves
     }
   } else if (warp == 1) {
     // ---------------- MMA issuer ----------------
@@ -335,6 +338,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       int stage = 0;
       uint32_t phase = 0;
+      Armed armed;
       for (int tile = pair; tile < n_tiles && !*abort; tile += n_pairs) {
         const int m0 = (tile % n_m) * BMP + (int)rank * BM;
         const int n0 = (tile / n_m) * bn + (int)rank * (bn / 2);
@@ -342,13 +346,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int wrow = m0 < p.C ? m0 : m0 - p.C;
         for (int kb = 0; kb < k_blocks; ++kb) {
           if (!mbar_wait(&sm.empty[stage], phase ^ 1u, abort)) break;
-          if (rank == 0) mbar_arrive_expect_tx(&sm.full[stage], 2 * sbytes);
+          if (rank == 0) {
+            mbar_arrive_expect_tx(&sm.full[stage], 2 * sbytes);
+            armed.note(stage, phase);
+          }
           unsigned char* st = ring + (size_t)stage * sbytes;
           tma_load_2d_pair(st, wmap, full0 + 8u * stage, kb * BK, wrow);
           tma_load_2d_pair(st + kStageBytesA, &map_x, full0 + 8u * stage, kb * BK, n0);
           if (++stage == stages) { stage = 0; phase ^= 1u; }
         }
       }
+      drain_armed(sm.full, stages, armed);  // the pair's copies (counted here on the even CTA)
     }
   } else if (warp == 1) {
     // ---------------- MMA issuer (even CTA) ----------------

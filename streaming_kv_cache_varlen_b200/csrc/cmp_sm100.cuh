@@ -83,6 +83,34 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
   }
 }
 
+// A TMA producer's record of the stages it armed: bit s of mask = stage s was
+// armed at least once, bit s of par = the parity of its last armed phase.
+struct Armed {
+  uint32_t mask = 0u, par = 0u;
+  __device__ __forceinline__ void note(int s, uint32_t phase) {
+    mask |= 1u << s;
+    par = (par & ~(1u << s)) | ((phase & 1u) << s);
+  }
+};
+
+// The producer thread, before its CTA leaves: wait (at most ~limit_ns in all)
+// until the last armed phase of every stage has completed, so that no copy it
+// issued is still writing into shared memory when the CTA exits (after a role
+// gave up, stages may be in flight that nobody consumes). In a normal run every
+// armed phase has completed and been consumed, and this returns at once.
+__device__ __forceinline__ bool drain_armed(uint64_t* full, int stages, const Armed& a,
+                                            uint64_t limit_ns = 20000000ull) {
+  const uint64_t t0 = globaltimer();
+  for (int s = 0; s < stages; ++s) {
+    if (!((a.mask >> s) & 1u)) continue;
+    const uint32_t bar = smem_u32(&full[s]);
+    const uint32_t par = (a.par >> s) & 1u;
+    while (!mbar_try_wait(bar, par))
+      if (globaltimer() - t0 > limit_ns) return false;
+  }
+  return true;
+}
+
 // ---- TMA -----------------------------------------------------------------------
 
 __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, uint64_t* bar, int x,
