@@ -130,7 +130,8 @@ struct Smem {
   alignas(16) float4 hst[kMaxOut][OWN];          // per window and channel: the state rows' running
                                                  // max, exp-sum and weighted sum
   float norm[OWN];
-  alignas(16) float hcolT[OWN][512];  // rotation: this CTA's columns of the hadamard matrix (column-major)
+  alignas(16) float hcolT[OWN][520];  // rotation: this CTA's columns of the hadamard matrix (column-major;
+                                      // rows padded by 8 floats onto different banks)
   TokInfo tok[MAXT];
   Win win[kMaxOut];
   int32_t cu[kMaxSeqs + 1];
@@ -805,20 +806,36 @@ __device__ void exchange_sums(const Params& p, Smem<MAXT>& sm, const CpArgs& a, 
   if (p.rotate) asm volatile("bar.arrive 5, 128;" ::: "memory");
   if (got) {
     const int per_lane = (int)gridDim.x / 32;  // 1 or 4 partials per lane and window
-    for (int i0 = 0; i0 < nw; i0 += 8) {
-      float v[8][4];
+    if (per_lane == 1) {  // 32 CTAs: 16 windows' partials in flight per lane at once
+      for (int i0 = 0; i0 < nw; i0 += 16) {
+        float v[16];
 #pragma unroll
-      for (int u = 0; u < 8; ++u)
+        for (int u = 0; u < 16; ++u)
+          v[u] = i0 + u < nw ? __ldcg(a.sums + (int64_t)(i0 + u) * kMaxCtas + lane) : 0.f;
 #pragma unroll
-        for (int k = 0; k < 4; ++k)
-          v[u][k] = (i0 + u < nw && k < per_lane) ? __ldcg(a.sums + (int64_t)(i0 + u) * kMaxCtas + lane + 32 * k)
-                                                 : 0.f;
+        for (int u = 0; u < 16; ++u) {
+          float t = v[u];
 #pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        float t = ((v[u][0] + v[u][1]) + v[u][2]) + v[u][3];
+          for (int o = 16; o > 0; o >>= 1) t += __shfl_xor_sync(0xffffffffu, t, o);
+          if (lane == 0 && i0 + u < nw) sm.ss_tot[i0 + u] = t;
+        }
+      }
+    } else {
+      for (int i0 = 0; i0 < nw; i0 += 8) {
+        float v[8][4];
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) t += __shfl_xor_sync(0xffffffffu, t, o);
-        if (lane == 0 && i0 + u < nw) sm.ss_tot[i0 + u] = t;
+        for (int u = 0; u < 8; ++u)
+#pragma unroll
+          for (int k = 0; k < 4; ++k)
+            v[u][k] = (i0 + u < nw && k < per_lane) ? __ldcg(a.sums + (int64_t)(i0 + u) * kMaxCtas + lane + 32 * k)
+                                                   : 0.f;
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          float t = ((v[u][0] + v[u][1]) + v[u][2]) + v[u][3];
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1) t += __shfl_xor_sync(0xffffffffu, t, o);
+          if (lane == 0 && i0 + u < nw) sm.ss_tot[i0 + u] = t;
+        }
       }
     }
   }
@@ -828,7 +845,7 @@ __device__ void exchange_sums(const Params& p, Smem<MAXT>& sm, const CpArgs& a, 
 
 // Rotation, warps 1-3 (96 threads) once every CTA has arrived: every window's
 // u (all D channels, published with the arrivals) into the now idle A ring,
-// rows of D + 4 floats (16-byte aligned, rows on different banks), 8 loads in
+// rows of D + 8 floats (16-byte aligned, rows on different banks), 8 loads in
 // flight per thread.
 template <int MAXT>
 __device__ void load_u_rows(const Params& p, Smem<MAXT>& sm, const CpArgs& a) {
@@ -849,16 +866,16 @@ __device__ void load_u_rows(const Params& p, Smem<MAXT>& sm, const CpArgs& a) {
 #pragma unroll
     for (int e = 0; e < 8; ++e) {
       const int v = v0 + t + 96 * e;
-      if (v < n4) *reinterpret_cast<float4*>(uall + (v / per_row) * (p.D + 4) + 4 * (v % per_row)) = x4[e];
+      if (v < n4) *reinterpret_cast<float4*>(uall + (v / per_row) * (p.D + 8) + 4 * (v % per_row)) = x4[e];
     }
   }
 }
 
 // Warps 0-3: RMSNorm scale, norm_weight, RoPE and the bf16 store of this CTA's
 // channels of every window row; with the rotation, output column ch0 + c of a
-// window is scale * sum_k u[k] * hadamard[k][ch0 + c], one thread per (window,
-// column) adding over k in order (four interleaved partial sums, four k per
-// step from 16-byte shared-memory loads).
+// window is scale * sum_k u[k] * hadamard[k][ch0 + c], one thread (two, for up
+// to 64 pairs, taking alternate groups of four k) per (window, column), four
+// interleaved partial sums from 16-byte shared-memory loads.
 template <int MAXT>
 __device__ void finish_rows(const Params& p, Smem<MAXT>& sm, const CpArgs& a, int ch0, bool ok) {
   const int tid = threadIdx.x;
@@ -866,14 +883,18 @@ __device__ void finish_rows(const Params& p, Smem<MAXT>& sm, const CpArgs& a, in
   const bool fin = ok && sm.xch_ok != 0;
   if (p.rotate) {
     const float* uall = reinterpret_cast<const float*>(&sm.a[0][0]);
-    for (int u = tid; u < nw * OWN; u += 128) {
-      const int i = u / OWN, c = u % OWN;
+    // up to 64 (window, column) pairs: two adjacent lanes per pair, one taking
+    // the even and one the odd groups of 4 channels, combined by a shuffle
+    const int split = nw * OWN <= 64 ? 2 : 1;
+    for (int u = tid; u < nw * OWN * split; u += 128) {
+      const int pr = u / split, part = u % split;
+      const int i = pr / OWN, c = pr % OWN;
       float o = 0.f;
       if (fin) {
-        const float* ui = uall + i * (p.D + 4);
-        const float* hc = sm.hcolT[c];
+        const float* ui = uall + i * (p.D + 8) + 4 * part;
+        const float* hc = sm.hcolT[c] + 4 * part;
         float s4[4] = {0.f, 0.f, 0.f, 0.f};
-        for (int k = 0; k < p.D; k += 4) {
+        for (int k = 0; k < p.D; k += 4 * split) {
           const float4 uv = *reinterpret_cast<const float4*>(ui + k);
           const float4 hv = *reinterpret_cast<const float4*>(hc + k);
           s4[0] = fmaf(uv.x, hv.x, s4[0]);
@@ -881,9 +902,13 @@ __device__ void finish_rows(const Params& p, Smem<MAXT>& sm, const CpArgs& a, in
           s4[2] = fmaf(uv.z, hv.z, s4[2]);
           s4[3] = fmaf(uv.w, hv.w, s4[3]);
         }
-        o = ((s4[0] + s4[1]) + (s4[2] + s4[3])) * rsqrtf(sm.ss_tot[i] / (float)p.D + 1e-6f);
+        o = (s4[0] + s4[1]) + (s4[2] + s4[3]);
       }
-      p.out[(int64_t)sm.wlist[i] * p.D + ch0 + c] = __float2bfloat16_rn(o);
+      if (split == 2) o += __shfl_xor_sync(__activemask(), o, 1);  // the pair's lanes are both active
+      if (part == 0) {
+        if (fin) o *= rsqrtf(sm.ss_tot[i] / (float)p.D + 1e-6f);
+        p.out[(int64_t)sm.wlist[i] * p.D + ch0 + c] = __float2bfloat16_rn(o);
+      }
     }
     CP_STAMP(tid == 0, 10);  // rows stored
     return;
@@ -1138,8 +1163,8 @@ int max_clusters(int (&conf)[64]) {
 
 bool decode_cp_supported(const Params& p) {
   if (p.T < 1 || p.T > 64 || p.B > kMaxSeqs || p.n_out > kMaxOut || p.rope != 64) return false;
-  // rotation: every window's u (n_out rows of D + 4 floats) fits in the A ring
-  if (p.rotate && (size_t)p.n_out * (p.D + 4) * 4 > sizeof(Smem<32>::a)) return false;
+  // rotation: every window's u (n_out rows of D + 8 floats) fits in the A ring
+  if (p.rotate && (size_t)p.n_out * (p.D + 8) * 4 > sizeof(Smem<32>::a)) return false;
   if (p.coff * p.ratio > kMaxWinRows || p.H % (KQ * KPS * BK) || p.D % GCH || kMaxClusters % (p.D / GCH) ||
       encode_fn() == nullptr)
     return false;
