@@ -284,7 +284,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 // less data per MMA and holds 6-8 stages, so more of the load latency is hidden.
 // Both CTAs' loads count on the even CTA's stage barrier; the MMA commits
 // arrive on the stage and accumulator barriers of both CTAs; both epilogues
-// report a drained accumulator to the even CTA. No TMA multicast.
+// report a drained accumulator to the even CTA. Every copy lands in the issuing CTA's own shared memory.
 constexpr int BMP = 256;  // weight rows per pair tile (MMA M over the pair)
 
 __host__ __device__ constexpr uint32_t stage_bytes_pair(int bn) {

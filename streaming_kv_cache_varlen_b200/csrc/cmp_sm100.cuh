@@ -272,7 +272,7 @@ __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
 // TMA tile load into this CTA's shared memory whose completion (bytes) is
 // counted on an mbarrier of either CTA of the pair (its shared::cluster
 // address): the loads of both CTAs feed the even CTA's barrier, on which the
-// pair's MMA issuer waits. No multicast.
+// pair's MMA issuer waits. The copy lands in the issuing CTA's own shared memory only.
 __device__ __forceinline__ void tma_load_2d_pair(void* dst, const CUtensorMap* map, uint32_t bar_cluster, int x,
                                                  int y) {
   asm volatile(
