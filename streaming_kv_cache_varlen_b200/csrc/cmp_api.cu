@@ -22,7 +22,7 @@ cudaError_t launch_decode_fused(const Params& p, float* part, void* bar, cudaStr
 bool decode_cp_supported(const Params& p);
 cudaError_t launch_decode_cp(const Params& p, void* counter, void* xch, void* u, cudaStream_t s,
                              bool unreachable);
-cudaError_t launch_nsa(const NsaParams& p, cudaStream_t s);
+cudaError_t launch_nsa(const NsaParams& p, cudaStream_t s, int sm_count);
 cudaError_t launch_nsa_scan(const NsaParams& p, cudaStream_t s);
 int noalloc_take_error(int dev, unsigned* word);
 void noalloc_forget_addresses();
@@ -507,7 +507,8 @@ int cmp_nsa_compress(const void* input, const void* weight, const int32_t* slot_
   p.result_len = d.result_len;
   if (!paged && launch(CMP_KERNEL_NSA_SCAN, s, [&] { return cmp::launch_nsa_scan(p, s); }) != cudaSuccess)
     return CMP_ERR_CUDA;
-  if (launch(CMP_KERNEL_NSA, s, [&] { return cmp::launch_nsa(p, s); }) != cudaSuccess) return CMP_ERR_CUDA;
+  if (launch(CMP_KERNEL_NSA, s, [&] { return cmp::launch_nsa(p, s, sm_count_cached()); }) != cudaSuccess)
+    return CMP_ERR_CUDA;
   return CMP_OK;
 }
 

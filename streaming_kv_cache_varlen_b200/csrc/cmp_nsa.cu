@@ -14,6 +14,11 @@
 // map over the cache [rows, N, D], a few large copies per CTA instead of one
 // per token and chunk (per-copy overhead in the copy engine, not DRAM, limited
 // the version with small copies).
+//
+// A CTA holds its whole window in shared memory (all runs in flight at once)
+// unless that would leave part of the grid for a second wave: then it cycles
+// its runs through a ring of fewer buffers, so that every CTA is resident from
+// the start and the GPU's whole shared memory streams the windows.
 #include "cmp_internal.cuh"
 #include "cmp_sm100.cuh"
 
@@ -25,7 +30,11 @@ namespace {
 
 constexpr int kThreads = 128;
 constexpr int kRun = 16;                 // cache rows per TMA box
+constexpr int kMaxRuns = 64 / kRun;      // compress_block_size <= 64
 constexpr int kTargetBytes = 32 << 10;   // window bytes per CTA the head group aims at
+constexpr int kCtasPerSm = 16;           // resident CTAs of kThreads (2048 threads; __launch_bounds__)
+constexpr int64_t kSmemPerSm = 228 << 10;  // shared memory of one SM
+constexpr int64_t kSmemPerCta = 1 << 10;   // reserved by the system for every resident CTA
 
 template <bool BF16>
 __device__ __forceinline__ float to_f32(uint16_t v) {
@@ -42,16 +51,43 @@ __device__ __forceinline__ uint32_t pack(float lo, float hi) {
   return *reinterpret_cast<const uint32_t*>(&h);
 }
 
+// Adds tokens [j0, j1) of the window to a thread's 4 sums: element e (of head
+// group-relative head hh) of token j is at w[(j - j0) * per_tok + e].
+template <bool BF16>
+__device__ __forceinline__ void add_tokens(const uint16_t* w, const float* wsm, int j0, int j1, int per_tok,
+                                           int nh, int e, int hh, float (&a)[4]) {
+  for (int j = j0; j < j1; ++j) {
+    const uint2 v = *reinterpret_cast<const uint2*>(w + (size_t)(j - j0) * per_tok + e);
+    const float wt = wsm[j * nh + hh];
+    a[0] = fmaf(to_f32<BF16>((uint16_t)(v.x & 0xFFFFu)), wt, a[0]);
+    a[1] = fmaf(to_f32<BF16>((uint16_t)(v.x >> 16)), wt, a[1]);
+    a[2] = fmaf(to_f32<BF16>((uint16_t)(v.y & 0xFFFFu)), wt, a[2]);
+    a[3] = fmaf(to_f32<BF16>((uint16_t)(v.y >> 16)), wt, a[3]);
+  }
+}
+
+template <bool BF16>
+__device__ __forceinline__ void store4(uint16_t* dst, const float (&a)[4]) {
+  uint2 o;
+  o.x = pack<BF16>(a[0], a[1]);
+  o.y = pack<BF16>(a[2], a[3]);
+  *reinterpret_cast<uint2*>(dst) = o;
+}
+
 // Warp 0 validates the batch's slot and the cache rows of its window, then lane
-// 0 issues the window's cbs / 16 boxes (heads h0 .. h0 + nh - 1; heads past N
-// read as zeros and are not stored), all completing on one mbarrier; the other
-// threads stage the weights meanwhile. Then each thread sums 4 consecutive
-// elements of one head over the window's tokens in order and stores them.
+// 0 issues the first nbuf of the window's cbs / 16 boxes (heads h0 .. h0 + nh -
+// 1; heads past N read as zeros and are not stored), box k on mbarrier k; the
+// other threads stage the weights meanwhile. Then each thread sums 4
+// consecutive elements of one head over the window's tokens in order and
+// stores them. nbuf = cbs / 16: the whole window is resident. nbuf < cbs / 16
+// (the host chooses it only when nh * D <= 4 * kThreads, one element group per
+// thread): box r lands in buffer r mod nbuf; once every thread has added it,
+// thread 0 issues box r + nbuf into the same buffer.
 // Packed layout (a programmatic dependent of nsa_scan_kernel): only lane 0 waits
 // for the scan, and every thread's stores come after it through __syncthreads.
 template <bool BF16>
-__global__ void __launch_bounds__(kThreads)
-    nsa_kernel(const __grid_constant__ CUtensorMap map, NsaParams p, int nh, int page_shift) {
+__global__ void __launch_bounds__(kThreads, kCtasPerSm)
+    nsa_kernel(const __grid_constant__ CUtensorMap map, NsaParams p, int nh, int page_shift, int nbuf) {
   const int b = blockIdx.y;
   const int h0 = blockIdx.x * nh;
   const int lane = threadIdx.x & 31;
@@ -69,13 +105,14 @@ __global__ void __launch_bounds__(kThreads)
   // TMA destinations start on 128-byte boundaries (the runs are multiples of 512 B)
   uint16_t* buf = reinterpret_cast<uint16_t*>(smem_raw + ((128u - (sm100::smem_u32(smem_raw) & 127u)) & 127u));
   const int per_tok = nh * p.D;
-  float* wsm = reinterpret_cast<float*>(buf + (size_t)p.cbs * per_tok);  // [cbs][nh]
-  __shared__ __align__(8) uint64_t full;
+  const int runs = p.cbs / kRun;
+  const uint32_t run_bytes = (uint32_t)(kRun * per_tok * 2);
+  float* wsm = reinterpret_cast<float*>(buf + (size_t)nbuf * kRun * per_tok);  // [cbs][nh]
+  __shared__ __align__(8) uint64_t full[kMaxRuns];
   __shared__ int ok;
+  int64_t row[kMaxRuns];  // first cache row of each box (thread 0 issues them all)
   if (threadIdx.x < 32) {  // warp 0: validation; lane 0 issues the copies
     const int64_t first = s - p.cbs;
-    const int runs = p.cbs / kRun;
-    int64_t row[64 / kRun];
     bool good = slot >= 0 && slot < p.result_len;
     if (p.packed) {
       if (lane == 0) {
@@ -105,11 +142,12 @@ __global__ void __launch_bounds__(kThreads)
       ok = good ? 1 : 0;
       if (good) {
         sm100::prefetch_tmap(&map);
-        sm100::mbar_init(&full, 1);
+        for (int k = 0; k < nbuf; ++k) sm100::mbar_init(&full[k], 1);
         sm100::fence_barrier_init();
-        sm100::mbar_arrive_expect_tx(&full, (uint32_t)(p.cbs * per_tok * 2));
-        for (int k = 0; k < runs; ++k)
-          sm100::tma_load_3d(buf + (size_t)k * kRun * per_tok, &map, &full, 0, h0, (int)row[k]);
+        for (int k = 0; k < nbuf; ++k) {
+          sm100::mbar_arrive_expect_tx(&full[k], run_bytes);
+          sm100::tma_load_3d(buf + (size_t)k * kRun * per_tok, &map, &full[k], 0, h0, (int)row[k]);
+        }
       }
     }
   }
@@ -120,28 +158,40 @@ __global__ void __launch_bounds__(kThreads)
   __syncthreads();
   if (!ok) return;
   int never = 0;
-  if (!sm100::mbar_wait(&full, 0, &never)) {
-    if (threadIdx.x == 0) atomicOr(p.err, kErrTimeout);
-    return;
-  }
   const int live = (p.N - h0 < nh ? p.N - h0 : nh) * p.D;  // elements of heads < N
   uint16_t* dst = p.out + (int64_t)__ldg(p.slot + b) * p.N * p.D + (int64_t)h0 * p.D;
-  for (int e = threadIdx.x * 4; e < live; e += kThreads * 4) {
-    const int hh = e / p.D;
-    float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
-    for (int j = 0; j < p.cbs; ++j) {
-      const uint2 v = *reinterpret_cast<const uint2*>(buf + (size_t)j * per_tok + e);
-      const float w = wsm[j * nh + hh];
-      a0 = fmaf(to_f32<BF16>((uint16_t)(v.x & 0xFFFFu)), w, a0);
-      a1 = fmaf(to_f32<BF16>((uint16_t)(v.x >> 16)), w, a1);
-      a2 = fmaf(to_f32<BF16>((uint16_t)(v.y & 0xFFFFu)), w, a2);
-      a3 = fmaf(to_f32<BF16>((uint16_t)(v.y >> 16)), w, a3);
+  if (nbuf == runs) {  // the whole window is resident
+    for (int k = 0; k < runs; ++k) {
+      if (!sm100::mbar_wait(&full[k], 0, &never)) {
+        if (threadIdx.x == 0) atomicOr(p.err, kErrTimeout);
+        return;
+      }
     }
-    uint2 o;
-    o.x = pack<BF16>(a0, a1);
-    o.y = pack<BF16>(a2, a3);
-    *reinterpret_cast<uint2*>(dst + e) = o;
+    for (int e = threadIdx.x * 4; e < live; e += kThreads * 4) {
+      float a[4] = {0.f, 0.f, 0.f, 0.f};
+      add_tokens<BF16>(buf, wsm, 0, p.cbs, per_tok, nh, e, e / p.D, a);
+      store4<BF16>(dst + e, a);
+    }
+    return;
   }
+  const int e = threadIdx.x * 4;  // live <= 4 * kThreads here
+  const bool mine = e < live;
+  float a[4] = {0.f, 0.f, 0.f, 0.f};
+  for (int r = 0; r < runs; ++r) {
+    const int k = r % nbuf;
+    const bool landed = sm100::mbar_wait(&full[k], (uint32_t)(r / nbuf) & 1u, &never);
+    if (landed && mine) add_tokens<BF16>(buf + (size_t)k * kRun * per_tok, wsm, r * kRun, r * kRun + kRun, per_tok,
+                                         nh, e, e / p.D, a);
+    if (__syncthreads_or(!landed)) {  // buffer k is free again, unless a wait gave up
+      if (threadIdx.x == 0) atomicOr(p.err, kErrTimeout);
+      return;
+    }
+    if (threadIdx.x == 0 && r + nbuf < runs) {
+      sm100::mbar_arrive_expect_tx(&full[k], run_bytes);
+      sm100::tma_load_3d(buf + (size_t)k * kRun * per_tok, &map, &full[k], 0, h0, (int)row[r + nbuf]);
+    }
+  }
+  if (mine) store4<BF16>(dst + e, a);
 }
 
 // Packed layout: the first row of every batch, starts[b] = sum of the lengths of
@@ -227,28 +277,52 @@ bool make_cache_map(CUtensorMap* m, const NsaParams& p, int64_t rows, int nh) {
 }
 
 int g_nsa_conf[2][64] = {{0}, {0}};
+int g_nsa_carve[2][64] = {{0}, {0}};
 
 }  // namespace
 
-cudaError_t launch_nsa(const NsaParams& p, cudaStream_t s) {
+cudaError_t launch_nsa(const NsaParams& p, cudaStream_t s, int sm_count) {
   const int head_bytes = p.cbs * p.D * 2;  // one head of the window
   int nh = kTargetBytes / head_bytes;
   nh = nh < 1 ? 1 : (nh > p.N ? p.N : nh);
   CUtensorMap map;
   if (!make_cache_map(&map, p, p.packed ? p.tokens : p.tokens * p.pbs, nh)) return cudaErrorNotSupported;
   const int page_shift = p.packed ? 0 : (p.pbs == 64 ? 6 : 7);
-  const size_t smem = 128 + (size_t)p.cbs * nh * p.D * 2 + (size_t)p.cbs * nh * 4;  // + alignment slack
+  const dim3 grid((unsigned)((p.N + nh - 1) / nh), (unsigned)p.B);
+  // Buffers of 16 cache rows per CTA: all cbs / 16 of them, unless the grid's
+  // whole windows do not fit on the GPU at once while a ring of fewer would
+  // (then the largest such ring: one wave, every CTA resident from the start).
+  const int runs = p.cbs / kRun;
+  const int64_t run_smem = (int64_t)kRun * nh * p.D * 2;
+  auto cta_smem = [&](int nb) { return 128 + nb * run_smem + (int64_t)p.cbs * nh * 4; };  // + alignment slack
+  const int64_t sms = sm_count > 0 ? sm_count : 1;
+  const int64_t per_sm = ((int64_t)grid.x * grid.y + sms - 1) / sms;
+  auto one_wave = [&](int nb) { return per_sm * (cta_smem(nb) + kSmemPerCta) <= kSmemPerSm; };
+  int nbuf = runs;
+  if (runs > 1 && nh * p.D <= 4 * kThreads && per_sm <= kCtasPerSm && !one_wave(runs)) {
+    int nb = runs - 1;
+    while (nb >= 1 && !one_wave(nb)) --nb;
+    if (nb >= 1) nbuf = nb;
+  }
+  const size_t smem = (size_t)cta_smem(nbuf);
   // the attribute is raised once per device, to the largest size a call can
   // ask for (window bytes <= kTargetBytes unless one head is larger: cbs <= 64,
   // D <= 256 gives 32 KB)
   constexpr size_t kMaxSmem = (size_t)kTargetBytes + kTargetBytes / 2 + 64 * 64 * 4;
-  const dim3 grid((unsigned)((p.N + nh - 1) / nh), (unsigned)p.B);
   auto* kernel = p.bf16 ? nsa_kernel<true> : nsa_kernel<false>;
   cudaError_t e = smem_attr_once(kernel, kMaxSmem, g_nsa_conf[p.bf16 ? 1 : 0]);
+  int dev = 0;
+  if (e == cudaSuccess) e = cudaGetDevice(&dev);
+  if (e == cudaSuccess && dev < 64 && !g_nsa_carve[p.bf16 ? 1 : 0][dev]) {
+    // the most shared memory per SM: the residency counted above relies on it
+    e = cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                             (int)cudaSharedmemCarveoutMaxShared);
+    g_nsa_carve[p.bf16 ? 1 : 0][dev] = e == cudaSuccess;
+  }
   if (e != cudaSuccess) return e;
   if (p.packed)  // a programmatic dependent of nsa_scan_kernel
-    return launch_chained(kernel, grid, dim3(kThreads), smem, s, 1, map, p, nh, page_shift);
-  kernel<<<grid, kThreads, smem, s>>>(map, p, nh, page_shift);
+    return launch_chained(kernel, grid, dim3(kThreads), smem, s, 1, map, p, nh, page_shift, nbuf);
+  kernel<<<grid, kThreads, smem, s>>>(map, p, nh, page_shift, nbuf);
   return cudaGetLastError();
 }
 

@@ -91,6 +91,25 @@ def test_head_shapes(lib, N, D):
     check(lib, i)
 
 
+# Grids whose whole windows do not all fit in the GPU's shared memory at once
+# (on 148 SMs), so that the kernel cycles each window's 16-row boxes through a
+# ring of fewer buffers: 1536 CTAs with 2 boxes in 1 buffer (the NSA decode
+# step of the bench), 1200 CTAs with 4 boxes in 2 buffers, 1320 CTAs with 3
+# boxes in 2 buffers (box 2 reuses buffer 0 in its second phase).
+@pytest.mark.parametrize("B,N,D,cbs,stride,layout,dtype", [
+    (128, 24, 192, 32, 16, "paged", "bf16"),
+    (200, 24, 64, 64, 16, "paged", "fp16"),
+    (200, 24, 64, 64, 32, "TND", "bf16"),
+    (110, 24, 128, 48, 16, "paged", "bf16"),
+])
+def test_window_ring(lib, B, N, D, cbs, stride, layout, dtype):
+    i = make_nsa_inputs(name="ring", seed=B + cbs, B=B, N=N, D=D, compress_block_size=cbs,
+                        compress_stride=stride, page_block_size=128, dtype=dtype, layout=layout,
+                        max_seq_len=256, trigger_fraction=1.0)
+    ref, _ = check(lib, i)
+    assert ref.written.sum() == B
+
+
 def test_pages_example(lib):
     c = json.load(open(os.path.join(GOLDEN, "nsa_example_case.json")))
     import torch
