@@ -82,7 +82,9 @@ __device__ __forceinline__ void store4(uint16_t* dst, const float (&a)[4]) {
 // stores them. nbuf = cbs / 16: the whole window is resident. nbuf < cbs / 16
 // (the host chooses it only when nh * D <= 4 * kThreads, one element group per
 // thread): box r lands in buffer r mod nbuf; once every thread has added it,
-// thread 0 issues box r + nbuf into the same buffer.
+// thread 0 issues box r + nbuf into the same buffer. A wait that gives up (2 s)
+// raises kErrTimeout, and thread 0 waits at most 20 ms more for the boxes it
+// armed, so that no copy is still landing when the CTA leaves.
 // Packed layout (a programmatic dependent of nsa_scan_kernel): only lane 0 waits
 // for the scan, and every thread's stores come after it through __syncthreads.
 template <bool BF16>
@@ -111,6 +113,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
   __shared__ __align__(8) uint64_t full[kMaxRuns];
   __shared__ int ok;
   int64_t row[kMaxRuns];  // first cache row of each box (thread 0 issues them all)
+  sm100::Armed armed;     // thread 0: the last phase it armed on each buffer
   if (threadIdx.x < 32) {  // warp 0: validation; lane 0 issues the copies
     const int64_t first = s - p.cbs;
     bool good = slot >= 0 && slot < p.result_len;
@@ -147,6 +150,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
         for (int k = 0; k < nbuf; ++k) {
           sm100::mbar_arrive_expect_tx(&full[k], run_bytes);
           sm100::tma_load_3d(buf + (size_t)k * kRun * per_tok, &map, &full[k], 0, h0, (int)row[k]);
+          armed.note(k, 0);
         }
       }
     }
@@ -163,7 +167,10 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
   if (nbuf == runs) {  // the whole window is resident
     for (int k = 0; k < runs; ++k) {
       if (!sm100::mbar_wait(&full[k], 0, &never)) {
-        if (threadIdx.x == 0) atomicOr(p.err, kErrTimeout);
+        if (threadIdx.x == 0) {  // no copy may still be landing when the CTA leaves
+          atomicOr(p.err, kErrTimeout);
+          sm100::drain_armed(full, nbuf, armed);
+        }
         return;
       }
     }
@@ -183,12 +190,16 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     if (landed && mine) add_tokens<BF16>(buf + (size_t)k * kRun * per_tok, wsm, r * kRun, r * kRun + kRun, per_tok,
                                          nh, e, e / p.D, a);
     if (__syncthreads_or(!landed)) {  // buffer k is free again, unless a wait gave up
-      if (threadIdx.x == 0) atomicOr(p.err, kErrTimeout);
+      if (threadIdx.x == 0) {  // no copy may still be landing when the CTA leaves
+        atomicOr(p.err, kErrTimeout);
+        sm100::drain_armed(full, nbuf, armed);
+      }
       return;
     }
     if (threadIdx.x == 0 && r + nbuf < runs) {
       sm100::mbar_arrive_expect_tx(&full[k], run_bytes);
       sm100::tma_load_3d(buf + (size_t)k * kRun * per_tok, &map, &full[k], 0, h0, (int)row[r + nbuf]);
+      armed.note(k, (uint32_t)((r + nbuf) / nbuf));
     }
   }
   if (mine) store4<BF16>(dst + e, a);
